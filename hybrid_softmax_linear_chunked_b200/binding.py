@@ -1,0 +1,254 @@
+"""Thin ctypes binding of librehyat.so (C ABI in include/rehyat.h).
+
+Argument marshalling only: tensors are checked for device/dtype/shape/contiguity, outputs and
+workspaces are allocated with torch on the tensors' device, and every computation runs in the
+library's CUDA kernels.  There is no CPU fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "librehyat.so")
+
+REHYAT_F32 = 0
+REHYAT_BF16 = 1
+
+STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_SHAPE", -3: "ERR_DTYPE", -4: "ERR_WORKSPACE",
+          -5: "ERR_CUDA", -6: "ERR_TIMEOUT", -7: "ERR_ALIGN"}
+
+EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
+            "rehyat_forward_workspace_size", "rehyat_forward", "rehyat_forward_states",
+            "rehyat_forward_attend", "rehyat_chunk_workspace_size",
+            "rehyat_chunk_forward", "rehyat_chunk_states", "rehyat_sync_status"]
+
+
+class RehyatError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("D", ctypes.c_int), ("F", ctypes.c_int),
+                ("G", ctypes.c_int), ("P", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load librehyat.so (built in-tree by the package build step) and declare its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"librehyat.so is not built ({_LIB_PATH}); run the package build "
+                           "step (hybrid_softmax_linear_chunked_b200.build.build()) first")
+    L = ctypes.CDLL(_LIB_PATH)
+    c_int, c_void_p, c_size_t = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+    P = c_void_p
+    L.rehyat_last_error.restype = ctypes.c_char_p
+    L.rehyat_last_error.argtypes = []
+    L.rehyat_version.restype = c_int
+    L.rehyat_featmap.argtypes = [Dims, c_int, c_int, P, P, P, P, P]
+    L.rehyat_forward_workspace_size.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int,
+                                                ctypes.POINTER(c_size_t)]
+    L.rehyat_forward.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P, P, P,
+                                 P, c_size_t, P]
+    L.rehyat_forward_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P,
+                                        c_size_t, P]
+    L.rehyat_forward_attend.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P,
+                                        P, P, c_size_t, P]
+    L.rehyat_chunk_workspace_size.argtypes = [Dims, c_int, c_int, c_int, c_int,
+                                              ctypes.POINTER(c_size_t)]
+    L.rehyat_chunk_forward.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
+                                       P, P, P, P, P, c_size_t, P]
+    L.rehyat_chunk_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
+                                      P, c_size_t, P]
+    L.rehyat_sync_status.argtypes = [P]
+    for name in EXPORTED:
+        if name not in ("rehyat_last_error",):
+            getattr(L, name).restype = c_int
+    _lib = L
+    return L
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise RehyatError(status, load().rehyat_last_error().decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return REHYAT_BF16
+    if t.dtype == torch.float32:
+        return REHYAT_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dev(*ts: torch.Tensor) -> torch.device:
+    dev = ts[0].device
+    for t in ts:
+        if t is None:
+            continue
+        if t.device.type != "cuda" or t.device != dev:
+            raise ValueError("all tensors must be on the same CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    return dev
+
+
+def _weights(W: torch.Tensor, b: torch.Tensor | None):
+    if W.dtype != torch.float32 or (b is not None and b.dtype != torch.float32):
+        raise TypeError("feature-map weights and biases are fp32")
+    return W, b
+
+
+def dims_of(x: torch.Tensor, W: torch.Tensor, P: int) -> Dims:
+    """Dims from x [B,H,n,D] and W [H,G,F/G,D/G]."""
+    B, H, _, D = x.shape
+    Hw, G, Fg, _ = W.shape
+    if Hw != H:
+        raise ValueError("W has a different head count than x")
+    return Dims(B, H, D, G * Fg, G, P)
+
+
+def version() -> int:
+    return load().rehyat_version()
+
+
+def featmap(x: torch.Tensor, W: torch.Tensor, bias: torch.Tensor | None, P: int) -> torch.Tensor:
+    """phi(x) for x [B,H,n,D] -> [B,H,n,F] (same dtype as x)."""
+    L = load()
+    dev = _dev(x, W, bias)
+    _weights(W, bias)
+    d = dims_of(x, W, P)
+    phi = torch.empty(x.shape[0], x.shape[1], x.shape[2], d.F, dtype=x.dtype, device=dev)
+    _check(L.rehyat_featmap(d, _dtype_code(x), x.shape[2], _ptr(x), _ptr(W), _ptr(bias),
+                            _ptr(phi), _stream(dev)))
+    return phi
+
+
+def forward_workspace_size(d: Dims, dtype_code: int, T: int, L_: int, Tc: int, To: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().rehyat_forward_workspace_size(d, dtype_code, T, L_, Tc, To, ctypes.byref(n)))
+    return n.value
+
+
+def chunk_workspace_size(d: Dims, dtype_code: int, L_: int, chunk_frames: int, To: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().rehyat_chunk_workspace_size(d, dtype_code, L_, chunk_frames, To,
+                                              ctypes.byref(n)))
+    return n.value
+
+
+def _workspace(nbytes: int, dev: torch.device, workspace: torch.Tensor | None) -> torch.Tensor:
+    if workspace is not None and workspace.numel() >= nbytes:
+        return workspace
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+
+
+def forward(q, k, v, Wq, bq, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
+            out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """Hybrid attention over a whole sequence: q, k, v [B,H,T*frame_tokens,D] -> out."""
+    lib = load()
+    dev = _dev(q, k, v, Wq, bq, Wk, bk)
+    _weights(Wq, bq), _weights(Wk, bk)
+    d = dims_of(q, Wq, P)
+    N = q.shape[2]
+    if N % frame_tokens:
+        raise ValueError("sequence length is not a multiple of frame_tokens")
+    T = N // frame_tokens
+    code = _dtype_code(q)
+    ws = _workspace(forward_workspace_size(d, code, T, frame_tokens, Tc, To), dev, workspace)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.rehyat_forward(d, code, T, frame_tokens, Tc, To, _ptr(q), _ptr(k), _ptr(v),
+                              _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(out), _ptr(ws),
+                              ws.numel(), _stream(dev)))
+    return out
+
+
+def forward_states(k, v, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
+                   workspace: torch.Tensor, Wq: torch.Tensor | None = None) -> torch.Tensor:
+    """First phase of `forward`: fills `workspace` with the state every chunk reads."""
+    lib = load()
+    dev = _dev(k, v, Wk, bk, workspace)
+    d = dims_of(k, Wk, P)
+    T = k.shape[2] // frame_tokens
+    _check(lib.rehyat_forward_states(d, _dtype_code(k), T, frame_tokens, Tc, To, _ptr(k), _ptr(v),
+                                     _ptr(Wk), _ptr(bk), _ptr(workspace), workspace.numel(),
+                                     _stream(dev)))
+    return workspace
+
+
+def forward_attend(q, k, v, Wq, bq, *, P: int, frame_tokens: int, Tc: int, To: int,
+                   workspace: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
+    """Second phase of `forward`: the hybrid output from q, k, v and the workspace states."""
+    lib = load()
+    dev = _dev(q, k, v, Wq, bq, workspace, out)
+    d = dims_of(q, Wq, P)
+    T = q.shape[2] // frame_tokens
+    _check(lib.rehyat_forward_attend(d, _dtype_code(q), T, frame_tokens, Tc, To, _ptr(q), _ptr(k),
+                                     _ptr(v), _ptr(Wq), _ptr(bq), _ptr(out), _ptr(workspace),
+                                     workspace.numel(), _stream(dev)))
+    return out
+
+
+def chunk_states(k, v, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
+                 workspace: torch.Tensor | None = None):
+    """States each chunk of `forward` reads: S [B,H,C,F,D], Z [B,H,C,F] (fp32)."""
+    lib = load()
+    dev = _dev(k, v, Wk, bk)
+    d = dims_of(k, Wk, P)
+    N = k.shape[2]
+    T = N // frame_tokens
+    C = -(-T // Tc)
+    code = _dtype_code(k)
+    ws = _workspace(forward_workspace_size(d, code, T, frame_tokens, Tc, To), dev, workspace)
+    S = torch.empty(d.B, d.H, C, d.F, d.D, dtype=torch.float32, device=dev)
+    Z = torch.empty(d.B, d.H, C, d.F, dtype=torch.float32, device=dev)
+    _check(lib.rehyat_chunk_states(d, code, T, frame_tokens, Tc, To, _ptr(k), _ptr(v), _ptr(Wk),
+                                   _ptr(bk), _ptr(S), _ptr(Z), _ptr(ws), ws.numel(),
+                                   _stream(dev)))
+    return S, Z
+
+
+def chunk_forward(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, frame_tokens: int,
+                  frames_before: int, To: int, out: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None):
+    """One streaming step; S [B,H,F,D] and Z [B,H,F] (fp32) are updated in place."""
+    lib = load()
+    dev = _dev(q, k_win, v_win, Wq, bq, Wk, bk, S, Z)
+    d = dims_of(q, Wq, P)
+    chunk_frames = q.shape[2] // frame_tokens
+    code = _dtype_code(q)
+    ws = _workspace(chunk_workspace_size(d, code, frame_tokens, chunk_frames, To), dev, workspace)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.rehyat_chunk_forward(d, code, frame_tokens, frames_before, chunk_frames, To,
+                                    _ptr(q), _ptr(k_win), _ptr(v_win), _ptr(Wq), _ptr(bq),
+                                    _ptr(Wk), _ptr(bk), _ptr(S), _ptr(Z), _ptr(out), _ptr(ws),
+                                    ws.numel(), _stream(dev)))
+    return out
+
+
+def sync_status(device: torch.device | None = None) -> None:
+    """Synchronise the current stream and raise if a kernel reported a device-side failure."""
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    _check(load().rehyat_sync_status(_stream(dev)))

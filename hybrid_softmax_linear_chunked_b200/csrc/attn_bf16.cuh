@@ -1,0 +1,487 @@
+// Fused hybrid attention forward, bf16 in / bf16 out, tcgen05 tensor cores (sm_100a).
+//
+// One CTA owns two 128-row query tiles of one temporal chunk of one (batch, head) and streams
+// the chunk's softmax window (its own frames plus the To frames before it) through shared memory
+// in 128-key tiles.  Per key tile j and query tile t:
+//     S_t = Q_t K_j^T                          (tcgen05.mma, smem x smem -> TMEM fp32)
+//     P_t = exp2(S_t * log2(e)/sqrt(D) - m_t)  (softmax warpgroup t, P written back into TMEM
+//                                               over S_t as packed bf16 pairs)
+//     O_t += P_t V_j                           (tcgen05.mma, A from TMEM, V MN-major in smem)
+// with the running max m_t kept lazily: O_t and l_t are rescaled only when the tile max exceeds
+// m_t by more than 8 (a factor 256), so exp2 arguments stay <= 8.
+// Epilogue (the hybrid joint normaliser of the "ReHyAt overview" page §2.2.1 and the state
+// readout of §2.3): the softmax warpgroup overwrites its Q tile in shared memory with
+// phi_q(q) * 2^-m (bf16), one more MMA adds phi_q 2^-m . S_c into O_t, and
+// l_t += 2^-m phi_q . Z_c; the output is O_t / l_t.  m starts at 0 for chunks that have a
+// linear region, so 2^-m <= 1 and a row can never lose both terms to underflow.
+//
+// Warp roles (320 threads): warps 0-3 softmax/epilogue of tile 0, warps 4-7 of tile 1, warp 8
+// TMA producer (+ TMEM allocation), warp 9 MMA issuer.  TMEM columns: S_0 [0,128), S_1
+// [128,256), O_0 [256,384), O_1 [384,512).
+#pragma once
+
+#include "featmap.cuh"
+#include "sm100.cuh"
+
+namespace rehyat {
+namespace attn {
+
+using namespace sm100;
+
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+constexpr int kHD = 128;  // head dim D
+constexpr int kFD = 128;  // feature dim F
+constexpr int kThreads = 320;
+constexpr int kTileBytes = kBM * kHD * 2;  // one 128 x 128 bf16 tile
+
+// dynamic shared memory layout (offsets from the 1024-aligned base)
+constexpr uint32_t kOffQ0 = 0;
+constexpr uint32_t kOffQ1 = kOffQ0 + kTileBytes;
+constexpr uint32_t kOffK = kOffQ1 + kTileBytes;       // 2 stages
+constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;    // 2 stages
+constexpr int kMinG = 4;                             // smallest supported group count
+constexpr uint32_t kOffW = kOffV + 2 * kTileBytes;    // W_q of the head, fp32 (F * D / G)
+constexpr uint32_t kWBytesMax = kFD * kHD / kMinG * 4;
+constexpr uint32_t kOffB = kOffW + kWBytesMax;         // bias, F fp32
+constexpr uint32_t kOffZ = kOffB + kFD * 4;            // Z_c, F fp32
+constexpr uint32_t kSmemBytes = kOffZ + kFD * 4 + 1024;  // + alignment slack
+
+enum Bar {
+  kQFull = 0,
+  kKFull = 1,    // 2
+  kKEmpty = 3,   // 2
+  kVFull = 5,    // 2
+  kVEmpty = 7,   // 2
+  kSFull = 9,    // 2 (per query tile)
+  kPFull = 11,   // 2 (per query tile, 128 arrivals)
+  kOFull = 13,   // 2 (per query tile)
+  kStFull = 15,
+  kPhiFull = 16,  // 2 (per query tile, 128 arrivals)
+  kRoDone = 18,   // 2
+  kMmaDone = 20,
+  kNumBars = 21
+};
+
+struct Params {
+  int L;              // tokens per frame
+  int T;              // frames of the query sequence
+  int Tc, To;         // chunk length, overlap
+  int frames_before;  // video frame index of query row 0
+  int kv_frame0;      // video frame index of key/value row 0
+  int H, P;
+  int n_states;       // states per (b, h) in St / Z (state index = chunk index)
+  int nq_rows;        // rows per (b, h) of q and out
+  float scale_log2;   // log2(e) / sqrt(D)
+  const float* Wq;    // [H, G, F/G, D/G]
+  const float* bq;    // [H, F] or null
+  const float* Z;     // [BH, n_states, F]
+  __nv_bfloat16* out; // [BH, nq_rows, D]
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// K-major SW128 descriptor of the kk-th 16-wide K step of a 128-row, 128-wide bf16 tile.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_addr, int kk) {
+  return sdesc_sw128(tile_addr + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
+}
+// MN-major SW128 descriptor of the kk-th 16-row K step of a [128 rows][128 cols] bf16 tile
+// whose columns are the M/N dimension.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_addr, int kk) {
+  return sdesc_sw128(tile_addr + kk * 16 * 128, kBM * 128, 1024);
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    hybrid_attn_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
+                            const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV,
+                            const __grid_constant__ CUtensorMap tmSt, const Params p) {
+  constexpr int Dg = kHD / G, Fg = kFD / G;
+  static_assert(Dg == Fg, "in-place phi_q needs equal group widths");
+  static_assert(Dg % 8 == 0, "group width must be a multiple of 8");
+  static_assert(G >= kMinG && kFD * Dg * 4 <= kWBytesMax, "W_q does not fit its shared-memory slot");
+  static_assert(kSmemBytes <= 232448, "shared memory over the per-CTA limit");
+
+  // ---- chunk geometry (uniform over the CTA) ----
+  const int c = blockIdx.y, bh = blockIdx.z, h = bh % p.H;
+  const int gs = p.frames_before + c * p.Tc;
+  const int ge = min(gs + p.Tc, p.frames_before + p.T);
+  const int gw = max(0, gs - p.To);
+  const int q_row0 = (gs - p.frames_before) * p.L;
+  const int nq = (ge - gs) * p.L;
+  const int k_row0 = (gw - p.kv_frame0) * p.L;
+  const int nk = (ge - gw) * p.L;
+  const bool has_linear = gw > 0;
+  const int tile_row0 = blockIdx.x * 2 * kBM;
+  if (tile_row0 >= nq) return;
+  const bool has_t1 = tile_row0 + kBM < nq;
+  const int n_kv = (nk + kBN - 1) / kBN;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  __shared__ __align__(8) uint64_t bars[kNumBars];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  volatile int* abort_flag = &abort_sh;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float* sW = reinterpret_cast<float*>(sm + kOffW);
+  float* sB = reinterpret_cast<float*>(sm + kOffB);
+  float* sZ = reinterpret_cast<float*>(sm + kOffZ);
+
+  if (warp == 8) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i) {
+      const bool many = (i == kPFull || i == kPFull + 1 || i == kPhiFull || i == kPhiFull + 1);
+      mbar_init(&bars[i], many ? 128 : 1);
+    }
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (tid < 256 && has_linear) {
+    const float* Wh = p.Wq + (size_t)h * kFD * Dg;
+    for (int i = tid; i < kFD * Dg; i += 256) sW[i] = Wh[i];
+    for (int i = tid; i < kFD; i += 256) {
+      sB[i] = p.bq ? p.bq[(size_t)h * kFD + i] : 0.f;
+      sZ[i] = p.Z[((size_t)bh * p.n_states + c) * kFD + i];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  const uint32_t sQ0 = smem_u32(sm + kOffQ0), sQ1 = smem_u32(sm + kOffQ1);
+  const uint32_t sK0 = smem_u32(sm + kOffK), sK1 = sK0 + kTileBytes;
+  const uint32_t sV0 = smem_u32(sm + kOffV), sV1 = sV0 + kTileBytes;
+
+  if (warp == 8) {
+    // ================================ TMA producer ================================
+    // The whole warp runs the loop and waits; lane 0 issues the copies.
+    const bool leader = lane == 0;
+    if (leader) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bars[kQFull], has_t1 ? 2 * kTileBytes : kTileBytes);
+      for (int t = 0; t < (has_t1 ? 2 : 1); ++t) {
+        uint8_t* dst = sm + (t ? kOffQ1 : kOffQ0);
+        const int row = q_row0 + tile_row0 + t * kBM;
+        tma_load_3d(dst, &tmQ, &bars[kQFull], 0, row, bh);
+        tma_load_3d(dst + kBM * 128, &tmQ, &bars[kQFull], 64, row, bh);
+      }
+    }
+    __syncwarp();
+    int issued_k = 0, issued_v = 0;
+    bool st_issued = false;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      const int row = k_row0 + j * kBN;
+      if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty + s], ((j >> 1) - 1) & 1, abort_flag));
+      if (!ok) break;
+      if (leader) {
+        uint8_t* dk = sm + kOffK + s * kTileBytes;
+        mbar_arrive_expect_tx(&bars[kKFull + s], kTileBytes);
+        tma_load_3d(dk, &tmK, &bars[kKFull + s], 0, row, bh);
+        tma_load_3d(dk + kBM * 128, &tmK, &bars[kKFull + s], 64, row, bh);
+      }
+      __syncwarp();
+      ++issued_k;
+      if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kVEmpty + s], ((j >> 1) - 1) & 1, abort_flag));
+      if (!ok) break;
+      if (leader) {
+        uint8_t* dv = sm + kOffV + s * kTileBytes;
+        mbar_arrive_expect_tx(&bars[kVFull + s], kTileBytes);
+        tma_load_3d(dv, &tmV, &bars[kVFull + s], 0, row, bh);
+        tma_load_3d(dv + kBM * 128, &tmV, &bars[kVFull + s], 64, row, bh);
+      }
+      __syncwarp();
+      ++issued_v;
+    }
+    if (ok && has_linear) {
+      // S_c^T goes into the K stage that the (absent) tile n_kv would use.
+      const int s = n_kv & 1;
+      if (n_kv >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty + s], ((n_kv >> 1) - 1) & 1, abort_flag));
+      if (ok) {
+        if (leader) {
+          uint8_t* dst = sm + kOffK + s * kTileBytes;
+          mbar_arrive_expect_tx(&bars[kStFull], kTileBytes);
+          tma_load_3d(dst, &tmSt, &bars[kStFull], 0, 0, bh * p.n_states + c);
+          tma_load_3d(dst + kBM * 128, &tmSt, &bars[kStFull], 64, 0, bh * p.n_states + c);
+        }
+        __syncwarp();
+        st_issued = true;
+      }
+    }
+    if (!ok) {
+      // Abort: let every copy already issued land before the CTA can exit.
+      mbar_wait_drain(&bars[kQFull], 0);
+      for (int j = max(0, issued_k - 2); j < issued_k; ++j)
+        mbar_wait_drain(&bars[kKFull + (j & 1)], (j >> 1) & 1);
+      for (int j = max(0, issued_v - 2); j < issued_v; ++j)
+        mbar_wait_drain(&bars[kVFull + (j & 1)], (j >> 1) & 1);
+      if (st_issued) mbar_wait_drain(&bars[kStFull], 0);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ================================ MMA issuer ================================
+    // The whole warp runs the loop and waits; lane 0 issues the MMAs and commits.
+    const bool leader = lane == 0;
+    const uint32_t id_qk = idesc_bf16(kBM, kBN, false, false);
+    const uint32_t id_pv = idesc_bf16(kBM, kHD, false, true);
+    const int nt = has_t1 ? 2 : 1;
+    auto issue_s = [&](int t, int j) {
+      if (leader) {
+        const uint32_t d = tmem + t * 128;
+        const uint32_t qb = t ? sQ1 : sQ0;
+        const uint32_t kb = (j & 1) ? sK1 : sK0;
+        for (int kk = 0; kk < kHD / 16; ++kk)
+          mma_ss(d, kmajor_desc(qb, kk), kmajor_desc(kb, kk), id_qk, kk > 0 ? 1u : 0u);
+        mma_commit(&bars[kSFull + t]);
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int t, int j) {
+      if (leader) {
+        const uint32_t d = tmem + 256 + t * 128;
+        const uint32_t a = tmem + t * 128;
+        const uint32_t vb = (j & 1) ? sV1 : sV0;
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(d, a + kk * 8, mnmajor_desc(vb, kk), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[kOFull + t]);
+      }
+      __syncwarp();
+    };
+    auto commit = [&](int b) {
+      if (leader) mma_commit(&bars[b]);
+      __syncwarp();
+    };
+    auto wait = [&](int b, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, abort_flag));
+    };
+    bool ok = wait(kQFull, 0) && wait(kKFull, 0);
+    if (ok) {
+      tc_fence_after();
+      for (int t = 0; t < nt; ++t) issue_s(t, 0);
+      commit(kKEmpty);
+    }
+    for (int j = 1; j < n_kv && ok; ++j) {
+      const int s = j & 1, sp = (j - 1) & 1;
+      ok = wait(kKFull + s, (j >> 1) & 1) && wait(kVFull + sp, ((j - 1) >> 1) & 1);
+      for (int t = 0; t < nt && ok; ++t) {
+        ok = wait(kPFull + t, (j - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(t, j - 1);
+        issue_s(t, j);
+      }
+      if (!ok) break;
+      commit(kVEmpty + sp);
+      commit(kKEmpty + s);
+    }
+    if (ok) {
+      const int j = n_kv - 1;
+      ok = wait(kVFull + (j & 1), (j >> 1) & 1);
+      for (int t = 0; t < nt && ok; ++t) {
+        ok = wait(kPFull + t, j & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(t, j);
+      }
+      if (ok) commit(kVEmpty + (j & 1));
+    }
+    if (ok && has_linear) {
+      const uint32_t stb = (n_kv & 1) ? sK1 : sK0;
+      ok = wait(kStFull, 0);
+      for (int t = 0; t < nt && ok; ++t) {
+        ok = wait(kPhiFull + t, 0);
+        if (!ok) break;
+        tc_fence_after();
+        if (leader) {
+          const uint32_t d = tmem + 256 + t * 128;
+          const uint32_t qb = t ? sQ1 : sQ0;
+          for (int kk = 0; kk < kFD / 16; ++kk)
+            mma_ss(d, kmajor_desc(qb, kk), kmajor_desc(stb, kk), id_qk, 1u);
+          mma_commit(&bars[kRoDone + t]);
+        }
+        __syncwarp();
+      }
+    }
+    // Every tcgen05 op (and the mbarrier arrivals it triggers) must finish before teardown.
+    commit(kMmaDone);
+    mbar_wait_drain(&bars[kMmaDone], 0);
+    __syncwarp();
+  } else {
+    // ============================ softmax / epilogue warpgroups ============================
+    const int t = warp >> 2;          // query tile of this warpgroup
+    const int r = tid & 127;          // row within the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * 128;
+    const uint32_t tO = tmem + lane_base + 256 + t * 128;
+    const bool active = (t == 0) || has_t1;
+    if (active) {
+      const float sl2 = p.scale_log2;
+      float m = has_linear ? 0.f : -INFINITY;
+      float l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n_kv; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull + t], j & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        float s[kBN];
+#pragma unroll
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          uint32_t rr[32];
+          tmem_ld32(tS + cc * 32, rr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(rr[i]);
+        }
+        const int valid = nk - j * kBN;
+        if (valid < kBN) {
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
+            if (i >= valid) s[i] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, s[i]);
+        const float m_tile = mx * sl2;
+        const float m_new = (m_tile > m + 8.f) ? m_tile : m;
+        const bool rescale = (m_new != m) && (j > 0);
+        if (__any_sync(0xffffffffu, rescale)) {
+          const float fac = rescale ? ex2(m - m_new) : 1.f;
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + t], (j - 1) & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < kHD / 32; ++cc) {
+            uint32_t rr[32];
+            tmem_ld32(tO + cc * 32, rr);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * fac);
+            tmem_st32(tO + cc * 32, rr);
+          }
+          l *= fac;
+        }
+        m = m_new;
+        float rowsum = 0.f;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pr[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float a = ex2(fmaf(s[hh * 64 + 2 * i], sl2, -m));
+            const float b = ex2(fmaf(s[hh * 64 + 2 * i + 1], sl2, -m));
+            rowsum += a + b;
+            pr[i] = pack_bf16x2(a, b);
+          }
+          tmem_st32(tS + hh * 32, pr);
+        }
+        l += rowsum;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars[kPFull + t]);
+      }
+      // ---- epilogue ----
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + t], (n_kv - 1) & 1, abort_flag));
+      if (ok && has_linear) {
+        tc_fence_after();
+        // phi_q(q) * 2^-m overwrites this row of the Q tile (group g reads and writes the same
+        // 16-byte chunks, so reading a group's inputs first makes the update in place safe).
+        uint8_t* qrow = sm + (t ? kOffQ1 : kOffQ0);
+        const float esc = ex2(-m);
+        float lin = 0.f;
+#pragma unroll 1
+        for (int g = 0; g < G; ++g) {
+          float x[Dg];
+#pragma unroll
+          for (int c8 = 0; c8 < Dg / 8; ++c8) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + sw128_offset(r, g * Dg + c8 * 8, kBM));
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f2 = __bfloat1622float2(b2[e]);
+              x[c8 * 8 + 2 * e] = f2.x;
+              x[c8 * 8 + 2 * e + 1] = f2.y;
+            }
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < Fg / 8; ++c8) {
+            uint32_t packed[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float ph2[2];
+#pragma unroll
+              for (int q2 = 0; q2 < 2; ++q2) {
+                const int o = c8 * 8 + 2 * e + q2;
+                const int f = g * Fg + o;
+                const float* w = sW + (g * Fg + o) * Dg;
+                float u = sB[f];
+#pragma unroll
+                for (int i = 0; i < Dg; ++i) u = fmaf(w[i], x[i], u);
+                const float ph = int_pow(softplus_fast(u), part_power(f, kFD, p.P)) * esc;
+                const float phr = __bfloat162float(__float2bfloat16_rn(ph));
+                lin = fmaf(phr, sZ[f], lin);
+                ph2[q2] = ph;
+              }
+              packed[e] = pack_bf16x2(ph2[0], ph2[1]);
+            }
+            *reinterpret_cast<uint4*>(qrow + sw128_offset(r, g * Fg + c8 * 8, kBM)) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          }
+        }
+        fence_async_smem();
+        mbar_arrive(&bars[kPhiFull + t]);
+        l += lin;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kRoDone + t], 0, abort_flag));
+      }
+      if (ok) {
+        tc_fence_after();
+        const int row_in_chunk = tile_row0 + t * kBM + r;
+        const bool row_valid = row_in_chunk < nq;
+        const float inv = 1.f / l;
+        __nv_bfloat16* orow = p.out + ((size_t)bh * p.nq_rows + q_row0 + row_in_chunk) * kHD;
+#pragma unroll
+        for (int cc = 0; cc < kHD / 32; ++cc) {
+          uint32_t rr[32];
+          tmem_ld32(tO + cc * 32, rr);
+          if (row_valid) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint4 o4;
+              o4.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
+              o4.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
+              o4.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
+              o4.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
+              *reinterpret_cast<uint4*>(orow + cc * 32 + q4 * 8) = o4;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ---- teardown ----
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace attn
+}  // namespace rehyat

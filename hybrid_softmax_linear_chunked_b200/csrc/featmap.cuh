@@ -1,0 +1,103 @@
+// Feature map phi of the "ReHyAt overview" page §2.2.2: grouped 1x1 linear (G groups, group g
+// maps input dims [g*D/G, (g+1)*D/G) to features [g*F/G, (g+1)*F/G)), plus bias, split into P
+// contiguous parts (the first F mod P parts one longer, numpy.array_split order), part p
+// (1-based) raised to softplus(.)^p, concatenated back in order.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace rehyat {
+
+// Power applied to feature f when F features are split into P parts.
+__host__ __device__ __forceinline__ int part_power(int f, int F, int P) {
+  const int base = F / P, extra = F % P;
+  const int big = extra * (base + 1);
+  const int p = (f < big) ? f / (base + 1) : extra + (f - big) / base;
+  return p + 1;
+}
+
+__device__ __forceinline__ float int_pow(float x, int p) {
+  float r = x;
+  for (int i = 1; i < p; ++i) r *= x;
+  return r;
+}
+
+// softplus(u) = max(u, 0) + log1p(e^{-|u|}) with the CUDA math library's expf/log1pf.
+__device__ __forceinline__ float softplus_accurate(float u) {
+  return fmaxf(u, 0.f) + log1pf(expf(-fabsf(u)));
+}
+
+// Same function with the fast hardware exp/log.  log1p(y) for y = e^{-|u|} in (0, 1] uses the
+// first terms of its Taylor series y - y^2/2 + y^3/3 below y = 2^-7 (truncation < y^4/4, i.e.
+// relative 1.2e-7) and log(1 + y) above it, where 1 + y >= 1.0078 keeps rounding of the sum
+// below 1e-5 relative.  Accurate to well within bf16 rounding.
+__device__ __forceinline__ float softplus_fast(float u) {
+  const float y = __expf(-fabsf(u));
+  const float l = (y < 0.0078125f) ? y * (1.f - y * (0.5f - y * (1.f / 3.f))) : __logf(1.f + y);
+  return fmaxf(u, 0.f) + l;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Standalone feature map: x [BH, n, D] -> phi [BH, n, F].  One thread per token; the head's W
+// and bias are staged in shared memory (read as broadcasts).  The x row is staged through a
+// per-thread slice of shared memory loaded cooperatively (coalesced) so global traffic is one
+// read of x and one write of phi.
+//   grid (ceil(n / 128), BH), block 128, dynamic smem: W (G*F/G*D/G floats) + F floats bias +
+//   128 * (D + 1) floats of x staging.
+template <typename Tin, typename Tout, bool kAccurate>
+__global__ void __launch_bounds__(128) featmap_kernel(const Tin* __restrict__ x,
+                                                      const float* __restrict__ W,
+                                                      const float* __restrict__ bias,
+                                                      Tout* __restrict__ phi, int n, int H, int D,
+                                                      int F, int G, int P) {
+  extern __shared__ float fm_smem[];
+  const int Dg = D / G, Fg = F / G;
+  float* sW = fm_smem;                 // [G][Fg][Dg]
+  float* sB = sW + G * Fg * Dg;        // [F]
+  float* sX = sB + F;                  // [128][D + 1]
+  const int bh = blockIdx.y, h = bh % H;
+  const int row0 = blockIdx.x * 128;
+  const float* Wh = W + (size_t)h * G * Fg * Dg;
+  for (int i = threadIdx.x; i < G * Fg * Dg; i += 128) sW[i] = Wh[i];
+  for (int i = threadIdx.x; i < F; i += 128) sB[i] = bias ? bias[(size_t)h * F + i] : 0.f;
+  const Tin* xb = x + ((size_t)bh * n + row0) * D;
+  const int rows = min(128, n - row0);
+  for (int i = threadIdx.x; i < rows * D; i += 128) {
+    const int r = i / D, c = i - r * D;
+    sX[r * (D + 1) + c] = to_f32<Tin>(xb[i]);
+  }
+  __syncthreads();
+  const int r = threadIdx.x;
+  if (r >= rows) return;
+  const float* xr = sX + r * (D + 1);
+  Tout* out = phi + ((size_t)bh * n + row0 + r) * F;
+  for (int g = 0; g < G; ++g) {
+    for (int o = 0; o < Fg; ++o) {
+      const int f = g * Fg + o;
+      const float* w = sW + (g * Fg + o) * Dg;
+      float u = sB[f];
+      for (int i = 0; i < Dg; ++i) u = fmaf(w[i], xr[g * Dg + i], u);
+      const float sp = kAccurate ? softplus_accurate(u) : softplus_fast(u);
+      out[f] = from_f32<Tout>(int_pow(sp, part_power(f, F, P)));
+    }
+  }
+}
+
+}  // namespace rehyat

@@ -1,0 +1,585 @@
+// librehyat.so: host side of the C ABI declared in include/rehyat.h.  Argument checks, workspace
+// carving, TMA tensor-map encoding and kernel launches; every kernel of the library is compiled
+// in this one translation unit.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/rehyat.h"
+#include "attn_bf16.cuh"
+#include "featmap.cuh"
+#include "fp32_path.cuh"
+#include "sm100.cuh"
+#include "state_bf16.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_check(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(REHYAT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return REHYAT_OK;
+}
+
+#define RH_TRY(expr)                 \
+  do {                               \
+    int rh_status_ = (expr);         \
+    if (rh_status_ != REHYAT_OK) return rh_status_; \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int check_dims(const rehyat_dims& d, rehyat_dtype dt) {
+  if (d.B < 1 || d.H < 1 || d.D < 1 || d.F < 1 || d.G < 1 || d.P < 1)
+    return fail(REHYAT_ERR_ARG, "dims must be positive (B=%d H=%d D=%d F=%d G=%d P=%d)", d.B, d.H,
+                d.D, d.F, d.G, d.P);
+  if (d.D % d.G || d.F % d.G)
+    return fail(REHYAT_ERR_ARG, "G=%d must divide D=%d and F=%d", d.G, d.D, d.F);
+  if (d.P > d.F) return fail(REHYAT_ERR_ARG, "P=%d exceeds F=%d", d.P, d.F);
+  if (dt != REHYAT_F32 && dt != REHYAT_BF16) return fail(REHYAT_ERR_DTYPE, "unknown dtype %d", (int)dt);
+  return REHYAT_OK;
+}
+
+// Shapes the attention / state kernels support (the standalone feature map is more general).
+int check_path_shape(const rehyat_dims& d, rehyat_dtype dt) {
+  if (dt == REHYAT_BF16) {
+    if (d.D != 128 || d.F != 128)
+      return fail(REHYAT_ERR_SHAPE, "bf16 path needs D = F = 128 (got D=%d F=%d)", d.D, d.F);
+    if (d.G != 4 && d.G != 8 && d.G != 16)
+      return fail(REHYAT_ERR_SHAPE, "bf16 path supports G in {4, 8, 16} (got %d)", d.G);
+  } else {
+    if (d.D % 32 || d.D > rehyat::fp32::kMaxD || d.F > 256)
+      return fail(REHYAT_ERR_SHAPE, "fp32 path needs D %% 32 == 0, D <= 256, F <= 256 (D=%d F=%d)",
+                  d.D, d.F);
+  }
+  return REHYAT_OK;
+}
+
+int check_sched(int T, int L, int Tc, int To) {
+  if (T < 1 || L < 1) return fail(REHYAT_ERR_ARG, "need T >= 1 and frame_tokens >= 1 (T=%d L=%d)", T, L);
+  if (Tc < 1 || To < 0) return fail(REHYAT_ERR_ARG, "need Tc >= 1 and To >= 0 (Tc=%d To=%d)", Tc, To);
+  if ((long long)T * L > (1LL << 30)) return fail(REHYAT_ERR_ARG, "sequence too long");
+  return REHYAT_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// TMA tensor maps
+// ---------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encoder(EncodeTiledFn* out) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || !p || q != cudaDriverEntryPointSuccess)
+      return fail(REHYAT_ERR_CUDA, "cuTensorMapEncodeTiled not available");
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *out = fn;
+  return REHYAT_OK;
+}
+
+// bf16 [outer][rows][cols] tensor, loaded as 128-row x 64-column boxes with 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* base, int cols, long long rows, long long outer) {
+  EncodeTiledFn enc;
+  RH_TRY(get_encoder(&enc));
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * 2 * (cuuint64_t)rows};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(REHYAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return REHYAT_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Workspace plans
+// ---------------------------------------------------------------------------------------------
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    size_t o = off;
+    off = round_up(off + bytes, 256);
+    return o;
+  }
+};
+
+int fold_splits(int BH, int n_fold, long long rows_per_fold) {
+  if (n_fold <= 0) return 1;
+  const long long tiles = (rows_per_fold + 127) / 128;
+  long long want = (2LL * 148 + (long long)BH * n_fold - 1) / ((long long)BH * n_fold);
+  long long s = want < 1 ? 1 : want;
+  const long long max_s = tiles / 2 > 0 ? tiles / 2 : 1;
+  if (s > max_s) s = max_s;
+  if (s > 16) s = 16;
+  return (int)s;
+}
+
+struct ForwardPlan {
+  int C, n_fold, splits;
+  size_t dS, dZ, St, Zc, phiq, phik, Sc, total;
+};
+
+ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, int Tc, int To) {
+  ForwardPlan p{};
+  const size_t BH = (size_t)d.B * d.H;
+  p.C = (T + Tc - 1) / Tc;
+  p.n_fold = p.C - 1;
+  Carve cv;
+  if (dt == REHYAT_BF16) {
+    p.splits = fold_splits((int)BH, p.n_fold, (long long)Tc * L);
+    const size_t nf = p.n_fold > 0 ? p.n_fold : 0;
+    p.dS = cv.take(BH * nf * p.splits * d.F * d.D * 4);
+    p.dZ = cv.take(BH * nf * p.splits * d.F * 4);
+    p.St = cv.take(BH * p.C * d.D * d.F * 2);
+    p.Zc = cv.take(BH * p.C * d.F * 4);
+  } else {
+    p.splits = 1;
+    const size_t N = (size_t)T * L;
+    const size_t nf = p.n_fold > 0 ? p.n_fold : 0;
+    p.phiq = cv.take(BH * N * d.F * 4);
+    p.phik = cv.take(BH * N * d.F * 4);
+    p.dS = cv.take(BH * nf * d.F * d.D * 4);
+    p.dZ = cv.take(BH * nf * d.F * 4);
+    p.Sc = cv.take(BH * p.C * d.F * d.D * 4);
+    p.Zc = cv.take(BH * p.C * d.F * 4);
+  }
+  p.total = cv.off;
+  return p;
+}
+
+struct ChunkPlan {
+  int o, nq, nkv, fold_rows, splits;
+  size_t St, dS, dZ, phiq, phik, total;
+};
+
+ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_before,
+                     int chunk_frames, int To) {
+  ChunkPlan p{};
+  const size_t BH = (size_t)d.B * d.H;
+  p.o = To < frames_before ? To : frames_before;
+  p.nq = chunk_frames * L;
+  p.nkv = (p.o + chunk_frames) * L;
+  const int w = frames_before - p.o;
+  int w_next = frames_before + chunk_frames - To;
+  if (w_next < 0) w_next = 0;
+  p.fold_rows = (w_next - w) * L;
+  if (p.fold_rows < 0) p.fold_rows = 0;
+  Carve cv;
+  if (dt == REHYAT_BF16) {
+    // the split count depends only on the chunk length so that one workspace size fits every
+    // call of a stream
+    p.splits = fold_splits((int)BH, 1, (long long)chunk_frames * L);
+    p.St = cv.take(BH * d.D * d.F * 2);
+    p.dS = cv.take(BH * p.splits * d.F * d.D * 4);
+    p.dZ = cv.take(BH * p.splits * d.F * 4);
+  } else {
+    p.splits = 1;
+    const size_t max_kv = (size_t)(To + chunk_frames) * L;
+    p.phiq = cv.take(BH * (size_t)p.nq * d.F * 4);
+    p.phik = cv.take(BH * max_kv * d.F * 4);
+    p.dS = cv.take(BH * d.F * d.D * 4);
+    p.dZ = cv.take(BH * d.F * 4);
+  }
+  p.total = cv.off;
+  return p;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Launch helpers
+// ---------------------------------------------------------------------------------------------
+int launch_featmap(const rehyat_dims& d, rehyat_dtype dt, int n, const void* x, const float* W,
+                   const float* b, void* phi, cudaStream_t st) {
+  const size_t smem = ((size_t)d.F * d.D / d.G + d.F + 128 * (size_t)(d.D + 1)) * 4;
+  if (smem > 227 * 1024)
+    return fail(REHYAT_ERR_SHAPE, "feature map of D=%d F=%d G=%d needs %zu B of shared memory", d.D,
+                d.F, d.G, smem);
+  dim3 grid((n + 127) / 128, d.B * d.H);
+  if (dt == REHYAT_BF16) {
+    auto k = rehyat::featmap_kernel<__nv_bfloat16, __nv_bfloat16, false>;
+    RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), "featmap attr"));
+    k<<<grid, 128, smem, st>>>(static_cast<const __nv_bfloat16*>(x), W, b,
+                               static_cast<__nv_bfloat16*>(phi), n, d.H, d.D, d.F, d.G, d.P);
+  } else {
+    auto k = rehyat::featmap_kernel<float, float, true>;
+    RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), "featmap attr"));
+    k<<<grid, 128, smem, st>>>(static_cast<const float*>(x), W, b, static_cast<float*>(phi), n,
+                               d.H, d.D, d.F, d.G, d.P);
+  }
+  return cuda_check(cudaGetLastError(), "featmap launch");
+}
+
+template <int G>
+int launch_attn_bf16_g(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& ms, const rehyat::attn::Params& ap, dim3 grid,
+                       cudaStream_t st) {
+  auto k = rehyat::attn::hybrid_attn_bf16_kernel<G>;
+  RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)rehyat::attn::kSmemBytes),
+                    "attn attr"));
+  k<<<grid, rehyat::attn::kThreads, rehyat::attn::kSmemBytes, st>>>(mq, mk, mv, ms, ap);
+  return cuda_check(cudaGetLastError(), "attention launch");
+}
+
+int launch_attn_bf16(int G, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& ms, const rehyat::attn::Params& ap, dim3 grid,
+                     cudaStream_t st) {
+  switch (G) {
+    case 4: return launch_attn_bf16_g<4>(mq, mk, mv, ms, ap, grid, st);
+    case 8: return launch_attn_bf16_g<8>(mq, mk, mv, ms, ap, grid, st);
+    case 16: return launch_attn_bf16_g<16>(mq, mk, mv, ms, ap, grid, st);
+  }
+  return fail(REHYAT_ERR_SHAPE, "unsupported G=%d", G);
+}
+
+template <int G>
+int launch_fold_bf16_g(const CUtensorMap& mk, const CUtensorMap& mv,
+                       const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st) {
+  auto k = rehyat::state::fold_partial_bf16_kernel<G>;
+  RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)rehyat::state::kSmemBytes),
+                    "fold attr"));
+  k<<<grid, rehyat::state::kThreads, rehyat::state::kSmemBytes, st>>>(mk, mv, fp);
+  return cuda_check(cudaGetLastError(), "fold launch");
+}
+
+int launch_fold_bf16(int G, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st) {
+  switch (G) {
+    case 4: return launch_fold_bf16_g<4>(mk, mv, fp, grid, st);
+    case 8: return launch_fold_bf16_g<8>(mk, mv, fp, grid, st);
+    case 16: return launch_fold_bf16_g<16>(mk, mv, fp, grid, st);
+  }
+  return fail(REHYAT_ERR_SHAPE, "unsupported G=%d", G);
+}
+
+int launch_scan_bf16(const rehyat_dims& d, const float* dS, const float* dZ, int n_fold,
+                     int splits, int C, const float* S0, const float* Z0, __nv_bfloat16* St,
+                     float* Zc, float* S_out, float* Z_out, cudaStream_t st) {
+  dim3 grid((d.F / 32) * (d.D / 32), d.B * d.H);
+  rehyat::state::state_scan_kernel<<<grid, dim3(32, 8), 0, st>>>(dS, dZ, n_fold, splits, C, d.F,
+                                                                  d.D, S0, Z0, St, Zc, S_out, Z_out);
+  return cuda_check(cudaGetLastError(), "scan launch");
+}
+
+// Enqueue the bf16 fold partials of the forward schedule and their scan.
+int forward_states_bf16(const rehyat_dims& d, int T, int L, int Tc, int To, const void* k,
+                        const void* v, const float* Wk, const float* bk, const ForwardPlan& pl,
+                        uint8_t* ws, __nv_bfloat16* St, float* Zc, float* S_out, float* Z_out,
+                        cudaStream_t st) {
+  const long long N = (long long)T * L;
+  const int BH = d.B * d.H;
+  float* dS = reinterpret_cast<float*>(ws + pl.dS);
+  float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
+  if (pl.n_fold > 0) {
+    CUtensorMap mk, mv;
+    RH_TRY(make_map(&mk, k, d.D, N, BH));
+    RH_TRY(make_map(&mv, v, d.D, N, BH));
+    rehyat::state::FoldParams fp{};
+    fp.L = L; fp.H = d.H; fp.P = d.P; fp.T = T; fp.Tc = Tc; fp.To = To; fp.kv_frame0 = 0;
+    fp.single_rows = -1; fp.n_fold = pl.n_fold; fp.splits = pl.splits;
+    fp.Wk = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(d.G, mk, mv, fp, dim3(pl.splits, pl.n_fold, BH), st));
+  }
+  return launch_scan_bf16(d, dS, dZ, pl.n_fold, pl.splits, pl.C, nullptr, nullptr, St, Zc, S_out,
+                          Z_out, st);
+}
+
+int forward_states_f32(const rehyat_dims& d, int T, int L, int Tc, int To, const void* k,
+                       const void* v, const float* Wk, const float* bk, const ForwardPlan& pl,
+                       uint8_t* ws, float* Sc, float* Zc, cudaStream_t st) {
+  const int N = T * L;
+  float* phik = reinterpret_cast<float*>(ws + pl.phik);
+  float* dS = reinterpret_cast<float*>(ws + pl.dS);
+  float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
+  RH_TRY(launch_featmap(d, REHYAT_F32, N, k, Wk, bk, phik, st));
+  if (pl.n_fold > 0) {
+    rehyat::fp32::FoldParams fp{};
+    fp.L = L; fp.T = T; fp.Tc = Tc; fp.To = To; fp.kv_frame0 = 0; fp.single_rows = -1;
+    fp.n_fold = pl.n_fold; fp.F = d.F; fp.D = d.D; fp.nkv_rows = N;
+    fp.phik = phik; fp.v = static_cast<const float*>(v); fp.dS = dS; fp.dZ = dZ;
+    rehyat::fp32::fold_partial_f32_kernel<<<dim3(pl.n_fold, d.B * d.H), 256, 0, st>>>(fp);
+    RH_TRY(cuda_check(cudaGetLastError(), "fold f32 launch"));
+  }
+  rehyat::fp32::state_scan_f32_kernel<<<dim3((d.F * d.D + 255) / 256, d.B * d.H), 256, 0, st>>>(
+      dS, dZ, pl.n_fold, pl.C, d.F, d.D, nullptr, nullptr, Sc, Zc);
+  return cuda_check(cudaGetLastError(), "scan f32 launch");
+}
+
+}  // namespace
+
+// =============================================================================================
+// C ABI
+// =============================================================================================
+extern "C" {
+
+const char* rehyat_last_error(void) { return g_msg; }
+
+int rehyat_version(void) { return 100; }
+
+int rehyat_featmap(rehyat_dims d, rehyat_dtype dt, int n_tokens, const void* x, const float* W,
+                   const float* bias, void* phi, void* stream) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  if (n_tokens < 1) return fail(REHYAT_ERR_ARG, "n_tokens must be >= 1");
+  if (!x || !W || !phi) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(phi)) return fail(REHYAT_ERR_ALIGN, "x/phi not 16-byte aligned");
+  return launch_featmap(d, dt, n_tokens, x, W, bias, phi, static_cast<cudaStream_t>(stream));
+}
+
+int rehyat_forward_workspace_size(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens,
+                                  int Tc, int To, size_t* bytes) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(T, frame_tokens, Tc, To));
+  if (!bytes) return fail(REHYAT_ERR_ARG, "null bytes pointer");
+  *bytes = plan_forward(d, dt, T, frame_tokens, Tc, To).total;
+  return REHYAT_OK;
+}
+
+static int forward_common_checks(const rehyat_dims& d, rehyat_dtype dt, int T, int L, int Tc,
+                                 int To, const void* workspace, size_t ws_bytes,
+                                 ForwardPlan* pl) {
+  RH_TRY(check_dims(d, dt));
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(T, L, Tc, To));
+  *pl = plan_forward(d, dt, T, L, Tc, To);
+  if (!workspace || ws_bytes < pl->total)
+    return fail(REHYAT_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", pl->total, ws_bytes);
+  if (!aligned16(workspace)) return fail(REHYAT_ERR_ALIGN, "workspace not 16-byte aligned");
+  return REHYAT_OK;
+}
+
+int rehyat_forward_states(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                          const void* k, const void* v, const float* Wk, const float* bk,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  g_msg[0] = 0;
+  ForwardPlan pl;
+  RH_TRY(forward_common_checks(d, dt, T, L, Tc, To, workspace, ws_bytes, &pl));
+  if (!k || !v || !Wk) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(k) || !aligned16(v)) return fail(REHYAT_ERR_ALIGN, "k/v not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (dt == REHYAT_BF16)
+    return forward_states_bf16(d, T, L, Tc, To, k, v, Wk, bk, pl, ws,
+                               reinterpret_cast<__nv_bfloat16*>(ws + pl.St),
+                               reinterpret_cast<float*>(ws + pl.Zc), nullptr, nullptr, st);
+  return forward_states_f32(d, T, L, Tc, To, k, v, Wk, bk, pl, ws,
+                            reinterpret_cast<float*>(ws + pl.Sc),
+                            reinterpret_cast<float*>(ws + pl.Zc), st);
+}
+
+int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                          const void* q, const void* k, const void* v, const float* Wq,
+                          const float* bq, void* out, const void* workspace, size_t ws_bytes,
+                          void* stream) {
+  g_msg[0] = 0;
+  ForwardPlan pl;
+  RH_TRY(forward_common_checks(d, dt, T, L, Tc, To, workspace, ws_bytes, &pl));
+  if (!q || !k || !v || !Wq || !out) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(REHYAT_ERR_ALIGN, "q/k/v/out not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(const_cast<void*>(workspace));
+  const int BH = d.B * d.H;
+  const long long N = (long long)T * L;
+  const int rows_per_chunk = (Tc < T ? Tc : T) * L;
+  if (dt == REHYAT_BF16) {
+    CUtensorMap mq, mk, mv, ms;
+    RH_TRY(make_map(&mq, q, d.D, N, BH));
+    RH_TRY(make_map(&mk, k, d.D, N, BH));
+    RH_TRY(make_map(&mv, v, d.D, N, BH));
+    RH_TRY(make_map(&ms, ws + pl.St, d.F, d.D, (long long)BH * pl.C));
+    rehyat::attn::Params ap{};
+    ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
+    ap.H = d.H; ap.P = d.P; ap.n_states = pl.C; ap.nq_rows = (int)N;
+    ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
+    ap.Wq = Wq; ap.bq = bq; ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
+    ap.out = static_cast<__nv_bfloat16*>(out);
+    dim3 grid((rows_per_chunk + 255) / 256, pl.C, BH);
+    return launch_attn_bf16(d.G, mq, mk, mv, ms, ap, grid, st);
+  }
+  float* phiq = reinterpret_cast<float*>(ws + pl.phiq);
+  RH_TRY(launch_featmap(d, REHYAT_F32, (int)N, q, Wq, bq, phiq, st));
+  rehyat::fp32::AttnParams ap{};
+  ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
+  ap.D = d.D; ap.F = d.F; ap.nq_rows = (int)N; ap.nkv_rows = (int)N; ap.n_states = pl.C;
+  ap.scale = (float)(1.0 / std::sqrt((double)d.D));
+  ap.q = static_cast<const float*>(q); ap.k = static_cast<const float*>(k);
+  ap.v = static_cast<const float*>(v); ap.phiq = phiq;
+  ap.S = reinterpret_cast<const float*>(ws + pl.Sc);
+  ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
+  ap.out = static_cast<float*>(out);
+  rehyat::fp32::hybrid_attn_f32_kernel<<<dim3((rows_per_chunk + 3) / 4, pl.C, BH), 128, 0, st>>>(ap);
+  return cuda_check(cudaGetLastError(), "attention f32 launch");
+}
+
+int rehyat_forward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To, const void* q,
+                   const void* k, const void* v, const float* Wq, const float* bq,
+                   const float* Wk, const float* bk, void* out, void* workspace,
+                   size_t ws_bytes, void* stream) {
+  g_msg[0] = 0;
+  // every argument is checked before the first phase enqueues anything
+  ForwardPlan pl;
+  RH_TRY(forward_common_checks(d, dt, T, L, Tc, To, workspace, ws_bytes, &pl));
+  if (!q || !k || !v || !Wq || !Wk || !out) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(REHYAT_ERR_ALIGN, "q/k/v/out not 16-byte aligned");
+  RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, workspace, ws_bytes, stream));
+  return rehyat_forward_attend(d, dt, T, L, Tc, To, q, k, v, Wq, bq, out, workspace, ws_bytes,
+                               stream);
+}
+
+int rehyat_chunk_workspace_size(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
+                                int chunk_frames, int To, size_t* bytes) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(chunk_frames, frame_tokens, 1, To));
+  if (!bytes) return fail(REHYAT_ERR_ARG, "null bytes pointer");
+  *bytes = plan_chunk(d, dt, frame_tokens, To, chunk_frames, To).total;
+  return REHYAT_OK;
+}
+
+int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int L, int frames_before,
+                         int chunk_frames, int To, const void* q, const void* k_win,
+                         const void* v_win, const float* Wq, const float* bq, const float* Wk,
+                         const float* bk, float* S, float* Z, void* out, void* workspace,
+                         size_t ws_bytes, void* stream) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(chunk_frames, L, 1, To));
+  if (frames_before < 0) return fail(REHYAT_ERR_ARG, "frames_before must be >= 0");
+  if (!q || !k_win || !v_win || !Wq || !Wk || !S || !Z || !out)
+    return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k_win) || !aligned16(v_win) || !aligned16(out))
+    return fail(REHYAT_ERR_ALIGN, "q/k_win/v_win/out not 16-byte aligned");
+  const ChunkPlan pl = plan_chunk(d, dt, L, frames_before, chunk_frames, To);
+  const size_t need = plan_chunk(d, dt, L, To, chunk_frames, To).total;
+  if (!workspace || ws_bytes < need || ws_bytes < pl.total)
+    return fail(REHYAT_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, ws_bytes);
+  if (!aligned16(workspace)) return fail(REHYAT_ERR_ALIGN, "workspace not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int BH = d.B * d.H;
+
+  if (dt == REHYAT_BF16) {
+    __nv_bfloat16* St = reinterpret_cast<__nv_bfloat16*>(ws + pl.St);
+    float* dS = reinterpret_cast<float*>(ws + pl.dS);
+    float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
+    // S^T in bf16 for the readout MMA (C = 1, no folds: a transposed copy of S)
+    RH_TRY(launch_scan_bf16(d, dS, dZ, 0, 1, 1, S, Z, St, nullptr, nullptr, nullptr, st));
+    CUtensorMap mq, mk, mv, ms;
+    RH_TRY(make_map(&mq, q, d.D, pl.nq, BH));
+    RH_TRY(make_map(&mk, k_win, d.D, pl.nkv, BH));
+    RH_TRY(make_map(&mv, v_win, d.D, pl.nkv, BH));
+    RH_TRY(make_map(&ms, St, d.F, d.D, BH));
+    rehyat::attn::Params ap{};
+    ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
+    ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
+    ap.H = d.H; ap.P = d.P; ap.n_states = 1; ap.nq_rows = pl.nq;
+    ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
+    ap.Wq = Wq; ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
+    RH_TRY(launch_attn_bf16(d.G, mq, mk, mv, ms, ap, dim3((pl.nq + 255) / 256, 1, BH), st));
+    if (pl.fold_rows > 0) {
+      rehyat::state::FoldParams fp{};
+      fp.L = L; fp.H = d.H; fp.P = d.P; fp.single_rows = pl.fold_rows; fp.n_fold = 1;
+      fp.splits = pl.splits; fp.Wk = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+      RH_TRY(launch_fold_bf16(d.G, mk, mv, fp, dim3(pl.splits, 1, BH), st));
+      rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
+          dS, dZ, pl.splits, d.F, d.D, S, Z);
+      RH_TRY(cuda_check(cudaGetLastError(), "state add launch"));
+    }
+    return REHYAT_OK;
+  }
+  // fp32
+  float* phiq = reinterpret_cast<float*>(ws + pl.phiq);
+  float* phik = reinterpret_cast<float*>(ws + pl.phik);
+  float* dS = reinterpret_cast<float*>(ws + pl.dS);
+  float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
+  RH_TRY(launch_featmap(d, REHYAT_F32, pl.nq, q, Wq, bq, phiq, st));
+  rehyat::fp32::AttnParams ap{};
+  ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
+  ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
+  ap.D = d.D; ap.F = d.F; ap.nq_rows = pl.nq; ap.nkv_rows = pl.nkv; ap.n_states = 1;
+  ap.scale = (float)(1.0 / std::sqrt((double)d.D));
+  ap.q = static_cast<const float*>(q); ap.k = static_cast<const float*>(k_win);
+  ap.v = static_cast<const float*>(v_win); ap.phiq = phiq; ap.S = S; ap.Z = Z;
+  ap.out = static_cast<float*>(out);
+  rehyat::fp32::hybrid_attn_f32_kernel<<<dim3((pl.nq + 3) / 4, 1, BH), 128, 0, st>>>(ap);
+  RH_TRY(cuda_check(cudaGetLastError(), "attention f32 launch"));
+  if (pl.fold_rows > 0) {
+    RH_TRY(launch_featmap(d, REHYAT_F32, pl.nkv, k_win, Wk, bk, phik, st));
+    rehyat::fp32::FoldParams fp{};
+    fp.single_rows = pl.fold_rows; fp.n_fold = 1; fp.F = d.F; fp.D = d.D; fp.nkv_rows = pl.nkv;
+    fp.phik = phik; fp.v = static_cast<const float*>(v_win); fp.dS = dS; fp.dZ = dZ;
+    rehyat::fp32::fold_partial_f32_kernel<<<dim3(1, BH), 256, 0, st>>>(fp);
+    RH_TRY(cuda_check(cudaGetLastError(), "fold f32 launch"));
+    rehyat::fp32::state_add_f32_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
+        dS, dZ, d.F, d.D, S, Z);
+    RH_TRY(cuda_check(cudaGetLastError(), "state add f32 launch"));
+  }
+  return REHYAT_OK;
+}
+
+int rehyat_chunk_states(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                        const void* k, const void* v, const float* Wk, const float* bk,
+                        float* S_out, float* Z_out, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(T, L, Tc, To));
+  if (!k || !v || !Wk || !S_out || !Z_out) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(k) || !aligned16(v)) return fail(REHYAT_ERR_ALIGN, "k/v not 16-byte aligned");
+  const ForwardPlan pl = plan_forward(d, dt, T, L, Tc, To);
+  if (!workspace || ws_bytes < pl.total)
+    return fail(REHYAT_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", pl.total, ws_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (dt == REHYAT_BF16)
+    return forward_states_bf16(d, T, L, Tc, To, k, v, Wk, bk, pl, ws, nullptr, nullptr, S_out,
+                               Z_out, st);
+  return forward_states_f32(d, T, L, Tc, To, k, v, Wk, bk, pl, ws, S_out, Z_out, st);
+}
+
+int rehyat_sync_status(void* stream) {
+  g_msg[0] = 0;
+  RH_TRY(cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "stream sync"));
+  int err = 0;
+  RH_TRY(cuda_check(cudaMemcpyFromSymbol(&err, rehyat::sm100::g_device_error, sizeof(int)),
+                    "read device error word"));
+  if (err) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(rehyat::sm100::g_device_error, &zero, sizeof(int));
+    return fail(REHYAT_ERR_TIMEOUT, "a kernel wait timed out (device error %d)", err);
+  }
+  return REHYAT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+/*
+ * rehyat.h - C ABI of librehyat.so: the forward pass of ReHyAt chunk-wise recurrent hybrid
+ * attention on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources: "ReHyAt overview" page, maplevalley.com.cn news 2180822, §2.2.1
+ * hybrid output, §2.2.2 feature map, §2.3 recurrence and states, §5.2 streaming loop; and
+ * "Neuer Ansatz zur effizienten Videogenerierung mit ReHyAt", mind-verse.de, sections
+ * "Temporär segmentierte hybride Aufmerksamkeit" and "Rekurrente Formulierung"):
+ *
+ *   A video of T latent frames with L = frame_tokens tokens per frame is a token sequence of
+ *   N = T*L rows, frame-major.  Frames are grouped into temporal chunks of Tc frames; chunk c
+ *   owns query frames [c*Tc, e_c), e_c = min((c+1)*Tc, T).  A query of chunk c attends
+ *     - with exact softmax weights exp(q.k/sqrt(D)) to the key frames [w_c, e_c),
+ *       w_c = max(0, c*Tc - To)  (its own chunk, bidirectional, plus To frames before it);
+ *     - with linear weights phi_q(q).phi_k(k) to every earlier key frame [0, w_c), read from
+ *       the running states S_c = sum phi_k(k) v^T (F x D) and Z_c = sum phi_k(k) (F);
+ *     - not at all to later frames;
+ *   and the two parts share one normaliser:
+ *     o = (sum_{j in window} e^{q.k_j/sqrt(D)} v_j + phi_q(q)^T S_c)
+ *       / (sum_{j in window} e^{q.k_j/sqrt(D)}     + phi_q(q)^T Z_c).
+ *   After chunk c the frames that leave the window, [w_c, w_{c+1}), are folded into (S, Z).
+ *
+ *   phi(x) (separate weights for q and k): u = grouped 1x1 linear of x (G groups; group g maps
+ *   x[g*D/G, (g+1)*D/G) to u[g*F/G, (g+1)*F/G) with W[g] of shape (F/G, D/G)) plus bias; u is
+ *   split into P contiguous parts (the first F mod P parts one longer) and part p (1-based)
+ *   becomes softplus(u_p)^p; the parts are concatenated back in order.
+ *
+ * Conventions for every call:
+ *   - Tensors are dense, row-major, per (b, h) contiguous: a "[B,H,n,D]" tensor holds row r of
+ *     head h of batch b at element ((b*H + h)*n + r)*D.  Device pointers unless stated.
+ *   - q, k, v, out, phi, the states and the workspace must be 16-byte aligned.
+ *   - Weights W are fp32 [H, G, F/G, D/G]; biases fp32 [H, F] or NULL (zero).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only enqueues work
+ *     on it: the library never allocates device memory, never synchronises, and keeps no state
+ *     between calls other than the device error word read by rehyat_sync_status().
+ *   - The caller owns every buffer.  Buffers may not overlap, except where stated.
+ *   - dtype REHYAT_BF16: q, k, v, out (and phi) are bf16; arithmetic is bf16 tensor-core
+ *     products with fp32 accumulation, fp32 softmax and fp32 states.  Requires D = F = 128.
+ *     dtype REHYAT_F32: everything fp32 on CUDA cores; requires D % 32 == 0, D <= 256,
+ *     F <= 256.
+ *   - Return value: REHYAT_OK or a negative rehyat_status; rehyat_last_error() then gives a
+ *     message (per host thread).  A bad argument is reported before anything is enqueued.
+ */
+#ifndef REHYAT_H
+#define REHYAT_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  REHYAT_OK = 0,
+  REHYAT_ERR_ARG = -1,       /* null pointer, non-positive size, Tc < 1, To < 0, P out of range */
+  REHYAT_ERR_SHAPE = -2,     /* D, F, G combination not supported for the dtype */
+  REHYAT_ERR_DTYPE = -3,     /* unknown dtype */
+  REHYAT_ERR_WORKSPACE = -4, /* workspace NULL or smaller than the *_workspace_size query */
+  REHYAT_ERR_CUDA = -5,      /* a CUDA runtime call or a launch failed */
+  REHYAT_ERR_TIMEOUT = -6,   /* a kernel's bounded wait gave up (from rehyat_sync_status) */
+  REHYAT_ERR_ALIGN = -7      /* a pointer is not 16-byte aligned */
+} rehyat_status;
+
+typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
+
+/* Problem dimensions shared by all calls: batch B, heads H, head dim D, feature count F of phi,
+ * group count G of its grouped linear (D % G == 0, F % G == 0), polynomial parts P (1..F). */
+typedef struct {
+  int B, H, D, F, G, P;
+} rehyat_dims;
+
+/* Message for the last non-OK status returned on this host thread ("" if none). */
+const char* rehyat_last_error(void);
+
+/* ABI version of this library (major*100 + minor). */
+int rehyat_version(void);
+
+/* Feature map phi of the "ReHyAt overview" page §2.2.2, standalone.
+ *   x    [B,H,n_tokens,D] (dtype), W [H,G,F/G,D/G] fp32, bias [H,F] fp32 or NULL,
+ *   phi  [B,H,n_tokens,F] (dtype), written.
+ * Any D, F, G, P that satisfy the dims rules (no D = F = 128 requirement here). */
+int rehyat_featmap(rehyat_dims d, rehyat_dtype dt, int n_tokens, const void* x, const float* W,
+                   const float* bias, void* phi, void* stream);
+
+/* Workspace bytes rehyat_forward needs for these sizes (written to *bytes). */
+int rehyat_forward_workspace_size(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens,
+                                  int Tc, int To, size_t* bytes);
+
+/* Hybrid attention over a whole sequence (every chunk of the §2.2.1 schedule in one call; the
+ * §2.3 states are formed as prefix sums of per-chunk folds, so chunks run in parallel).
+ *   q, k, v  [B,H,T*frame_tokens,D] (dtype);  Wq/bq, Wk/bk: phi_q and phi_k parameters;
+ *   out      [B,H,T*frame_tokens,D] (dtype), written;
+ *   workspace: device scratch of at least rehyat_forward_workspace_size() bytes. */
+int rehyat_forward(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
+                   const void* q, const void* k, const void* v, const float* Wq, const float* bq,
+                   const float* Wk, const float* bk, void* out, void* workspace,
+                   size_t ws_bytes, void* stream);
+
+/* rehyat_forward in two phases on the same workspace (rehyat_forward is exactly
+ * rehyat_forward_states followed by rehyat_forward_attend):
+ *   _states: the §2.3 folds of every chunk and their prefix sums (the state each chunk reads),
+ *            written into the workspace; reads k, v and phi_k's parameters;
+ *   _attend: the hybrid output of every chunk from q, k, v and the workspace states.
+ * The workspace must not change between the two calls.  Useful to reuse the states of one
+ * (k, v) across several query sets, and to time the phases separately. */
+int rehyat_forward_states(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
+                          const void* k, const void* v, const float* Wk, const float* bk,
+                          void* workspace, size_t ws_bytes, void* stream);
+int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
+                          const void* q, const void* k, const void* v, const float* Wq,
+                          const float* bq, void* out, const void* workspace, size_t ws_bytes,
+                          void* stream);
+
+/* Workspace bytes rehyat_chunk_forward needs for one chunk of chunk_frames frames. */
+int rehyat_chunk_workspace_size(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
+                                int chunk_frames, int To, size_t* bytes);
+
+/* One step of the streaming loop of the "ReHyAt overview" page §5.2: the chunk whose first
+ * frame is frame `frames_before` of the video, `chunk_frames` frames long.
+ *   o = min(To, frames_before) overlap frames precede it in the softmax window.
+ *   q      [B,H,chunk_frames*L,D]              the chunk's queries;
+ *   k_win, v_win [B,H,(o+chunk_frames)*L,D]    the overlap frames followed by the chunk's own;
+ *   S [B,H,F,D] fp32, Z [B,H,F] fp32 (in/out)  the states holding every frame before the
+ *                                              window (zeros for the first chunk);
+ *   out    [B,H,chunk_frames*L,D]              written.
+ * After the output, the window frames the next chunk no longer sees (the first
+ * max(0, frames_before + chunk_frames - To) - (frames_before - o) of them, assuming the next
+ * chunk uses the same To) are folded into S and Z in place.  Memory use does not depend on how
+ * many chunks came before. */
+int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int frame_tokens, int frames_before,
+                         int chunk_frames, int To, const void* q, const void* k_win,
+                         const void* v_win, const float* Wq, const float* bq, const float* Wk,
+                         const float* bk, float* S, float* Z, void* out, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/* The states every chunk of rehyat_forward reads (§2.3), for inspection and testing:
+ *   S_out [B,H,C,F,D] fp32 and Z_out [B,H,C,F] fp32 with C = ceil(T/Tc); S_out[..,c,..] is the
+ *   sum over key frames [0, w_c) of phi_k(k) v^T.  Same workspace as rehyat_forward. */
+int rehyat_chunk_states(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
+                        const void* k, const void* v, const float* Wk, const float* bk,
+                        float* S_out, float* Z_out, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/* Synchronise `stream` and report device-side failures of earlier calls: REHYAT_ERR_TIMEOUT if
+ * a kernel's bounded wait gave up (the error word is then cleared), REHYAT_ERR_CUDA if the
+ * stream reports a CUDA error, else REHYAT_OK. */
+int rehyat_sync_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* REHYAT_H */

@@ -56,6 +56,7 @@ __all__ = [
     "chunk_forward",
     "prefix_states",
     "hybrid_attention_bruteforce",
+    "hybrid_attention_rows",
     "SET_SOFTMAX",
     "SET_LINEAR",
     "SET_NONE",
@@ -189,6 +190,37 @@ def hybrid_attention_quadratic(q, k, v, phi_q, phi_k, frame_tokens: int, Tc: int
     """The ReHyAt hybrid output for the standard chunk pattern, quadratic form."""
     T = q.shape[0] // frame_tokens
     return hybrid_attention_masked(q, k, v, phi_q, phi_k, frame_tokens, rehyat_mask(T, Tc, To))
+
+
+def hybrid_attention_rows(q, k, v, Wq, bq, Wk, bk, P: int, frame_tokens: int, Tc: int, To: int,
+                          rows) -> np.ndarray:
+    """The quadratic form evaluated for selected query rows only (for sequences too long to
+    evaluate whole): row i of chunk c = (i // L) // Tc weighs keys [w_c L, e_c L) by
+    exp(q.k/sqrt(D)) and keys [0, w_c L) by phi_q(q).phi_k(k), shifted by the row max of the
+    window logits, and divides by the sum of the weights."""
+    q = np.asarray(q, np.float64); k = np.asarray(k, np.float64); v = np.asarray(v, np.float64)
+    n, D = q.shape
+    L = frame_tokens
+    T = n // L
+    bounds = chunk_bounds(T, Tc, To)
+    rows = np.asarray(rows, dtype=np.int64)
+    out = np.empty((len(rows), v.shape[1]))
+    phi_q = feature_map(q[rows], Wq, bq, P)
+    need = max(bounds[(int(r) // L) // Tc][0] for r in rows) * L
+    phi_k = feature_map(k[:need], Wk, bk, P) if need > 0 else None
+    for a, r in enumerate(rows):
+        w, s, e = bounds[(int(r) // L) // Tc]
+        logits = k[w * L:e * L] @ q[r] / math.sqrt(D)
+        mu = logits.max()
+        ws = np.exp(logits - mu)
+        num = ws @ v[w * L:e * L]
+        den = ws.sum()
+        if w > 0:
+            wl = (phi_k[:w * L] @ phi_q[a]) * math.exp(-mu)
+            num = num + wl @ v[:w * L]
+            den = den + wl.sum()
+        out[a] = num / den
+    return out
 
 
 # ---------------------------------------------------------------------------------------------

@@ -1,0 +1,95 @@
+"""Host-side checks of librehyat.so that need no GPU: it loads, exports every function the header
+declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hybrid_softmax_linear_chunked_b200 import binding as rb
+from hybrid_softmax_linear_chunked_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "rehyat.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return rb.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rehyat_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_surface():
+    assert declared_functions() == sorted(rb.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.rehyat_version() == 100
+
+
+FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced: checks come first
+
+
+def dims(B=1, H=2, D=128, F=128, G=8, P=2):
+    return rb.Dims(B, H, D, F, G, P)
+
+
+def call_forward(lib, d, dt=rb.REHYAT_BF16, T=7, L=64, Tc=3, To=1, ws_bytes=1 << 40, **ptrs):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, Wq=FAKE, bq=None, Wk=FAKE, bk=None, out=FAKE, ws=FAKE)
+    p.update(ptrs)
+    return lib.rehyat_forward(d, dt, T, L, Tc, To, p["q"], p["k"], p["v"], p["Wq"], p["bq"],
+                              p["Wk"], p["bk"], p["out"], p["ws"], ws_bytes, None)
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(d=dims(B=0)), -1),
+    (dict(d=dims(G=3)), -1),
+    (dict(d=dims(P=200)), -1),
+    (dict(d=dims(D=64, F=64)), -2),
+    (dict(d=dims(G=2)), -2),
+    (dict(d=dims(), dt=7), -3),
+    (dict(d=dims(), Tc=0), -1),
+    (dict(d=dims(), To=-1), -1),
+    (dict(d=dims(), T=0), -1),
+    (dict(d=dims(), ws_bytes=16), -4),
+    (dict(d=dims(), q=None), -1),
+    (dict(d=dims(), q=ctypes.c_void_p(0x10008)), -7),
+    (dict(d=dims(D=48, F=48, G=4), dt=rb.REHYAT_F32), -2),
+])
+def test_forward_rejects_bad_arguments(lib, kwargs, status):
+    assert call_forward(lib, **kwargs) == status
+    assert lib.rehyat_last_error().decode()
+
+
+def test_workspace_sizes(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.rehyat_forward_workspace_size(dims(H=12), rb.REHYAT_BF16, 21, 1560, 3, 1,
+                                             ctypes.byref(n)) == 0
+    # 6 folds x splits x (F*D + F) fp32 partials, 7 transposed bf16 states, 7 Z vectors
+    assert n.value >= 12 * (7 * 128 * 128 * 2 + 7 * 128 * 4)
+    m = ctypes.c_size_t(0)
+    assert lib.rehyat_chunk_workspace_size(dims(B=2, H=12), rb.REHYAT_BF16, 1560, 3, 1,
+                                           ctypes.byref(m)) == 0
+    # streaming workspace does not depend on how long the video is
+    assert m.value < 64 << 20
+
+
+def test_chunk_forward_rejects_bad_arguments(lib):
+    d = dims()
+    st = lib.rehyat_chunk_forward(d, rb.REHYAT_BF16, 64, -1, 3, 1, FAKE, FAKE, FAKE, FAKE, None,
+                                  FAKE, None, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert st == -1
+    st = lib.rehyat_chunk_forward(d, rb.REHYAT_BF16, 64, 3, 3, 1, FAKE, FAKE, FAKE, FAKE, None,
+                                  FAKE, None, None, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert st == -1
+    st = lib.rehyat_chunk_forward(d, rb.REHYAT_BF16, 64, 3, 3, 1, FAKE, FAKE, FAKE, FAKE, None,
+                                  FAKE, None, FAKE, FAKE, FAKE, FAKE, 8, None)
+    assert st == -4

@@ -188,7 +188,18 @@ def check_invariants(mod):
     np.testing.assert_allclose(out_p, out, rtol=1e-12, atol=1e-12)
 
 
-PINS = [check_golden, check_featmap_conv1d, check_single_chunk_is_softmax, check_linear_only,
+def check_rows_form(mod):
+    rng = np.random.default_rng(7)
+    for (T, L, Tc, To, P) in [(7, 5, 3, 1, 2), (5, 4, 1, 2, 3)]:
+        q, k, v, Wq, bq, Wk, bk = _rand_problem(rng, T, L, 8, 8, 2)
+        pq, pk = mod.feature_map(q, Wq, bq, P), mod.feature_map(k, Wk, bk, P)
+        quad = mod.hybrid_attention_quadratic(q, k, v, pq, pk, L, Tc, To)
+        rows = np.array([0, 3, L * Tc, T * L - 1, (T * L) // 2])
+        got = mod.hybrid_attention_rows(q, k, v, Wq, bq, Wk, bk, P, L, Tc, To, rows)
+        np.testing.assert_allclose(got, quad[rows], rtol=1e-12, atol=1e-12)
+
+
+PINS = [check_rows_form, check_golden, check_featmap_conv1d, check_single_chunk_is_softmax, check_linear_only,
         check_bruteforce, check_recurrent_and_streaming, check_invariants]
 
 
