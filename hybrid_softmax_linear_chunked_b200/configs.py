@@ -91,6 +91,20 @@ class Workload:
         tot += (phi_q_tokens + folded) * 2.0 * D * F / self.G
         return tot * self.B * self.H
 
+    def attn_tensor_flops(self) -> float:
+        """Tensor-core FLOPs of the fused attention kernel over all (b, h): Q K^T and P V over
+        each chunk's window and the phi_q . S readout (2 F D per query of a chunk that has a
+        linear region).  The CUDA-core work in the same kernel (phi_q, phi_q . Z, softmax) is
+        not counted."""
+        L, D, F = self.frame_tokens, self.D, self.F
+        tot = 0.0
+        for (w, s, e) in self.chunk_bounds():
+            nq, nw = (e - s) * L, (e - w) * L
+            tot += 4.0 * nq * nw * D
+            if w > 0:
+                tot += 2.0 * nq * F * D
+        return tot * self.B * self.H
+
     def io_bytes(self) -> float:
         """Algorithmic HBM bytes: q, k, v read once and the output written once."""
         el = 4 if self.dtype == "f32" else 2
