@@ -22,7 +22,8 @@ STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_SHAPE", -3: "ERR_DTYPE", -4: "ERR_WOR
 EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_forward_workspace_size", "rehyat_forward", "rehyat_forward_states",
             "rehyat_forward_attend", "rehyat_chunk_workspace_size",
-            "rehyat_chunk_forward", "rehyat_chunk_states", "rehyat_sync_status"]
+            "rehyat_chunk_forward", "rehyat_chunk_forward_static", "rehyat_chunk_states",
+            "rehyat_sync_status"]
 
 
 class RehyatError(RuntimeError):
@@ -70,6 +71,8 @@ def load() -> ctypes.CDLL:
                                               ctypes.POINTER(c_size_t)]
     L.rehyat_chunk_forward.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
                                        P, P, P, P, P, c_size_t, P]
+    L.rehyat_chunk_forward_static.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P,
+                                              P, P, P, P, P, P, P]
     L.rehyat_chunk_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
                                       P, c_size_t, P]
     L.rehyat_sync_status.argtypes = [P]
@@ -245,6 +248,23 @@ def chunk_forward(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, frame_tokens
                                     _ptr(q), _ptr(k_win), _ptr(v_win), _ptr(Wq), _ptr(bq),
                                     _ptr(Wk), _ptr(bk), _ptr(S), _ptr(Z), _ptr(out), _ptr(ws),
                                     ws.numel(), _stream(dev)))
+    return out
+
+
+def chunk_forward_static(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, frame_tokens: int,
+                         frames_before: int, To: int, out: torch.Tensor | None = None):
+    """chunk_forward without a workspace: the library's own fixed device scratch is used (for
+    callers that cannot allocate); bf16 only."""
+    lib = load()
+    dev = _dev(q, k_win, v_win, Wq, bq, Wk, bk, S, Z)
+    d = dims_of(q, Wq, P)
+    chunk_frames = q.shape[2] // frame_tokens
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.rehyat_chunk_forward_static(d, _dtype_code(q), frame_tokens, frames_before,
+                                           chunk_frames, To, _ptr(q), _ptr(k_win), _ptr(v_win),
+                                           _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(S),
+                                           _ptr(Z), _ptr(out), _stream(dev)))
     return out
 
 

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/rehyat.h"
 #include "attn_bf16.cuh"
@@ -329,6 +330,35 @@ int forward_states_f32(const rehyat_dims& d, int T, int L, int Tc, int To, const
   return cuda_check(cudaGetLastError(), "scan f32 launch");
 }
 
+// ---------------------------------------------------------------------------------------------
+// Library-owned scratch for rehyat_chunk_forward_static (callers that cannot allocate device
+// memory themselves).  A fixed array in the module's device memory: every GPU that loads the
+// library holds kStaticScratchBytes of it until the process exits.
+// ---------------------------------------------------------------------------------------------
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mutex;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device.  The host-side name of the array is
+// only a stand-in, so the address is looked up once per device (with that device current) and
+// cached.
+int static_scratch_for_current_device(void** out) {
+  int dev = -1;
+  RH_TRY(cuda_check(cudaGetDevice(&dev), "cudaGetDevice"));
+  if (dev < 0 || dev >= kMaxDevices) return fail(REHYAT_ERR_CUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    RH_TRY(cuda_check(cudaGetSymbolAddress(&p, g_static_scratch), "cudaGetSymbolAddress(scratch)"));
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return REHYAT_OK;
+}
+
 }  // namespace
 
 // =============================================================================================
@@ -543,6 +573,69 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int L, int frames_befor
     rehyat::fp32::state_add_f32_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
         dS, dZ, d.F, d.D, S, Z);
     RH_TRY(cuda_check(cudaGetLastError(), "state add f32 launch"));
+  }
+  return REHYAT_OK;
+}
+
+int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frames_before,
+                                int chunk_frames, int To, const void* q, const void* k_win,
+                                const void* v_win, const float* Wq, const float* bq,
+                                const float* Wk, const float* bk, float* S, float* Z, void* out,
+                                void* stream) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  if (dt != REHYAT_BF16) return fail(REHYAT_ERR_DTYPE, "the static-scratch call is bf16 only");
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(chunk_frames, L, 1, To));
+  if (frames_before < 0) return fail(REHYAT_ERR_ARG, "frames_before must be >= 0");
+  if (!q || !k_win || !v_win || !Wq || !Wk || !S || !Z || !out)
+    return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k_win) || !aligned16(v_win) || !aligned16(out))
+    return fail(REHYAT_ERR_ALIGN, "q/k_win/v_win/out not 16-byte aligned");
+  // Same plan as rehyat_chunk_forward, with the fold split count lowered until the scratch fits.
+  ChunkPlan pl = plan_chunk(d, dt, L, frames_before, chunk_frames, To);
+  const size_t BH = (size_t)d.B * d.H;
+  const size_t st_bytes = round_up(BH * d.D * d.F * 2, 256);
+  auto total_for = [&](int splits) {
+    return st_bytes + round_up(BH * splits * d.F * d.D * 4, 256) + round_up(BH * splits * d.F * 4, 256);
+  };
+  int splits = pl.splits;
+  while (splits > 1 && total_for(splits) > kStaticScratchBytes) --splits;
+  if (total_for(splits) > kStaticScratchBytes)
+    return fail(REHYAT_ERR_WORKSPACE,
+                "B*H=%zu needs %zu bytes of scratch; the library's static scratch holds %zu",
+                BH, total_for(splits), kStaticScratchBytes);
+  void* scratch = nullptr;
+  RH_TRY(static_scratch_for_current_device(&scratch));
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  __nv_bfloat16* St = reinterpret_cast<__nv_bfloat16*>(ws);
+  float* dS = reinterpret_cast<float*>(ws + st_bytes);
+  float* dZ = reinterpret_cast<float*>(ws + st_bytes + round_up(BH * splits * d.F * d.D * 4, 256));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nbh = d.B * d.H;
+  // Nothing in the scratch has to start at zero: every byte a kernel reads was written earlier
+  // in this call (S^T by the scan, every split's partial by the fold kernel).
+  RH_TRY(launch_scan_bf16(d, dS, dZ, 0, 1, 1, S, Z, St, nullptr, nullptr, nullptr, st));
+  CUtensorMap mq, mk, mv, ms;
+  RH_TRY(make_map(&mq, q, d.D, pl.nq, nbh));
+  RH_TRY(make_map(&mk, k_win, d.D, pl.nkv, nbh));
+  RH_TRY(make_map(&mv, v_win, d.D, pl.nkv, nbh));
+  RH_TRY(make_map(&ms, St, d.F, d.D, nbh));
+  rehyat::attn::Params ap{};
+  ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
+  ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
+  ap.H = d.H; ap.P = d.P; ap.n_states = 1; ap.nq_rows = pl.nq;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
+  ap.Wq = Wq; ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
+  RH_TRY(launch_attn_bf16(d.G, mq, mk, mv, ms, ap, dim3((pl.nq + 255) / 256, 1, nbh), st));
+  if (pl.fold_rows > 0) {
+    rehyat::state::FoldParams fp{};
+    fp.L = L; fp.H = d.H; fp.P = d.P; fp.single_rows = pl.fold_rows; fp.n_fold = 1;
+    fp.splits = splits; fp.Wk = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(d.G, mk, mv, fp, dim3(splits, 1, nbh), st));
+    rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, nbh), 256, 0, st>>>(
+        dS, dZ, splits, d.F, d.D, S, Z);
+    RH_TRY(cuda_check(cudaGetLastError(), "state add launch"));
   }
   return REHYAT_OK;
 }

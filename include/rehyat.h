@@ -133,6 +133,27 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int frame_tokens, int f
                          const float* bk, float* S, float* Z, void* out, void* workspace,
                          size_t ws_bytes, void* stream);
 
+/* rehyat_chunk_forward for callers that cannot allocate device memory: no workspace argument.
+ * The pages have no counterpart of this call; it exists for callers such as a plugin inside a
+ * host framework that owns every allocation, or a code path that must not call cudaMalloc
+ * (for example while another component is capturing or replaying work).  Same arguments and
+ * results as rehyat_chunk_forward (bf16 only); the scratch it needs lives in a fixed 16 MiB
+ * array inside the library's device memory, which every GPU that loads the library keeps for
+ * the life of the process.
+ *   - The first call on a device looks up that array's device address (once per device, with
+ *     the device current); make that first call before any stream capture.
+ *   - Returns REHYAT_ERR_WORKSPACE if B*H is too large for the array (above 169); the fold
+ *     then uses fewer token splits than rehyat_chunk_forward when that is needed to fit.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - Every call shares the one array, whatever the stream: calls whose work overlaps on the
+ *     GPU race on it and must be ordered by the caller (same stream, or events).
+ *   - Nothing in the array needs to start at zero; it keeps the last call's contents. */
+int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
+                                int frames_before, int chunk_frames, int To, const void* q,
+                                const void* k_win, const void* v_win, const float* Wq,
+                                const float* bq, const float* Wk, const float* bk, float* S,
+                                float* Z, void* out, void* stream);
+
 /* The states every chunk of rehyat_forward reads (§2.3), for inspection and testing:
  *   S_out [B,H,C,F,D] fp32 and Z_out [B,H,C,F] fp32 with C = ceil(T/Tc); S_out[..,c,..] is the
  *   sum over key frames [0, w_c) of phi_k(k) v^T.  Same workspace as rehyat_forward. */
