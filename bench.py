@@ -381,7 +381,7 @@ def main():
                          "traffic": read_traffic()},
             "e2e": {"value": tokens_per_step / (e2e_ms / E * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * K,
+            "gpu_launches": 5 * K,  # per step: 2 weight preps, fold, scan, attention
             "clocks": sampler.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

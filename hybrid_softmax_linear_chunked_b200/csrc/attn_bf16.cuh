@@ -10,10 +10,13 @@
 // with the running max m_t kept lazily: O_t and l_t are rescaled only when the tile max exceeds
 // m_t by more than 8 (a factor 256), so exp2 arguments stay <= 8.
 // Epilogue (the hybrid joint normaliser of the "ReHyAt overview" page §2.2.1 and the state
-// readout of §2.3): the softmax warpgroup overwrites its Q tile in shared memory with
-// phi_q(q) * 2^-m (bf16), one more MMA adds phi_q 2^-m . S_c into O_t, and
-// l_t += 2^-m phi_q . Z_c; the output is O_t / l_t.  m starts at 0 for chunks that have a
-// linear region, so 2^-m <= 1 and a row can never lose both terms to underflow.
+// readout of §2.3), for chunks that have a linear region: the grouped linear of phi_q runs on the
+// tensor cores as U_t = Q_t Wbd^T (block-diagonal W in bf16 hi + lo parts, two MMAs into the now
+// free S_t columns); the softmax warpgroup turns its U row into phi_q(q) * 2^-m (bias, softplus,
+// part powers) and writes it as bf16 over its Q tile in shared memory; one more MMA adds
+// phi_q 2^-m . S_c into O_t, and l_t += 2^-m phi_q . Z_c; the output is O_t / l_t.  m starts at
+// 0 for chunks that have a linear region, so 2^-m <= 1 and a row can never lose both terms to
+// underflow.
 //
 // Warp roles (320 threads): warps 0-3 softmax/epilogue of tile 0, warps 4-7 of tile 1, warp 8
 // TMA producer (+ TMEM allocation), warp 9 MMA issuer.  TMEM columns: S_0 [0,128), S_1
@@ -40,12 +43,10 @@ constexpr uint32_t kOffQ0 = 0;
 constexpr uint32_t kOffQ1 = kOffQ0 + kTileBytes;
 constexpr uint32_t kOffK = kOffQ1 + kTileBytes;       // 2 stages
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;    // 2 stages
-constexpr int kMinG = 4;                             // smallest supported group count
-constexpr uint32_t kOffW = kOffV + 2 * kTileBytes;    // W_q of the head, fp32 (F * D / G)
-constexpr uint32_t kWBytesMax = kFD * kHD / kMinG * 4;
-constexpr uint32_t kOffB = kOffW + kWBytesMax;         // bias, F fp32
+constexpr uint32_t kOffB = kOffV + 2 * kTileBytes;    // bias of phi_q, F fp32
 constexpr uint32_t kOffZ = kOffB + kFD * 4;            // Z_c, F fp32
-constexpr uint32_t kSmemBytes = kOffZ + kFD * 4 + 1024;  // + alignment slack
+constexpr uint32_t kOffPw = kOffZ + kFD * 4;           // part power of each feature, int
+constexpr uint32_t kSmemBytes = kOffPw + kFD * 4 + 1024;  // + alignment slack
 
 enum Bar {
   kQFull = 0,
@@ -60,7 +61,9 @@ enum Bar {
   kPhiFull = 16,  // 2 (per query tile, 128 arrivals)
   kRoDone = 18,   // 2
   kMmaDone = 20,
-  kNumBars = 21
+  kWbFull = 21,  // block-diagonal W_q (hi, lo) loaded into the V stages
+  kUFull = 22,   // 2 (per query tile): U_t = Q_t Wbd^T complete
+  kNumBars = 24
 };
 
 struct Params {
@@ -73,7 +76,6 @@ struct Params {
   int n_states;       // states per (b, h) in St / Z (state index = chunk index)
   int nq_rows;        // rows per (b, h) of q and out
   float scale_log2;   // log2(e) / sqrt(D)
-  const float* Wq;    // [H, G, F/G, D/G]
   const float* bq;    // [H, F] or null
   const float* Z;     // [BH, n_states, F]
   __nv_bfloat16* out; // [BH, nq_rows, D]
@@ -99,17 +101,13 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_addr, int kk) {
   return sdesc_sw128(tile_addr + kk * 16 * 128, kBM * 128, 1024);
 }
 
-template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
     hybrid_attn_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                             const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV,
-                            const __grid_constant__ CUtensorMap tmSt, const Params p) {
-  constexpr int Dg = kHD / G, Fg = kFD / G;
-  static_assert(Dg == Fg, "in-place phi_q needs equal group widths");
-  static_assert(Dg % 8 == 0, "group width must be a multiple of 8");
-  static_assert(G >= kMinG && kFD * Dg * 4 <= kWBytesMax, "W_q does not fit its shared-memory slot");
-  static_assert(kSmemBytes <= 232448, "shared memory over the per-CTA limit");
+                            const __grid_constant__ CUtensorMap tmSt,
+                            const __grid_constant__ CUtensorMap tmW, const Params p) {
+  static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
 
   // ---- chunk geometry (uniform over the CTA) ----
   const int c = blockIdx.y, bh = blockIdx.z, h = bh % p.H;
@@ -134,9 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &abort_sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  float* sW = reinterpret_cast<float*>(sm + kOffW);
   float* sB = reinterpret_cast<float*>(sm + kOffB);
   float* sZ = reinterpret_cast<float*>(sm + kOffZ);
+  int* sPw = reinterpret_cast<int*>(sm + kOffPw);
 
   if (warp == 8) {
     tmem_alloc(&tmem_base_sh, 512);
@@ -151,9 +149,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (tid < 256 && has_linear) {
-    const float* Wh = p.Wq + (size_t)h * kFD * Dg;
-    for (int i = tid; i < kFD * Dg; i += 256) sW[i] = Wh[i];
     for (int i = tid; i < kFD; i += 256) {
+      sPw[i] = part_power(i, kFD, p.P);
       sB[i] = p.bq ? p.bq[(size_t)h * kFD + i] : 0.f;
       sZ[i] = p.Z[((size_t)bh * p.n_states + c) * kFD + i];
     }
@@ -226,8 +223,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         st_issued = true;
       }
     }
+    bool wb_issued = false;
+    if (ok && has_linear) {
+      // Block-diagonal W_q (hi, lo) goes into the two V stages once their last P.V is done.
+      for (int s = 0; s < 2 && ok; ++s) {
+        const int last = (n_kv - 1) - (((n_kv - 1) & 1) != s ? 1 : 0);  // last use of stage s
+        if (last >= 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars[kVEmpty + s], (last >> 1) & 1, abort_flag));
+      }
+      if (ok) {
+        if (leader) {
+          mbar_arrive_expect_tx(&bars[kWbFull], 2 * kTileBytes);
+          for (int s = 0; s < 2; ++s) {
+            uint8_t* dst = sm + kOffV + s * kTileBytes;
+            tma_load_3d(dst, &tmW, &bars[kWbFull], 0, 0, h * 2 + s);
+            tma_load_3d(dst + kBM * 128, &tmW, &bars[kWbFull], 64, 0, h * 2 + s);
+          }
+        }
+        __syncwarp();
+        wb_issued = true;
+      }
+    }
     if (!ok) {
       // Abort: let every copy already issued land before the CTA can exit.
+      if (wb_issued) mbar_wait_drain(&bars[kWbFull], 0);
       mbar_wait_drain(&bars[kQFull], 0);
       for (int j = max(0, issued_k - 2); j < issued_k; ++j)
         mbar_wait_drain(&bars[kKFull + (j & 1)], (j >> 1) & 1);
@@ -304,8 +323,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) commit(kVEmpty + (j & 1));
     }
     if (ok && has_linear) {
+      // U_t = Q_t Wbd_hi^T + Q_t Wbd_lo^T into the S_t columns (free once P_t.V is issued).
+      ok = wait(kWbFull, 0);
+      if (ok) {
+        tc_fence_after();
+        if (leader) {
+          for (int t = 0; t < nt; ++t) {
+            const uint32_t d = tmem + t * 128;
+            const uint32_t qb = t ? sQ1 : sQ0;
+            for (int part = 0; part < 2; ++part) {
+              const uint32_t wb = part ? sV1 : sV0;
+              for (int kk = 0; kk < kHD / 16; ++kk)
+                mma_ss(d, kmajor_desc(qb, kk), kmajor_desc(wb, kk), id_qk,
+                       (part > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&bars[kUFull + t]);
+          }
+        }
+        __syncwarp();
+      }
       const uint32_t stb = (n_kv & 1) ? sK1 : sK0;
-      ok = wait(kStFull, 0);
+      if (ok) ok = wait(kStFull, 0);
       for (int t = 0; t < nt && ok; ++t) {
         ok = wait(kPhiFull + t, 0);
         if (!ok) break;
@@ -341,112 +379,115 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull + t], j & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        float s[kBN];
-#pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          uint32_t rr[32];
-          tmem_ld32(tS + cc * 32, rr);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(rr[i]);
-        }
-        const int valid = nk - j * kBN;
+        // The S row (128 fp32) is read once into registers; the row max is a tree over eight
+        // partial maxima and the row sum uses four accumulators, so neither is one long
+        // dependency chain.  Only the window's last tile can be ragged (uniform branch).
+        const int valid = nk - j * kBN;  // key columns of this tile inside the window
+        uint32_t rr[kBN];
+        tmem_ld128(tS, rr);
         if (valid < kBN) {
 #pragma unroll
           for (int i = 0; i < kBN; ++i)
-            if (i >= valid) s[i] = -INFINITY;
+            if (i >= valid) rr[i] = __float_as_uint(-INFINITY);
         }
-        float mx = s[0];
+        float mx;
+        {
+          float m8[8];
 #pragma unroll
-        for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, s[i]);
+          for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(rr[i]);
+#pragma unroll
+          for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(rr[i]));
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        }
         const float m_tile = mx * sl2;
         const float m_new = (m_tile > m + 8.f) ? m_tile : m;
         const bool rescale = (m_new != m) && (j > 0);
         if (__any_sync(0xffffffffu, rescale)) {
+          // Rare: rescale O and l.  S is reloaded afterwards so it need not stay live here.
           const float fac = rescale ? ex2(m - m_new) : 1.f;
           ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + t], (j - 1) & 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < kHD / 16; ++cc) {
+            uint32_t ro[16];
+            tmem_ld16(tO + cc * 16, ro);
 #pragma unroll
-          for (int cc = 0; cc < kHD / 32; ++cc) {
-            uint32_t rr[32];
-            tmem_ld32(tO + cc * 32, rr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * fac);
-            tmem_st32(tO + cc * 32, rr);
+            for (int i = 0; i < 16; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * fac);
+            tmem_st16(tO + cc * 16, ro);
           }
           l *= fac;
+          tmem_ld128(tS, rr);
+          if (valid < kBN) {
+#pragma unroll
+            for (int i = 0; i < kBN; ++i)
+              if (i >= valid) rr[i] = __float_as_uint(-INFINITY);
+          }
         }
         m = m_new;
-        float rowsum = 0.f;
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pr[32];
+        for (int hh = 0; hh < kBN / 16; ++hh) {  // 16 probabilities -> 8 packed columns per store
+          uint32_t pr[8];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float a = ex2(fmaf(s[hh * 64 + 2 * i], sl2, -m));
-            const float b = ex2(fmaf(s[hh * 64 + 2 * i + 1], sl2, -m));
-            rowsum += a + b;
+          for (int i = 0; i < 8; ++i) {
+            const float a = ex2(fmaf(__uint_as_float(rr[hh * 16 + 2 * i]), sl2, -m));
+            const float b = ex2(fmaf(__uint_as_float(rr[hh * 16 + 2 * i + 1]), sl2, -m));
+            rs[i & 3] += a + b;
             pr[i] = pack_bf16x2(a, b);
           }
-          tmem_st32(tS + hh * 32, pr);
+          tmem_st8(tS + hh * 8, pr);
         }
+        const float rowsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
         l += rowsum;
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars[kPFull + t]);
       }
       // ---- epilogue ----
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + t], (n_kv - 1) & 1, abort_flag));
       if (ok && has_linear) {
-        tc_fence_after();
-        // phi_q(q) * 2^-m overwrites this row of the Q tile (group g reads and writes the same
-        // 16-byte chunks, so reading a group's inputs first makes the update in place safe).
-        uint8_t* qrow = sm + (t ? kOffQ1 : kOffQ0);
-        const float esc = ex2(-m);
-        float lin = 0.f;
+        // U_FULL also means every earlier MMA of this CTA (the last P.V included) is complete.
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kUFull + t], 0, abort_flag));
+        if (ok) {
+          tc_fence_after();
+          // phi_q(q) * 2^-m in bf16 over this row of the Q tile (its last reader, the U MMA, is
+          // done); 16 features per step keeps the loop body small.
+          uint8_t* qrow = sm + (t ? kOffQ1 : kOffQ0);
+          const float esc = ex2(-m);
+          float lin[2] = {0.f, 0.f};
 #pragma unroll 1
-        for (int g = 0; g < G; ++g) {
-          float x[Dg];
+          for (int c16 = 0; c16 < kFD / 16; ++c16) {
+            const int f0 = c16 * 16;
+            uint32_t uu[16];
+            tmem_ld16(tS + f0, uu);
+            uint32_t packed[8];
 #pragma unroll
-          for (int c8 = 0; c8 < Dg / 8; ++c8) {
-            const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + sw128_offset(r, g * Dg + c8 * 8, kBM));
-            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f2 = __bfloat1622float2(b2[e]);
-              x[c8 * 8 + 2 * e] = f2.x;
-              x[c8 * 8 + 2 * e + 1] = f2.y;
-            }
-          }
-#pragma unroll
-          for (int c8 = 0; c8 < Fg / 8; ++c8) {
-            uint32_t packed[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int f2 = 0; f2 < 8; ++f2) {
               float ph2[2];
 #pragma unroll
               for (int q2 = 0; q2 < 2; ++q2) {
-                const int o = c8 * 8 + 2 * e + q2;
-                const int f = g * Fg + o;
-                const float* w = sW + (g * Fg + o) * Dg;
-                float u = sB[f];
-#pragma unroll
-                for (int i = 0; i < Dg; ++i) u = fmaf(w[i], x[i], u);
-                const float ph = int_pow(softplus_fast(u), part_power(f, kFD, p.P)) * esc;
-                const float phr = __bfloat162float(__float2bfloat16_rn(ph));
-                lin = fmaf(phr, sZ[f], lin);
-                ph2[q2] = ph;
+                const int f = f0 + 2 * f2 + q2;
+                const float u = __uint_as_float(uu[2 * f2 + q2]) + sB[f];
+                const float ph = small_pow(softplus_fast(u), sPw[f]) * esc;
+                ph2[q2] = __bfloat162float(__float2bfloat16_rn(ph));
+                lin[q2] = fmaf(ph2[q2], sZ[f], lin[q2]);
               }
-              packed[e] = pack_bf16x2(ph2[0], ph2[1]);
+              packed[f2] = pack_bf16x2(ph2[0], ph2[1]);
             }
-            *reinterpret_cast<uint4*>(qrow + sw128_offset(r, g * Fg + c8 * 8, kBM)) =
+            *reinterpret_cast<uint4*>(qrow + sw128_offset(r, f0, kBM)) =
                 make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            *reinterpret_cast<uint4*>(qrow + sw128_offset(r, f0 + 8, kBM)) =
+                make_uint4(packed[4], packed[5], packed[6], packed[7]);
           }
+          fence_async_smem();
+          tc_fence_before();
+          mbar_arrive(&bars[kPhiFull + t]);
+          l += lin[0] + lin[1];
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars[kRoDone + t], 0, abort_flag));
         }
-        fence_async_smem();
-        mbar_arrive(&bars[kPhiFull + t]);
-        l += lin;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kRoDone + t], 0, abort_flag));
+      } else if (ok) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + t], (n_kv - 1) & 1, abort_flag));
       }
       if (ok) {
         tc_fence_after();

@@ -23,6 +23,17 @@ __device__ __forceinline__ float int_pow(float x, int p) {
   return r;
 }
 
+// x^p without branches for 1 <= p <= 4 (the usual part counts); larger p takes the loop.
+__device__ __forceinline__ float small_pow(float x, int p) {
+  float r = x;
+  const float x2 = x * x;
+  r = (p == 2) ? x2 : r;
+  r = (p == 3) ? x2 * x : r;
+  r = (p == 4) ? x2 * x2 : r;
+  if (p > 4) r = int_pow(x, p);
+  return r;
+}
+
 // softplus(u) = max(u, 0) + log1p(e^{-|u|}) with the CUDA math library's expf/log1pf.
 __device__ __forceinline__ float softplus_accurate(float u) {
   return fmaxf(u, 0.f) + log1pf(expf(-fabsf(u)));
@@ -98,6 +109,42 @@ __global__ void __launch_bounds__(128) featmap_kernel(const Tin* __restrict__ x,
       out[f] = from_f32<Tout>(int_pow(sp, part_power(f, F, P)));
     }
   }
+}
+
+// Block-diagonal form of the grouped linear for the tensor cores: for head h, the dense
+// F x D matrix Wbd[f][d] = W[g][f - g F/G][d - g D/G] when d lies in f's group g, else 0, split
+// into bf16 hi = bf16(Wbd) and lo = bf16(Wbd - hi) so that x.Wbd^T from two bf16 MMAs with fp32
+// accumulation carries about 16 mantissa bits of W.
+//   out [H][2][F][D] bf16 (hi at [h][0], lo at [h][1]).
+//   grid (ceil(F*D / 2048), H), block 256: each thread writes 8 consecutive d of one f.
+__global__ void __launch_bounds__(256) blockdiag_weights_kernel(const float* __restrict__ W, int D,
+                                                                int F, int G,
+                                                                __nv_bfloat16* __restrict__ out) {
+  const int h = blockIdx.y;
+  const int Dg = D / G, Fg = F / G;
+  const int e0 = (blockIdx.x * 256 + threadIdx.x) * 8;
+  if (e0 >= F * D) return;
+  const int f = e0 / D, d0 = e0 - f * D;  // D % 8 == 0, so the 8 elements share f
+  const int g = f / Fg;
+  const float* Wrow = W + (size_t)h * F * Dg + (size_t)f * Dg;
+  uint32_t hi2[4], lo2[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float w[2], r[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int d = d0 + 2 * q + e;
+      w[e] = (d / Dg == g) ? Wrow[d - g * Dg] : 0.f;
+      r[e] = w[e] - __bfloat162float(__float2bfloat16_rn(w[e]));
+    }
+    __nv_bfloat162 hv = __floats2bfloat162_rn(w[0], w[1]);
+    __nv_bfloat162 lv = __floats2bfloat162_rn(r[0], r[1]);
+    hi2[q] = *reinterpret_cast<uint32_t*>(&hv);
+    lo2[q] = *reinterpret_cast<uint32_t*>(&lv);
+  }
+  __nv_bfloat16* hi = out + (size_t)h * 2 * F * D;
+  *reinterpret_cast<uint4*>(hi + e0) = make_uint4(hi2[0], hi2[1], hi2[2], hi2[3]);
+  *reinterpret_cast<uint4*>(hi + (size_t)F * D + e0) = make_uint4(lo2[0], lo2[1], lo2[2], lo2[3]);
 }
 
 }  // namespace rehyat

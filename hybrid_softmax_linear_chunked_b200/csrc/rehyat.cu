@@ -62,8 +62,6 @@ int check_path_shape(const rehyat_dims& d, rehyat_dtype dt) {
   if (dt == REHYAT_BF16) {
     if (d.D != 128 || d.F != 128)
       return fail(REHYAT_ERR_SHAPE, "bf16 path needs D = F = 128 (got D=%d F=%d)", d.D, d.F);
-    if (d.G != 4 && d.G != 8 && d.G != 16)
-      return fail(REHYAT_ERR_SHAPE, "bf16 path supports G in {4, 8, 16} (got %d)", d.G);
   } else {
     if (d.D % 32 || d.D > rehyat::fp32::kMaxD || d.F > 256)
       return fail(REHYAT_ERR_SHAPE, "fp32 path needs D %% 32 == 0, D <= 256, F <= 256 (D=%d F=%d)",
@@ -141,7 +139,7 @@ int fold_splits(int BH, int n_fold, long long rows_per_fold) {
 
 struct ForwardPlan {
   int C, n_fold, splits;
-  size_t dS, dZ, St, Zc, phiq, phik, Sc, total;
+  size_t dS, dZ, St, Zc, Wqbd, Wkbd, phiq, phik, Sc, total;
 };
 
 ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, int Tc, int To) {
@@ -157,6 +155,8 @@ ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, in
     p.dZ = cv.take(BH * nf * p.splits * d.F * 4);
     p.St = cv.take(BH * p.C * d.D * d.F * 2);
     p.Zc = cv.take(BH * p.C * d.F * 4);
+    p.Wqbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
+    p.Wkbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
   } else {
     p.splits = 1;
     const size_t N = (size_t)T * L;
@@ -174,7 +174,7 @@ ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, in
 
 struct ChunkPlan {
   int o, nq, nkv, fold_rows, splits;
-  size_t St, dS, dZ, phiq, phik, total;
+  size_t St, dS, dZ, Wqbd, Wkbd, phiq, phik, total;
 };
 
 ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_before,
@@ -197,6 +197,8 @@ ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_be
     p.St = cv.take(BH * d.D * d.F * 2);
     p.dS = cv.take(BH * p.splits * d.F * d.D * 4);
     p.dZ = cv.take(BH * p.splits * d.F * 4);
+    p.Wqbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
+    p.Wkbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
   } else {
     p.splits = 1;
     const size_t max_kv = (size_t)(To + chunk_frames) * L;
@@ -233,48 +235,35 @@ int launch_featmap(const rehyat_dims& d, rehyat_dtype dt, int n, const void* x, 
   return cuda_check(cudaGetLastError(), "featmap launch");
 }
 
-template <int G>
-int launch_attn_bf16_g(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const CUtensorMap& ms, const rehyat::attn::Params& ap, dim3 grid,
-                       cudaStream_t st) {
-  auto k = rehyat::attn::hybrid_attn_bf16_kernel<G>;
+int launch_attn_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& ms, const CUtensorMap& mw, const rehyat::attn::Params& ap,
+                     dim3 grid, cudaStream_t st) {
+  auto k = rehyat::attn::hybrid_attn_bf16_kernel;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)rehyat::attn::kSmemBytes),
                     "attn attr"));
-  k<<<grid, rehyat::attn::kThreads, rehyat::attn::kSmemBytes, st>>>(mq, mk, mv, ms, ap);
+  k<<<grid, rehyat::attn::kThreads, rehyat::attn::kSmemBytes, st>>>(mq, mk, mv, ms, mw, ap);
   return cuda_check(cudaGetLastError(), "attention launch");
 }
 
-int launch_attn_bf16(int G, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const CUtensorMap& ms, const rehyat::attn::Params& ap, dim3 grid,
-                     cudaStream_t st) {
-  switch (G) {
-    case 4: return launch_attn_bf16_g<4>(mq, mk, mv, ms, ap, grid, st);
-    case 8: return launch_attn_bf16_g<8>(mq, mk, mv, ms, ap, grid, st);
-    case 16: return launch_attn_bf16_g<16>(mq, mk, mv, ms, ap, grid, st);
-  }
-  return fail(REHYAT_ERR_SHAPE, "unsupported G=%d", G);
-}
-
-template <int G>
-int launch_fold_bf16_g(const CUtensorMap& mk, const CUtensorMap& mv,
-                       const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st) {
-  auto k = rehyat::state::fold_partial_bf16_kernel<G>;
+int launch_fold_bf16(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mw,
+                     const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st) {
+  auto k = rehyat::state::fold_partial_bf16_kernel;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)rehyat::state::kSmemBytes),
                     "fold attr"));
-  k<<<grid, rehyat::state::kThreads, rehyat::state::kSmemBytes, st>>>(mk, mv, fp);
+  k<<<grid, rehyat::state::kThreads, rehyat::state::kSmemBytes, st>>>(mk, mv, mw, fp);
   return cuda_check(cudaGetLastError(), "fold launch");
 }
 
-int launch_fold_bf16(int G, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st) {
-  switch (G) {
-    case 4: return launch_fold_bf16_g<4>(mk, mv, fp, grid, st);
-    case 8: return launch_fold_bf16_g<8>(mk, mv, fp, grid, st);
-    case 16: return launch_fold_bf16_g<16>(mk, mv, fp, grid, st);
-  }
-  return fail(REHYAT_ERR_SHAPE, "unsupported G=%d", G);
+// Block-diagonal bf16 hi/lo weights of one feature map into `out` ([H][2][F][D] bf16) and the
+// tensor map the kernels load them with.
+int prepare_blockdiag(const rehyat_dims& d, const float* W, __nv_bfloat16* out, CUtensorMap* map,
+                      cudaStream_t st) {
+  rehyat::blockdiag_weights_kernel<<<dim3((d.F * d.D + 2047) / 2048, d.H), 256, 0, st>>>(
+      W, d.D, d.F, d.G, out);
+  RH_TRY(cuda_check(cudaGetLastError(), "block-diagonal weights launch"));
+  return make_map(map, out, d.D, d.F, 2LL * d.H);
 }
 
 int launch_scan_bf16(const rehyat_dims& d, const float* dS, const float* dZ, int n_fold,
@@ -296,14 +285,15 @@ int forward_states_bf16(const rehyat_dims& d, int T, int L, int Tc, int To, cons
   float* dS = reinterpret_cast<float*>(ws + pl.dS);
   float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
   if (pl.n_fold > 0) {
-    CUtensorMap mk, mv;
+    CUtensorMap mk, mv, mw;
     RH_TRY(make_map(&mk, k, d.D, N, BH));
     RH_TRY(make_map(&mv, v, d.D, N, BH));
+    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mw, st));
     rehyat::state::FoldParams fp{};
     fp.L = L; fp.H = d.H; fp.P = d.P; fp.T = T; fp.Tc = Tc; fp.To = To; fp.kv_frame0 = 0;
     fp.single_rows = -1; fp.n_fold = pl.n_fold; fp.splits = pl.splits;
-    fp.Wk = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
-    RH_TRY(launch_fold_bf16(d.G, mk, mv, fp, dim3(pl.splits, pl.n_fold, BH), st));
+    fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(mk, mv, mw, fp, dim3(pl.splits, pl.n_fold, BH), st));
   }
   return launch_scan_bf16(d, dS, dZ, pl.n_fold, pl.splits, pl.C, nullptr, nullptr, St, Zc, S_out,
                           Z_out, st);
@@ -439,19 +429,20 @@ int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
   const long long N = (long long)T * L;
   const int rows_per_chunk = (Tc < T ? Tc : T) * L;
   if (dt == REHYAT_BF16) {
-    CUtensorMap mq, mk, mv, ms;
+    CUtensorMap mq, mk, mv, ms, mw;
     RH_TRY(make_map(&mq, q, d.D, N, BH));
     RH_TRY(make_map(&mk, k, d.D, N, BH));
     RH_TRY(make_map(&mv, v, d.D, N, BH));
     RH_TRY(make_map(&ms, ws + pl.St, d.F, d.D, (long long)BH * pl.C));
+    RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mw, st));
     rehyat::attn::Params ap{};
     ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
     ap.H = d.H; ap.P = d.P; ap.n_states = pl.C; ap.nq_rows = (int)N;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
-    ap.Wq = Wq; ap.bq = bq; ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
+    ap.bq = bq; ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
     ap.out = static_cast<__nv_bfloat16*>(out);
     dim3 grid((rows_per_chunk + 255) / 256, pl.C, BH);
-    return launch_attn_bf16(d.G, mq, mk, mv, ms, ap, grid, st);
+    return launch_attn_bf16(mq, mk, mv, ms, mw, ap, grid, st);
   }
   float* phiq = reinterpret_cast<float*>(ws + pl.phiq);
   RH_TRY(launch_featmap(d, REHYAT_F32, (int)N, q, Wq, bq, phiq, st));
@@ -524,23 +515,25 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int L, int frames_befor
     float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
     // S^T in bf16 for the readout MMA (C = 1, no folds: a transposed copy of S)
     RH_TRY(launch_scan_bf16(d, dS, dZ, 0, 1, 1, S, Z, St, nullptr, nullptr, nullptr, st));
-    CUtensorMap mq, mk, mv, ms;
+    CUtensorMap mq, mk, mv, ms, mwq, mwk;
     RH_TRY(make_map(&mq, q, d.D, pl.nq, BH));
     RH_TRY(make_map(&mk, k_win, d.D, pl.nkv, BH));
     RH_TRY(make_map(&mv, v_win, d.D, pl.nkv, BH));
     RH_TRY(make_map(&ms, St, d.F, d.D, BH));
+    RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mwq, st));
     rehyat::attn::Params ap{};
     ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
     ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
     ap.H = d.H; ap.P = d.P; ap.n_states = 1; ap.nq_rows = pl.nq;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
-    ap.Wq = Wq; ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
-    RH_TRY(launch_attn_bf16(d.G, mq, mk, mv, ms, ap, dim3((pl.nq + 255) / 256, 1, BH), st));
+    ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
+    RH_TRY(launch_attn_bf16(mq, mk, mv, ms, mwq, ap, dim3((pl.nq + 255) / 256, 1, BH), st));
     if (pl.fold_rows > 0) {
+      RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
       rehyat::state::FoldParams fp{};
       fp.L = L; fp.H = d.H; fp.P = d.P; fp.single_rows = pl.fold_rows; fp.n_fold = 1;
-      fp.splits = pl.splits; fp.Wk = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
-      RH_TRY(launch_fold_bf16(d.G, mk, mv, fp, dim3(pl.splits, 1, BH), st));
+      fp.splits = pl.splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+      RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(pl.splits, 1, BH), st));
       rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
           dS, dZ, pl.splits, d.F, d.D, S, Z);
       RH_TRY(cuda_check(cudaGetLastError(), "state add launch"));
@@ -596,8 +589,10 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   ChunkPlan pl = plan_chunk(d, dt, L, frames_before, chunk_frames, To);
   const size_t BH = (size_t)d.B * d.H;
   const size_t st_bytes = round_up(BH * d.D * d.F * 2, 256);
+  const size_t wbd_bytes = round_up((size_t)d.H * 2 * d.F * d.D * 2, 256);
   auto total_for = [&](int splits) {
-    return st_bytes + round_up(BH * splits * d.F * d.D * 4, 256) + round_up(BH * splits * d.F * 4, 256);
+    return st_bytes + 2 * wbd_bytes + round_up(BH * splits * d.F * d.D * 4, 256) +
+           round_up(BH * splits * d.F * 4, 256);
   };
   int splits = pl.splits;
   while (splits > 1 && total_for(splits) > kStaticScratchBytes) --splits;
@@ -609,30 +604,35 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   RH_TRY(static_scratch_for_current_device(&scratch));
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   __nv_bfloat16* St = reinterpret_cast<__nv_bfloat16*>(ws);
-  float* dS = reinterpret_cast<float*>(ws + st_bytes);
-  float* dZ = reinterpret_cast<float*>(ws + st_bytes + round_up(BH * splits * d.F * d.D * 4, 256));
+  __nv_bfloat16* Wqbd = reinterpret_cast<__nv_bfloat16*>(ws + st_bytes);
+  __nv_bfloat16* Wkbd = reinterpret_cast<__nv_bfloat16*>(ws + st_bytes + wbd_bytes);
+  float* dS = reinterpret_cast<float*>(ws + st_bytes + 2 * wbd_bytes);
+  float* dZ = reinterpret_cast<float*>(ws + st_bytes + 2 * wbd_bytes +
+                                       round_up(BH * splits * d.F * d.D * 4, 256));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int nbh = d.B * d.H;
   // Nothing in the scratch has to start at zero: every byte a kernel reads was written earlier
   // in this call (S^T by the scan, every split's partial by the fold kernel).
   RH_TRY(launch_scan_bf16(d, dS, dZ, 0, 1, 1, S, Z, St, nullptr, nullptr, nullptr, st));
-  CUtensorMap mq, mk, mv, ms;
+  CUtensorMap mq, mk, mv, ms, mwq, mwk;
   RH_TRY(make_map(&mq, q, d.D, pl.nq, nbh));
   RH_TRY(make_map(&mk, k_win, d.D, pl.nkv, nbh));
   RH_TRY(make_map(&mv, v_win, d.D, pl.nkv, nbh));
   RH_TRY(make_map(&ms, St, d.F, d.D, nbh));
+  RH_TRY(prepare_blockdiag(d, Wq, Wqbd, &mwq, st));
   rehyat::attn::Params ap{};
   ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
   ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
   ap.H = d.H; ap.P = d.P; ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
-  ap.Wq = Wq; ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
-  RH_TRY(launch_attn_bf16(d.G, mq, mk, mv, ms, ap, dim3((pl.nq + 255) / 256, 1, nbh), st));
+  ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
+  RH_TRY(launch_attn_bf16(mq, mk, mv, ms, mwq, ap, dim3((pl.nq + 255) / 256, 1, nbh), st));
   if (pl.fold_rows > 0) {
+    RH_TRY(prepare_blockdiag(d, Wk, Wkbd, &mwk, st));
     rehyat::state::FoldParams fp{};
     fp.L = L; fp.H = d.H; fp.P = d.P; fp.single_rows = pl.fold_rows; fp.n_fold = 1;
-    fp.splits = splits; fp.Wk = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
-    RH_TRY(launch_fold_bf16(d.G, mk, mv, fp, dim3(splits, 1, nbh), st));
+    fp.splits = splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(splits, 1, nbh), st));
     rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, nbh), 256, 0, st>>>(
         dS, dZ, splits, d.F, d.D, S, Z);
     RH_TRY(cuda_check(cudaGetLastError(), "state add launch"));

@@ -3,9 +3,10 @@
 //
 //  * fold_partial_bf16_kernel: for one fold range of key rows (the frames leaving a chunk's
 //    softmax window) and one split of it, dS = phi_k(K)^T V (F x D) and dZ = phi_k(K)^T 1 on the
-//    tensor cores: phi_k is computed by the CUDA cores from the TMA-loaded K tile straight into
-//    shared memory in the layout of an MN-major MMA operand, and both products accumulate in
-//    TMEM in fp32 over the split's 128-token tiles.
+//    tensor cores.  The grouped linear of phi_k is a tensor-core product too (block-diagonal
+//    weights); the CUDA cores apply bias, softplus and powers and write phi_k straight into the
+//    shared-memory layout of an MN-major MMA operand; both sums accumulate in TMEM in fp32 over
+//    the split's 128-token tiles.
 //  * state_scan_kernel: exclusive prefix over fold ranges (the state chunk c reads), written as
 //    a transposed bf16 copy S_c^T [D][F] for the attention kernel's readout MMA, plus fp32 Z_c
 //    (and fp32 S_c on request).
@@ -23,22 +24,25 @@ using namespace sm100;
 constexpr int kTok = 128;  // tokens per tile (MMA K)
 constexpr int kHD = 128;
 constexpr int kFD = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // warps 0-7 feature map, 8 producer, 9 MMA
+constexpr int kPhiThreads = 256;
 constexpr int kTileBytes = kTok * kHD * 2;
 
-constexpr uint32_t kOffK = 0;                          // 2 stages
-constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;      // 2 stages
-constexpr uint32_t kOffPhi = kOffV + 2 * kTileBytes;    // 2 stages
-constexpr uint32_t kOffOnes = kOffPhi + 2 * kTileBytes; // 16 x 128 bf16 of 1.0
-constexpr int kMinG = 4;                                 // smallest supported group count
-constexpr uint32_t kOffW = kOffOnes + 4096;             // W_k of the head (F * D / G fp32)
-constexpr uint32_t kWBytesMax = kFD * kHD / kMinG * 4;
-constexpr uint32_t kOffB = kOffW + kWBytesMax;          // bias
-constexpr uint32_t kSmemBytes = kOffB + kFD * 4 + 1024;
+constexpr uint32_t kOffK = 0;                           // 1 stage (consumed early by the U MMA)
+constexpr uint32_t kOffV = kOffK + kTileBytes;           // 2 stages
+constexpr uint32_t kOffPhi = kOffV + 2 * kTileBytes;     // 2 stages
+constexpr uint32_t kOffW = kOffPhi + 2 * kTileBytes;     // block-diagonal W_k, hi and lo
+constexpr uint32_t kOffOnes = kOffW + 2 * kTileBytes;    // 8 rows x 128 B of bf16 1.0
+constexpr uint32_t kOffB = kOffOnes + 1024;              // bias of phi_k, F fp32
+constexpr uint32_t kOffPw = kOffB + kFD * 4;             // part power of each feature, uint8
+constexpr uint32_t kSmemBytes = kOffPw + kFD + 1024;      // + alignment slack
+
+// TMEM columns: U buffers [0,128) and [128,256), dS [256,384), dZ [384,400).
+constexpr uint32_t kColDS = 256, kColDZ = 384;
 
 enum Bar {
-  kKFull = 0, kKEmpty = 2, kVFull = 4, kVEmpty = 6, kPhiFull = 8, kPhiEmpty = 10, kDone = 12,
-  kNumBars = 13
+  kKFull = 0, kKEmpty = 1, kVFull = 2, kVEmpty = 4, kUFull = 6, kUEmpty = 8, kPhiFull = 10,
+  kPhiEmpty = 12, kWbFull = 14, kDone = 15, kNumBars = 16
 };
 
 struct FoldParams {
@@ -46,7 +50,6 @@ struct FoldParams {
   int T, Tc, To, kv_frame0;  // schedule (mode 0)
   int single_rows;           // mode 1: fold rows [0, single_rows) of the k/v buffer; -1 = mode 0
   int n_fold, splits;
-  const float* Wk;
   const float* bk;
   float* dS;  // [BH][n_fold][splits][F][D]
   float* dZ;  // [BH][n_fold][splits][F]
@@ -56,16 +59,27 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// grid (splits, n_fold, BH), block 192: warps 0-3 feature map (one token per thread), warp 4
-// TMA producer, warp 5 MMA issuer (both run their loop warp-wide; lane 0 issues).
-// TMEM: dS in columns [0, 128), dZ in [128, 144).
-template <int G>
+// K-major SW128 descriptor of the kk-th 16-wide K step of a 128 x 128 bf16 tile.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_addr, int kk) {
+  return sdesc_sw128(tile_addr + (kk >> 2) * (kTok * 128) + (kk & 3) * 32, 16, 1024);
+}
+// MN-major SW128 descriptor of the kk-th 16-row K step of a [128 rows][128 cols] bf16 tile.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_addr, int kk) {
+  return sdesc_sw128(tile_addr + kk * 16 * 128, kTok * 128, 1024);
+}
+
+// grid (splits, n_fold, BH), block 320: warps 0-7 feature map (token row = TMEM lane
+// 32*(warp%4) + lane; warps 0-3 take features 0-63, warps 4-7 features 64-127), warp 8 TMA
+// producer, warp 9 MMA issuer (both run their loop warp-wide; lane 0 issues).
+// Per 128-token tile i: U = K_i Wbd_hi^T + K_i Wbd_lo^T (grouped linear of phi_k on the tensor
+// cores, fp32 in TMEM); the feature-map warps add the bias, apply softplus and the part powers,
+// and write phi_k as bf16 into the MN-major A operand of dS += phi_k^T V_i and
+// dZ += phi_k^T 1 (a ones matrix as B: N = 16, every row group read from the same 1 KiB).
 __global__ void __launch_bounds__(kThreads, 1)
     fold_partial_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
-                             const __grid_constant__ CUtensorMap tmV, const FoldParams p) {
-  constexpr int Dg = kHD / G, Fg = kFD / G;
-  static_assert(G >= kMinG && kFD * Dg * 4 <= kWBytesMax, "W_k does not fit its shared-memory slot");
-  static_assert(kSmemBytes <= 232448, "shared memory over the per-CTA limit");
+                             const __grid_constant__ CUtensorMap tmV,
+                             const __grid_constant__ CUtensorMap tmW, const FoldParams p) {
+  static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
   const int split = blockIdx.x, fc = blockIdx.y, bh = blockIdx.z, h = bh % p.H;
   int r0, r1;
   if (p.single_rows >= 0) {
@@ -95,53 +109,64 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   volatile int* abort_flag = &abort_sh;
-  float* sW = reinterpret_cast<float*>(sm + kOffW);
   float* sB = reinterpret_cast<float*>(sm + kOffB);
+  uint8_t* sPw = sm + kOffPw;
 
-  if (warp == 4) {
-    tmem_alloc(&tmem_base_sh, 256);
+  if (warp == 8) {
+    tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) {
-      const bool many = (i == kKEmpty || i == kKEmpty + 1 || i == kPhiFull || i == kPhiFull + 1);
-      mbar_init(&bars[i], many ? 128 : 1);
+      const bool many = (i == kUEmpty || i == kUEmpty + 1 || i == kPhiFull || i == kPhiFull + 1);
+      mbar_init(&bars[i], many ? kPhiThreads : 1);
     }
     abort_sh = 0;
     fence_mbar_init();
   }
+  for (int i = tid; i < kFD; i += kThreads) {
+    sB[i] = p.bk ? p.bk[(size_t)h * kFD + i] : 0.f;
+    sPw[i] = static_cast<uint8_t>(part_power(i, kFD, p.P));
+  }
   {
-    const float* Wh = p.Wk + (size_t)h * kFD * Dg;
-    for (int i = tid; i < kFD * Dg; i += kThreads) sW[i] = Wh[i];
-    for (int i = tid; i < kFD; i += kThreads) sB[i] = p.bk ? p.bk[(size_t)h * kFD + i] : 0.f;
     uint32_t* ones = reinterpret_cast<uint32_t*>(sm + kOffOnes);
-    for (int i = tid; i < 1024; i += kThreads) ones[i] = 0x3F803F80u;  // bf16 pair (1.0, 1.0)
+    for (int i = tid; i < 256; i += kThreads) ones[i] = 0x3F803F80u;  // bf16 pair (1.0, 1.0)
   }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  const uint32_t sK0 = smem_u32(sm + kOffK), sV0 = smem_u32(sm + kOffV);  // one K stage
+  const uint32_t sPhi = smem_u32(sm + kOffPhi), sW0 = smem_u32(sm + kOffW);
+  const uint32_t sOnes = smem_u32(sm + kOffOnes);
 
   const bool leader = lane == 0;
-  if (warp == 4) {
+  if (warp == 8) {
     // ---- producer ----
     if (leader) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bars[kWbFull], 2 * kTileBytes);
+      for (int part = 0; part < 2; ++part) {
+        uint8_t* dst = sm + kOffW + part * kTileBytes;
+        tma_load_3d(dst, &tmW, &bars[kWbFull], 0, 0, h * 2 + part);
+        tma_load_3d(dst + kTok * 128, &tmW, &bars[kWbFull], 64, 0, h * 2 + part);
+      }
     }
+    __syncwarp();
     bool ok = true;
     int issued_k = 0, issued_v = 0;
     for (int i = 0; i < n_tiles; ++i) {
       const int s = i & 1;
       const int row = r0 + (t_begin + i) * kTok;
-      if (i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty + s], ((i >> 1) - 1) & 1, abort_flag));
+      if (i >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty], (i - 1) & 1, abort_flag));
       if (!ok) break;
       if (leader) {
-        uint8_t* dk = sm + kOffK + s * kTileBytes;
-        mbar_arrive_expect_tx(&bars[kKFull + s], kTileBytes);
-        tma_load_3d(dk, &tmK, &bars[kKFull + s], 0, row, bh);
-        tma_load_3d(dk + kTok * 128, &tmK, &bars[kKFull + s], 64, row, bh);
+        uint8_t* dk = sm + kOffK;
+        mbar_arrive_expect_tx(&bars[kKFull], kTileBytes);
+        tma_load_3d(dk, &tmK, &bars[kKFull], 0, row, bh);
+        tma_load_3d(dk + kTok * 128, &tmK, &bars[kKFull], 64, row, bh);
       }
       __syncwarp();
       ++issued_k;
@@ -157,123 +182,139 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++issued_v;
     }
     if (!ok) {
-      for (int i = max(0, issued_k - 2); i < issued_k; ++i)
-        mbar_wait_drain(&bars[kKFull + (i & 1)], (i >> 1) & 1);
+      mbar_wait_drain(&bars[kWbFull], 0);
+      if (issued_k > 0) mbar_wait_drain(&bars[kKFull], (issued_k - 1) & 1);
       for (int i = max(0, issued_v - 2); i < issued_v; ++i)
         mbar_wait_drain(&bars[kVFull + (i & 1)], (i >> 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---- MMA issuer ----
-    const uint32_t id_s = idesc_bf16(kFD, kHD, true, true);
-    const uint32_t id_z = idesc_bf16(kFD, 16, true, false);
-    const uint32_t ones = smem_u32(sm + kOffOnes);
-    bool ok = true;
-    for (int i = 0; i < n_tiles; ++i) {
+    const uint32_t id_u = idesc_bf16(kTok, kFD, false, false);  // K (K-major) x Wbd (K-major)
+    const uint32_t id_s = idesc_bf16(kFD, kHD, true, true);     // phi^T (MN) x V (MN)
+    const uint32_t id_z = idesc_bf16(kFD, 16, true, false);     // phi^T (MN) x ones (K)
+    auto wait = [&](int b, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, abort_flag));
+    };
+    auto issue_fold = [&](int i) {  // dS, dZ += tile i (phi and V in stage i & 1)
+      if (leader) {
+        const uint32_t vb = sV0 + (i & 1) * kTileBytes;
+        const uint32_t pb = sPhi + (i & 1) * kTileBytes;
+        for (int kk = 0; kk < kTok / 16; ++kk) {
+          const uint64_t a = mnmajor_desc(pb, kk);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          mma_ss(tmem + kColDS, a, mnmajor_desc(vb, kk), id_s, acc);
+          // ones: SBO = 0 so both 8-row groups of the 16 B rows read the same 1 KiB
+          mma_ss(tmem + kColDZ, a, sdesc_sw128(sOnes + (kk & 3) * 32, 16, 0), id_z, acc);
+        }
+        mma_commit(&bars[kPhiEmpty + (i & 1)]);
+        mma_commit(&bars[kVEmpty + (i & 1)]);
+      }
+      __syncwarp();
+    };
+    bool ok = wait(kWbFull, 0);
+    for (int i = 0; i < n_tiles && ok; ++i) {
       const int s = i & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kPhiFull + s], (i >> 1) & 1, abort_flag) &&
-                                       mbar_wait(&bars[kVFull + s], (i >> 1) & 1, abort_flag));
+      ok = wait(kKFull, i & 1);
+      if (ok && i >= 2) ok = wait(kUEmpty + s, ((i >> 1) - 1) & 1);
       if (!ok) break;
       tc_fence_after();
       if (leader) {
-        const uint32_t ph = smem_u32(sm + kOffPhi + s * kTileBytes);
-        const uint32_t vb = smem_u32(sm + kOffV + s * kTileBytes);
-        for (int kk = 0; kk < kTok / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(ph + kk * 16 * 128, kTok * 128, 1024);
-          mma_ss(tmem, a, sdesc_sw128(vb + kk * 16 * 128, kTok * 128, 1024), id_s,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-          mma_ss(tmem + 128, a,
-                 sdesc_sw128(ones + (kk >> 2) * (16 * 128) + (kk & 3) * 32, 16, 1024), id_z,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars[kPhiEmpty + s]);
-        mma_commit(&bars[kVEmpty + s]);
+        for (int part = 0; part < 2; ++part)
+          for (int kk = 0; kk < kHD / 16; ++kk)
+            mma_ss(tmem + s * 128, kmajor_desc(sK0, kk), kmajor_desc(sW0 + part * kTileBytes, kk),
+                   id_u, (part > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[kUFull + s]);
+        mma_commit(&bars[kKEmpty]);
       }
       __syncwarp();
+      if (i >= 1) {
+        const int ip = i - 1;
+        ok = wait(kPhiFull + (ip & 1), (ip >> 1) & 1) && wait(kVFull + (ip & 1), (ip >> 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_fold(i - 1);
+      }
+    }
+    if (ok) {
+      const int i = n_tiles - 1;
+      ok = wait(kPhiFull + (i & 1), (i >> 1) & 1) && wait(kVFull + (i & 1), (i >> 1) & 1);
+      if (ok) {
+        tc_fence_after();
+        issue_fold(i);
+      }
     }
     if (leader) mma_commit(&bars[kDone]);
     __syncwarp();
     mbar_wait_drain(&bars[kDone], 0);
     __syncwarp();
   } else {
-    // ---- feature map warps: thread tid owns token row tid of each tile ----
-    const int r = tid;
+    // ---- feature-map warps: token row r = TMEM lane, feature half hf ----
+    const int r = tid & 127, hf = tid >> 7;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t col0 = hf * 64;
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
       const int s = i & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKFull + s], (i >> 1) & 1, abort_flag));
-      if (ok && i >= 2)
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kUFull + s], (i >> 1) & 1, abort_flag));
+      if (ok && i >= 2)  // the fold of tile i - 2 has read this phi stage
         ok = __all_sync(0xffffffffu, mbar_wait(&bars[kPhiEmpty + s], ((i >> 1) - 1) & 1, abort_flag));
       if (!ok) break;
-      const uint8_t* krow = sm + kOffK + s * kTileBytes;
+      tc_fence_after();
       uint8_t* prow = sm + kOffPhi + s * kTileBytes;
       const bool valid = r0 + (t_begin + i) * kTok + r < r1;
 #pragma unroll 1
-      for (int g = 0; g < G; ++g) {
-        float x[Dg];
+      for (int c16 = 0; c16 < 4; ++c16) {  // 16 features per step keeps the loop body small
+        const int f0 = col0 + c16 * 16;
+        uint32_t uu[16];
+        tmem_ld16(tmem + lane_base + s * 128 + f0, uu);
+        uint32_t packed[8];
 #pragma unroll
-        for (int c8 = 0; c8 < Dg / 8; ++c8) {
-          const uint4 v4 = *reinterpret_cast<const uint4*>(krow + sw128_offset(r, g * Dg + c8 * 8, kTok));
-          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
+        for (int f2 = 0; f2 < 8; ++f2) {
+          float ph[2];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f2 = __bfloat1622float2(b2[e]);
-            x[c8 * 8 + 2 * e] = f2.x;
-            x[c8 * 8 + 2 * e + 1] = f2.y;
+          for (int q2 = 0; q2 < 2; ++q2) {
+            const int f = f0 + 2 * f2 + q2;
+            const float u = __uint_as_float(uu[2 * f2 + q2]) + sB[f];
+            ph[q2] = small_pow(softplus_fast(u), sPw[f]);
           }
+          packed[f2] = valid ? pack_bf16x2(ph[0], ph[1]) : 0u;
         }
-#pragma unroll
-        for (int c8 = 0; c8 < Fg / 8; ++c8) {
-          uint32_t packed[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float ph2[2];
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-              const int o = c8 * 8 + 2 * e + q2;
-              const int f = g * Fg + o;
-              const float* w = sW + (g * Fg + o) * Dg;
-              float u = sB[f];
-#pragma unroll
-              for (int k2 = 0; k2 < Dg; ++k2) u = fmaf(w[k2], x[k2], u);
-              ph2[q2] = valid ? int_pow(softplus_fast(u), part_power(f, kFD, p.P)) : 0.f;
-            }
-            packed[e] = pack_bf16x2(ph2[0], ph2[1]);
-          }
-          *reinterpret_cast<uint4*>(prow + sw128_offset(r, g * Fg + c8 * 8, kTok)) =
-              make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        }
+        *reinterpret_cast<uint4*>(prow + sw128_offset(r, f0, kTok)) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        *reinterpret_cast<uint4*>(prow + sw128_offset(r, f0 + 8, kTok)) =
+            make_uint4(packed[4], packed[5], packed[6], packed[7]);
       }
+      tc_fence_before();
+      mbar_arrive(&bars[kUEmpty + s]);
       fence_async_smem();
-      mbar_arrive(&bars[kKEmpty + s]);
       mbar_arrive(&bars[kPhiFull + s]);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0, abort_flag));
     if (ok) {
       tc_fence_after();
-      // lane r of TMEM is feature f = r: dS row f (128 columns), dZ in column 128.
-      const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;  // warps 0-3
-      float* srow = dS + (size_t)r * kHD;
+      // lane r of TMEM is feature f = r: dS row f (this thread writes columns col0 .. col0+63),
+      // dZ in column kColDZ.
+      float* srow = dS + (size_t)r * kHD + col0;
+      uint32_t rr[64];
+      tmem_ld64(tmem + lane_base + kColDS + col0, rr);
 #pragma unroll
-      for (int cc = 0; cc < kHD / 32; ++cc) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_base + cc * 32, rr);
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          *reinterpret_cast<float4*>(srow + cc * 32 + q4 * 4) =
-              make_float4(__uint_as_float(rr[q4 * 4]), __uint_as_float(rr[q4 * 4 + 1]),
-                          __uint_as_float(rr[q4 * 4 + 2]), __uint_as_float(rr[q4 * 4 + 3]));
+      for (int q4 = 0; q4 < 16; ++q4)
+        *reinterpret_cast<float4*>(srow + q4 * 4) =
+            make_float4(__uint_as_float(rr[q4 * 4]), __uint_as_float(rr[q4 * 4 + 1]),
+                        __uint_as_float(rr[q4 * 4 + 2]), __uint_as_float(rr[q4 * 4 + 3]));
+      if (hf == 0) {  // warps 0-3
+        uint32_t z16[16];
+        tmem_ld16(tmem + lane_base + kColDZ, z16);
+        dZ[r] = __uint_as_float(z16[0]);
       }
-      uint32_t z16[16];
-      tmem_ld16(tmem + lane_base + 128, z16);
-      dZ[r] = __uint_as_float(z16[0]);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 

@@ -54,7 +54,7 @@ def call_forward(lib, d, dt=rb.REHYAT_BF16, T=7, L=64, Tc=3, To=1, ws_bytes=1 <<
     (dict(d=dims(G=3)), -1),
     (dict(d=dims(P=200)), -1),
     (dict(d=dims(D=64, F=64)), -2),
-    (dict(d=dims(G=2)), -2),
+    (dict(d=dims(F=64)), -2),
     (dict(d=dims(), dt=7), -3),
     (dict(d=dims(), Tc=0), -1),
     (dict(d=dims(), To=-1), -1),

@@ -192,6 +192,8 @@ SMALL = [
     (4, 8, 8, 4, 1, 2, 8, 1, 1, 1.0, 0.0),      # one chunk: plain softmax attention
     (9, 1, 17, 2, 3, 2, 4, 1, 2, 2.0, 0.0),     # 17-token frames, To > Tc, k x 2, G = 4
     (6, 16, 16, 3, 1, 2, 16, 1, 1, 1.0, 0.0),   # 256-token frames (tile-aligned), G = 16
+    (6, 8, 16, 2, 1, 2, 2, 1, 1, 1.0, 0.0),     # G = 2 (wide groups)
+    (5, 8, 16, 2, 1, 2, 1, 1, 1, 1.0, 0.0),     # G = 1 (dense 1x1 linear)
     (7, 10, 20, 3, 1, 2, 8, 1, 1, 1.0, -30.0),  # bias -30: linear mass ~1e-18, windowed softmax
     (7, 10, 20, 3, 1, 2, 8, 1, 1, 1.0, 4.0),    # bias +4: linear term dominates
 ]
