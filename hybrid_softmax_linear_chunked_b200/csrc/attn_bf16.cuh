@@ -63,7 +63,8 @@ enum Bar {
   kMmaDone = 20,
   kWbFull = 21,  // block-diagonal W_q (hi, lo) loaded into the V stages
   kUFull = 22,   // 2 (per query tile): U_t = Q_t Wbd^T complete
-  kNumBars = 24
+  kPhiqFull = 24,  // precomputed phi_q tiles loaded over the Q tiles
+  kNumBars = 25
 };
 
 struct Params {
@@ -101,12 +102,17 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_addr, int kk) {
   return sdesc_sw128(tile_addr + kk * 16 * 128, kBM * 128, 1024);
 }
 
+// kPhiGlobal: phi_q of the query rows comes precomputed (bf16, one row per query) through tmPhi
+// and is loaded over the Q tiles once their last S MMA is done; otherwise the kernel computes it
+// in its epilogue from U = Q Wbd^T (tmW).
+template <bool kPhiGlobal>
 __global__ void __launch_bounds__(kThreads, 1)
     hybrid_attn_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                             const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV,
                             const __grid_constant__ CUtensorMap tmSt,
-                            const __grid_constant__ CUtensorMap tmW, const Params p) {
+                            const __grid_constant__ CUtensorMap tmW,
+                            const __grid_constant__ CUtensorMap tmPhi, const Params p) {
   static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
 
   // ---- chunk geometry (uniform over the CTA) ----
@@ -134,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* sB = reinterpret_cast<float*>(sm + kOffB);
   float* sZ = reinterpret_cast<float*>(sm + kOffZ);
-  int* sPw = reinterpret_cast<int*>(sm + kOffPw);
+  uint8_t* sPw = sm + kOffPw;
 
   if (warp == 8) {
     tmem_alloc(&tmem_base_sh, 512);
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid < 256 && has_linear) {
     for (int i = tid; i < kFD; i += 256) {
-      sPw[i] = part_power(i, kFD, p.P);
+      sPw[i] = static_cast<uint8_t>(part_power(i, kFD, p.P));
       sB[i] = p.bq ? p.bq[(size_t)h * kFD + i] : 0.f;
       sZ[i] = p.Z[((size_t)bh * p.n_states + c) * kFD + i];
     }
@@ -224,7 +230,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     bool wb_issued = false;
-    if (ok && has_linear) {
+    if (ok && has_linear && kPhiGlobal) {
+      // phi_q tiles go over the Q tiles once both tiles' last S MMAs are done.
+      const int last = n_kv - 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty + (last & 1)], (last >> 1) & 1, abort_flag));
+      if (ok) {
+        if (leader) {
+          mbar_arrive_expect_tx(&bars[kPhiqFull], has_t1 ? 2 * kTileBytes : kTileBytes);
+          for (int t = 0; t < (has_t1 ? 2 : 1); ++t) {
+            uint8_t* dst = sm + (t ? kOffQ1 : kOffQ0);
+            const int row = q_row0 + tile_row0 + t * kBM;
+            tma_load_3d(dst, &tmPhi, &bars[kPhiqFull], 0, row, bh);
+            tma_load_3d(dst + kBM * 128, &tmPhi, &bars[kPhiqFull], 64, row, bh);
+          }
+        }
+        __syncwarp();
+        wb_issued = true;
+      }
+    } else if (ok && has_linear) {
       // Block-diagonal W_q (hi, lo) goes into the two V stages once their last P.V is done.
       for (int s = 0; s < 2 && ok; ++s) {
         const int last = (n_kv - 1) - (((n_kv - 1) & 1) != s ? 1 : 0);  // last use of stage s
@@ -246,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok) {
       // Abort: let every copy already issued land before the CTA can exit.
-      if (wb_issued) mbar_wait_drain(&bars[kWbFull], 0);
+      if (wb_issued) mbar_wait_drain(&bars[kPhiGlobal ? kPhiqFull : kWbFull], 0);
       mbar_wait_drain(&bars[kQFull], 0);
       for (int j = max(0, issued_k - 2); j < issued_k; ++j)
         mbar_wait_drain(&bars[kKFull + (j & 1)], (j >> 1) & 1);
@@ -324,8 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && has_linear) {
       // U_t = Q_t Wbd_hi^T + Q_t Wbd_lo^T into the S_t columns (free once P_t.V is issued).
-      ok = wait(kWbFull, 0);
-      if (ok) {
+      if (!kPhiGlobal) ok = wait(kWbFull, 0);
+      if (ok && !kPhiGlobal) {
         tc_fence_after();
         if (leader) {
           for (int t = 0; t < nt; ++t) {
@@ -446,7 +469,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars[kPFull + t]);
       }
       // ---- epilogue ----
-      if (ok && has_linear) {
+      if (ok && has_linear && kPhiGlobal) {
+        // The precomputed phi_q row sits in this row of the Q tile: scale it by 2^-m in place
+        // (bf16) and form phi_q . Z_c with the same rounded values the MMA will use.
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kPhiqFull], 0, abort_flag));
+        if (ok) {
+          uint8_t* qrow = sm + (t ? kOffQ1 : kOffQ0);
+          const float esc = ex2(-m);
+          float lin[2] = {0.f, 0.f};
+#pragma unroll 4
+          for (int c8 = 0; c8 < kFD / 8; ++c8) {
+            uint4* a4 = reinterpret_cast<uint4*>(qrow + sw128_offset(r, c8 * 8, kBM));
+            uint4 v4 = *a4;
+            uint32_t* w = reinterpret_cast<uint32_t*>(&v4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 b2 = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
+              const float2 f2 = __bfloat1622float2(b2);
+              const float x0 = __bfloat162float(__float2bfloat16_rn(f2.x * esc));
+              const float x1 = __bfloat162float(__float2bfloat16_rn(f2.y * esc));
+              lin[0] = fmaf(x0, sZ[c8 * 8 + 2 * e], lin[0]);
+              lin[1] = fmaf(x1, sZ[c8 * 8 + 2 * e + 1], lin[1]);
+              w[e] = pack_bf16x2(x0, x1);
+            }
+            *a4 = v4;
+          }
+          fence_async_smem();
+          tc_fence_before();
+          mbar_arrive(&bars[kPhiFull + t]);
+          l += lin[0] + lin[1];
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars[kRoDone + t], 0, abort_flag));
+        }
+      } else if (ok && has_linear) {
         // U_FULL also means every earlier MMA of this CTA (the last P.V included) is complete.
         ok = __all_sync(0xffffffffu, mbar_wait(&bars[kUFull + t], 0, abort_flag));
         if (ok) {
@@ -462,18 +516,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t uu[16];
             tmem_ld16(tS + f0, uu);
             uint32_t packed[8];
+            phi16(uu, f0, sB, sPw, esc, packed);
 #pragma unroll
             for (int f2 = 0; f2 < 8; ++f2) {
-              float ph2[2];
-#pragma unroll
-              for (int q2 = 0; q2 < 2; ++q2) {
-                const int f = f0 + 2 * f2 + q2;
-                const float u = __uint_as_float(uu[2 * f2 + q2]) + sB[f];
-                const float ph = small_pow(softplus_fast(u), sPw[f]) * esc;
-                ph2[q2] = __bfloat162float(__float2bfloat16_rn(ph));
-                lin[q2] = fmaf(ph2[q2], sZ[f], lin[q2]);
-              }
-              packed[f2] = pack_bf16x2(ph2[0], ph2[1]);
+              const float2 pf = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&packed[f2]));
+              lin[0] = fmaf(pf.x, sZ[f0 + 2 * f2], lin[0]);
+              lin[1] = fmaf(pf.y, sZ[f0 + 2 * f2 + 1], lin[1]);
             }
             *reinterpret_cast<uint4*>(qrow + sw128_offset(r, f0, kBM)) =
                 make_uint4(packed[0], packed[1], packed[2], packed[3]);

@@ -7,7 +7,11 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "sm100.cuh"
+
 namespace rehyat {
+
+using sm100::pack_bf16x2;
 
 // Power applied to feature f when F features are split into P parts.
 __host__ __device__ __forceinline__ int part_power(int f, int F, int P) {
@@ -23,14 +27,13 @@ __device__ __forceinline__ float int_pow(float x, int p) {
   return r;
 }
 
-// x^p without branches for 1 <= p <= 4 (the usual part counts); larger p takes the loop.
-__device__ __forceinline__ float small_pow(float x, int p) {
-  float r = x;
+// x^p by selects, for 1 <= p <= 4.
+__device__ __forceinline__ float pow_upto4(float x, int p) {
   const float x2 = x * x;
+  float r = x;
   r = (p == 2) ? x2 : r;
   r = (p == 3) ? x2 * x : r;
   r = (p == 4) ? x2 * x2 : r;
-  if (p > 4) r = int_pow(x, p);
   return r;
 }
 
@@ -47,6 +50,38 @@ __device__ __forceinline__ float softplus_fast(float u) {
   const float y = __expf(-fabsf(u));
   const float l = (y < 0.0078125f) ? y * (1.f - y * (0.5f - y * (1.f / 3.f))) : __logf(1.f + y);
   return fmaxf(u, 0.f) + l;
+}
+
+// phi of 16 consecutive features f0 .. f0+15 from their grouped-linear outputs u (fp32 bits):
+// softplus(u + bias)^p, with p the feature's part power (pw[], non-decreasing in f), times
+// `scale`, packed as 8 bf16 pairs.  Parts are contiguous, so a 16-feature chunk nearly always
+// has a single power: that case (a uniform branch) costs at most two multiplies per feature.
+__device__ __forceinline__ void phi16(const uint32_t* u, int f0, const float* bias,
+                                      const uint8_t* pw, float scale, uint32_t* packed) {
+  float ph[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) ph[i] = softplus_fast(__uint_as_float(u[i]) + bias[f0 + i]);
+  const int p_first = pw[f0], p_last = pw[f0 + 15];
+  if (p_first == p_last) {
+    if (p_first == 2) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ph[i] *= ph[i];
+    } else if (p_first == 3) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ph[i] = ph[i] * ph[i] * ph[i];
+    } else if (p_first != 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ph[i] = int_pow(ph[i], p_first);
+    }
+  } else if (p_last <= 4) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) ph[i] = pow_upto4(ph[i], pw[f0 + i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) ph[i] = int_pow(ph[i], pw[f0 + i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(ph[2 * i] * scale, ph[2 * i + 1] * scale);
 }
 
 template <typename T>

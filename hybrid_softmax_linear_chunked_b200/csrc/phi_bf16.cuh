@@ -1,0 +1,194 @@
+// Feature map phi of the "ReHyAt overview" page §2.2.2 for many bf16 rows, on the tensor cores:
+// u = x Wbd^T (block-diagonal grouped 1x1 linear, bf16 hi + lo weight parts, fp32 in TMEM) by
+// tcgen05, then bias, softplus and the part powers on the CUDA cores, written as bf16 rows.
+// Used for phi_q of the query rows that read a linear state, so that the attention kernel's
+// epilogue only has to load a finished phi_q tile.
+#pragma once
+
+#include "featmap.cuh"
+#include "sm100.cuh"
+
+namespace rehyat {
+namespace phi {
+
+using namespace sm100;
+
+constexpr int kRows = 128;  // rows per tile (MMA M)
+constexpr int kHD = 128;
+constexpr int kFD = 128;
+constexpr int kThreads = 320;  // warps 0-7 feature map, 8 producer, 9 MMA
+constexpr int kPhiThreads = 256;
+constexpr int kTileBytes = kRows * kHD * 2;
+
+constexpr uint32_t kOffX = 0;                          // 2 stages
+constexpr uint32_t kOffW = kOffX + 2 * kTileBytes;      // block-diagonal W, hi and lo
+constexpr uint32_t kOffB = kOffW + 2 * kTileBytes;      // bias, F fp32
+constexpr uint32_t kOffPw = kOffB + kFD * 4;            // part power of each feature, uint8
+constexpr uint32_t kSmemBytes = kOffPw + kFD + 1024;    // + alignment slack
+
+enum Bar { kXFull = 0, kXEmpty = 2, kUFull = 4, kUEmpty = 6, kWbFull = 8, kDone = 9, kNumBars = 10 };
+
+struct Params {
+  int row0;           // first row (of each (b, h) sequence) to map
+  int n_rows;         // rows to map, starting at row0
+  int rows_per_bh;    // rows of each (b, h) in x and phi
+  int tiles_per_cta;  // 128-row tiles per CTA (blockIdx.x picks a run of them)
+  int H, P;
+  const float* bias;  // [H, F] or null
+  __nv_bfloat16* phi; // [BH, rows_per_bh, F]
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// grid (ceil(n_tiles / tiles_per_cta), BH), block 320.  Feature-map thread tid owns row
+// (tid & 127) = TMEM lane and features [64 (tid >> 7), +64).
+__global__ void __launch_bounds__(kThreads, 1)
+    featmap_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                      const __grid_constant__ CUtensorMap tmW, const Params p) {
+  static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
+  const int bh = blockIdx.y, h = bh % p.H;
+  const int n_tiles_all = (p.n_rows + kRows - 1) / kRows;
+  const int t_begin = blockIdx.x * p.tiles_per_cta;
+  const int n_tiles = min(p.tiles_per_cta, n_tiles_all - t_begin);
+  if (n_tiles <= 0) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  __shared__ __align__(8) uint64_t bars[kNumBars];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  volatile int* abort_flag = &abort_sh;
+  float* sB = reinterpret_cast<float*>(sm + kOffB);
+  uint8_t* sPw = sm + kOffPw;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (warp == 8) {
+    tmem_alloc(&tmem_base_sh, 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i)
+      mbar_init(&bars[i], (i == kUEmpty || i == kUEmpty + 1) ? kPhiThreads : 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  for (int i = tid; i < kFD; i += kThreads) {
+    sB[i] = p.bias ? p.bias[(size_t)h * kFD + i] : 0.f;
+    sPw[i] = static_cast<uint8_t>(part_power(i, kFD, p.P));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const bool leader = lane == 0;
+
+  if (warp == 8) {
+    // ---- producer ----
+    if (leader) {
+      tma_prefetch_desc(&tmX);
+      mbar_arrive_expect_tx(&bars[kWbFull], 2 * kTileBytes);
+      for (int part = 0; part < 2; ++part) {
+        uint8_t* dst = sm + kOffW + part * kTileBytes;
+        tma_load_3d(dst, &tmW, &bars[kWbFull], 0, 0, h * 2 + part);
+        tma_load_3d(dst + kRows * 128, &tmW, &bars[kWbFull], 64, 0, h * 2 + part);
+      }
+    }
+    __syncwarp();
+    bool ok = true;
+    int issued = 0;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int s = i & 1;
+      const int row = p.row0 + (t_begin + i) * kRows;
+      if (i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kXEmpty + s], ((i >> 1) - 1) & 1, abort_flag));
+      if (!ok) break;
+      if (leader) {
+        uint8_t* dx = sm + kOffX + s * kTileBytes;
+        mbar_arrive_expect_tx(&bars[kXFull + s], kTileBytes);
+        tma_load_3d(dx, &tmX, &bars[kXFull + s], 0, row, bh);
+        tma_load_3d(dx + kRows * 128, &tmX, &bars[kXFull + s], 64, row, bh);
+      }
+      __syncwarp();
+      ++issued;
+    }
+    if (!ok) {
+      mbar_wait_drain(&bars[kWbFull], 0);
+      for (int i = max(0, issued - 2); i < issued; ++i)
+        mbar_wait_drain(&bars[kXFull + (i & 1)], (i >> 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---- MMA issuer: U[s] = X_i Wbd_hi^T + X_i Wbd_lo^T ----
+    const uint32_t id_u = idesc_bf16(kRows, kFD, false, false);
+    const uint64_t dX0 = sdesc_sw128(smem_u32(sm + kOffX), 16, 1024);
+    const uint64_t dW0 = sdesc_sw128(smem_u32(sm + kOffW), 16, 1024);
+    auto koff = [](int kk) { return (uint64_t)((kk >> 2) * (kRows * 128 / 16) + (kk & 3) * 2); };
+    auto wait = [&](int b, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, abort_flag));
+    };
+    bool ok = wait(kWbFull, 0);
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const int s = i & 1;
+      ok = wait(kXFull + s, (i >> 1) & 1);
+      if (ok && i >= 2) ok = wait(kUEmpty + s, ((i >> 1) - 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (leader) {
+        const uint64_t dx = dX0 + (uint64_t)(s * kTileBytes / 16);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk)
+            mma_ss(tmem + s * 128, dx + koff(kk), dW0 + (uint64_t)(part * kTileBytes / 16) + koff(kk),
+                   id_u, (part > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[kUFull + s]);
+        mma_commit(&bars[kXEmpty + s]);
+      }
+      __syncwarp();
+    }
+    if (leader) mma_commit(&bars[kDone]);
+    __syncwarp();
+    mbar_wait_drain(&bars[kDone], 0);
+    __syncwarp();
+  } else {
+    // ---- feature-map warps ----
+    const int r = tid & 127, hf = tid >> 7;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int col0 = hf * 64;
+    bool ok = true;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int s = i & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kUFull + s], (i >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int row_in = (t_begin + i) * kRows + r;  // row index inside [row0, row0 + n_rows)
+      const bool valid = row_in < p.n_rows;
+      __nv_bfloat16* dst = p.phi + ((size_t)bh * p.rows_per_bh + p.row0 + row_in) * kFD + col0;
+#pragma unroll 1
+      for (int c16 = 0; c16 < 4; ++c16) {
+        const int f0 = col0 + c16 * 16;
+        uint32_t uu[16];
+        tmem_ld16(tmem + lane_base + s * 128 + f0, uu);
+        uint32_t packed[8];
+        phi16(uu, f0, sB, sPw, 1.f, packed);
+        if (valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c16 * 16);
+          d4[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          d4[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[kUEmpty + s]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace phi
+}  // namespace rehyat

@@ -16,6 +16,7 @@
 #include "attn_bf16.cuh"
 #include "featmap.cuh"
 #include "fp32_path.cuh"
+#include "phi_bf16.cuh"
 #include "sm100.cuh"
 #include "state_bf16.cuh"
 
@@ -139,7 +140,7 @@ int fold_splits(int BH, int n_fold, long long rows_per_fold) {
 
 struct ForwardPlan {
   int C, n_fold, splits;
-  size_t dS, dZ, St, Zc, Wqbd, Wkbd, phiq, phik, Sc, total;
+  size_t dS, dZ, St, Zc, Wqbd, Wkbd, phiq_bf16, phiq, phik, Sc, total;
 };
 
 ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, int Tc, int To) {
@@ -157,6 +158,7 @@ ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, in
     p.Zc = cv.take(BH * p.C * d.F * 4);
     p.Wqbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
     p.Wkbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
+    p.phiq_bf16 = cv.take(BH * (size_t)T * L * d.F * 2);
   } else {
     p.splits = 1;
     const size_t N = (size_t)T * L;
@@ -174,7 +176,7 @@ ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, in
 
 struct ChunkPlan {
   int o, nq, nkv, fold_rows, splits;
-  size_t St, dS, dZ, Wqbd, Wkbd, phiq, phik, total;
+  size_t St, dS, dZ, Wqbd, Wkbd, phiq_bf16, phiq, phik, total;
 };
 
 ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_before,
@@ -199,6 +201,7 @@ ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_be
     p.dZ = cv.take(BH * p.splits * d.F * 4);
     p.Wqbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
     p.Wkbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
+    p.phiq_bf16 = cv.take(BH * (size_t)p.nq * d.F * 2);
   } else {
     p.splits = 1;
     const size_t max_kv = (size_t)(To + chunk_frames) * L;
@@ -235,15 +238,41 @@ int launch_featmap(const rehyat_dims& d, rehyat_dtype dt, int n, const void* x, 
   return cuda_check(cudaGetLastError(), "featmap launch");
 }
 
+template <bool kPhiGlobal>
 int launch_attn_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const CUtensorMap& ms, const CUtensorMap& mw, const rehyat::attn::Params& ap,
-                     dim3 grid, cudaStream_t st) {
-  auto k = rehyat::attn::hybrid_attn_bf16_kernel;
+                     const CUtensorMap& ms, const CUtensorMap& mw, const CUtensorMap& mphi,
+                     const rehyat::attn::Params& ap, dim3 grid, cudaStream_t st) {
+  auto k = rehyat::attn::hybrid_attn_bf16_kernel<kPhiGlobal>;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)rehyat::attn::kSmemBytes),
                     "attn attr"));
-  k<<<grid, rehyat::attn::kThreads, rehyat::attn::kSmemBytes, st>>>(mq, mk, mv, ms, mw, ap);
+  k<<<grid, rehyat::attn::kThreads, rehyat::attn::kSmemBytes, st>>>(mq, mk, mv, ms, mw, mphi, ap);
   return cuda_check(cudaGetLastError(), "attention launch");
+}
+
+// phi of rows [row0, row0 + n_rows) of every (b, h) sequence of x (rows_per_bh rows each) into
+// phi ([BH][rows_per_bh][F] bf16) on the tensor cores; `mw` maps the block-diagonal weights.
+int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int row0, int n_rows,
+                      const CUtensorMap& mw, const float* bias, __nv_bfloat16* phi,
+                      cudaStream_t st) {
+  if (n_rows <= 0) return REHYAT_OK;
+  const int BH = d.B * d.H;
+  CUtensorMap mx;
+  RH_TRY(make_map(&mx, x, d.D, rows_per_bh, BH));
+  const int n_tiles = (n_rows + 127) / 128;
+  int per_cta = (int)(((long long)n_tiles * BH + 2 * 148 - 1) / (2 * 148));
+  if (per_cta < 1) per_cta = 1;
+  if (per_cta > n_tiles) per_cta = n_tiles;
+  rehyat::phi::Params pp{};
+  pp.row0 = row0; pp.n_rows = n_rows; pp.rows_per_bh = rows_per_bh; pp.tiles_per_cta = per_cta;
+  pp.H = d.H; pp.P = d.P; pp.bias = bias; pp.phi = phi;
+  auto k = rehyat::phi::featmap_tc_kernel;
+  RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)rehyat::phi::kSmemBytes),
+                    "featmap_tc attr"));
+  k<<<dim3((n_tiles + per_cta - 1) / per_cta, BH), rehyat::phi::kThreads, rehyat::phi::kSmemBytes,
+      st>>>(mx, mw, pp);
+  return cuda_check(cudaGetLastError(), "featmap_tc launch");
 }
 
 int launch_fold_bf16(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mw,
@@ -435,6 +464,14 @@ int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
     RH_TRY(make_map(&mv, v, d.D, N, BH));
     RH_TRY(make_map(&ms, ws + pl.St, d.F, d.D, (long long)BH * pl.C));
     RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mw, st));
+    // phi_q of every query row whose chunk has a linear region: chunks c >= To / Tc + 1
+    __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
+    const long long c_lin = To / Tc + 1;
+    const long long row_lin = c_lin * Tc * L;
+    if (row_lin < N)
+      RH_TRY(launch_featmap_tc(d, q, (int)N, (int)row_lin, (int)(N - row_lin), mw, bq, phiq, st));
+    CUtensorMap mphi;
+    RH_TRY(make_map(&mphi, phiq, d.F, N, BH));
     rehyat::attn::Params ap{};
     ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
     ap.H = d.H; ap.P = d.P; ap.n_states = pl.C; ap.nq_rows = (int)N;
@@ -442,7 +479,7 @@ int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
     ap.bq = bq; ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
     ap.out = static_cast<__nv_bfloat16*>(out);
     dim3 grid((rows_per_chunk + 255) / 256, pl.C, BH);
-    return launch_attn_bf16(mq, mk, mv, ms, mw, ap, grid, st);
+    return launch_attn_bf16<true>(mq, mk, mv, ms, mw, mphi, ap, grid, st);
   }
   float* phiq = reinterpret_cast<float*>(ws + pl.phiq);
   RH_TRY(launch_featmap(d, REHYAT_F32, (int)N, q, Wq, bq, phiq, st));
@@ -521,13 +558,19 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int L, int frames_befor
     RH_TRY(make_map(&mv, v_win, d.D, pl.nkv, BH));
     RH_TRY(make_map(&ms, St, d.F, d.D, BH));
     RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mwq, st));
+    __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
+    if (frames_before - pl.o > 0)  // the chunk reads a linear state
+      RH_TRY(launch_featmap_tc(d, q, pl.nq, 0, pl.nq, mwq, bq, phiq, st));
+    CUtensorMap mphi;
+    RH_TRY(make_map(&mphi, phiq, d.F, pl.nq, BH));
     rehyat::attn::Params ap{};
     ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
     ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
     ap.H = d.H; ap.P = d.P; ap.n_states = 1; ap.nq_rows = pl.nq;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
     ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
-    RH_TRY(launch_attn_bf16(mq, mk, mv, ms, mwq, ap, dim3((pl.nq + 255) / 256, 1, BH), st));
+    RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
+                                  dim3((pl.nq + 255) / 256, 1, BH), st));
     if (pl.fold_rows > 0) {
       RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
       rehyat::state::FoldParams fp{};
@@ -626,7 +669,8 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   ap.H = d.H; ap.P = d.P; ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
-  RH_TRY(launch_attn_bf16(mq, mk, mv, ms, mwq, ap, dim3((pl.nq + 255) / 256, 1, nbh), st));
+  RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3((pl.nq + 255) / 256, 1, nbh),
+                                 st));
   if (pl.fold_rows > 0) {
     RH_TRY(prepare_blockdiag(d, Wk, Wkbd, &mwk, st));
     rehyat::state::FoldParams fp{};

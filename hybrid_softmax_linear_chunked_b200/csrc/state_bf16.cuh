@@ -269,17 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t uu[16];
         tmem_ld16(tmem + lane_base + s * 128 + f0, uu);
         uint32_t packed[8];
-#pragma unroll
-        for (int f2 = 0; f2 < 8; ++f2) {
-          float ph[2];
-#pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
-            const int f = f0 + 2 * f2 + q2;
-            const float u = __uint_as_float(uu[2 * f2 + q2]) + sB[f];
-            ph[q2] = small_pow(softplus_fast(u), sPw[f]);
-          }
-          packed[f2] = valid ? pack_bf16x2(ph[0], ph[1]) : 0u;
-        }
+        phi16(uu, f0, sB, sPw, valid ? 1.f : 0.f, packed);
         *reinterpret_cast<uint4*>(prow + sw128_offset(r, f0, kTok)) =
             make_uint4(packed[0], packed[1], packed[2], packed[3]);
         *reinterpret_cast<uint4*>(prow + sw128_offset(r, f0 + 8, kTok)) =
