@@ -280,9 +280,11 @@ def main():
 
     def step(ev_mid=None, ev_end=None):
         rb.forward_states(k, v, Wk, bk, workspace=ws, **kw)
+        rb.forward_phiq(q, Wq, bq, workspace=ws, **kw)
         if ev_mid is not None:
             ev_mid.record(stream)
-        rb.forward_attend(q, k, v, Wq, bq, workspace=ws, out=out, **kw)
+        rb.forward_attend(q, k, v, dims=d, frame_tokens=w.frame_tokens, Tc=w.Tc, To=w.To,
+                          workspace=ws, out=out)
         if ev_end is not None:
             ev_end.record(stream)
 
@@ -311,7 +313,7 @@ def main():
     rb.sync_status(dev)
     elapsed_ms = start.elapsed_time(stop)
     attn_ms = statistics.mean(mids[i].elapsed_time(ends[i]) for i in range(K))
-    # states phase of step i runs between end of step i-1 (or start) and mid of step i
+    # states + phi_q phases of step i run between the end of step i-1 (or start) and mid of step i
     state_ms = statistics.mean((ends[i - 1].elapsed_time(mids[i]) if i else
                                 start.elapsed_time(mids[0])) for i in range(K))
     if dist is not None:
@@ -371,7 +373,7 @@ def main():
             "config": workload_config(w, world),
             "tflops": w.flops() * world / (ms_per_step * 1e-3) / 1e12,
             "frac_of_bf16_peak_step": w.flops() / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
-            "kernel_ms": {"attention": attn_ms, "states": state_ms},
+            "kernel_ms": {"attention": attn_ms, "states_and_phiq": state_ms},
             "roofline": {"kernel": "hybrid_attn_bf16_kernel", "bound": "tensor",
                          "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"],
@@ -381,7 +383,7 @@ def main():
                          "traffic": read_traffic()},
             "e2e": {"value": tokens_per_step / (e2e_ms / E * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 5 * K,  # per step: 2 weight preps, fold, scan, attention
+            "gpu_launches": 6 * K,  # per step: 2 weight preps, fold, scan, phi_q, attention
             "clocks": sampler.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

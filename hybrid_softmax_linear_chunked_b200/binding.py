@@ -21,7 +21,7 @@ STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_SHAPE", -3: "ERR_DTYPE", -4: "ERR_WOR
 
 EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_forward_workspace_size", "rehyat_forward", "rehyat_forward_states",
-            "rehyat_forward_attend", "rehyat_chunk_workspace_size",
+            "rehyat_forward_phiq", "rehyat_forward_attend", "rehyat_chunk_workspace_size",
             "rehyat_chunk_forward", "rehyat_chunk_forward_static", "rehyat_chunk_states",
             "rehyat_sync_status"]
 
@@ -65,8 +65,10 @@ def load() -> ctypes.CDLL:
                                  P, c_size_t, P]
     L.rehyat_forward_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P,
                                         c_size_t, P]
+    L.rehyat_forward_phiq.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P,
+                                      c_size_t, P]
     L.rehyat_forward_attend.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P,
-                                        P, P, c_size_t, P]
+                                        c_size_t, P]
     L.rehyat_chunk_workspace_size.argtypes = [Dims, c_int, c_int, c_int, c_int,
                                               ctypes.POINTER(c_size_t)]
     L.rehyat_chunk_forward.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
@@ -188,7 +190,7 @@ def forward(q, k, v, Wq, bq, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: 
 
 
 def forward_states(k, v, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
-                   workspace: torch.Tensor, Wq: torch.Tensor | None = None) -> torch.Tensor:
+                   workspace: torch.Tensor) -> torch.Tensor:
     """First phase of `forward`: fills `workspace` with the state every chunk reads."""
     lib = load()
     dev = _dev(k, v, Wk, bk, workspace)
@@ -200,15 +202,26 @@ def forward_states(k, v, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
     return workspace
 
 
-def forward_attend(q, k, v, Wq, bq, *, P: int, frame_tokens: int, Tc: int, To: int,
-                   workspace: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
-    """Second phase of `forward`: the hybrid output from q, k, v and the workspace states."""
+def forward_phiq(q, Wq, bq, *, P: int, frame_tokens: int, Tc: int, To: int,
+                 workspace: torch.Tensor) -> torch.Tensor:
+    """Second phase of `forward`: phi_q of the query rows that read a state, into `workspace`."""
     lib = load()
-    dev = _dev(q, k, v, Wq, bq, workspace, out)
+    dev = _dev(q, Wq, bq, workspace)
     d = dims_of(q, Wq, P)
     T = q.shape[2] // frame_tokens
-    _check(lib.rehyat_forward_attend(d, _dtype_code(q), T, frame_tokens, Tc, To, _ptr(q), _ptr(k),
-                                     _ptr(v), _ptr(Wq), _ptr(bq), _ptr(out), _ptr(workspace),
+    _check(lib.rehyat_forward_phiq(d, _dtype_code(q), T, frame_tokens, Tc, To, _ptr(q), _ptr(Wq),
+                                   _ptr(bq), _ptr(workspace), workspace.numel(), _stream(dev)))
+    return workspace
+
+
+def forward_attend(q, k, v, *, dims: Dims, frame_tokens: int, Tc: int, To: int,
+                   workspace: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
+    """Third phase of `forward`: the hybrid output from q, k, v and the workspace."""
+    lib = load()
+    dev = _dev(q, k, v, workspace, out)
+    T = q.shape[2] // frame_tokens
+    _check(lib.rehyat_forward_attend(dims, _dtype_code(q), T, frame_tokens, Tc, To, _ptr(q),
+                                     _ptr(k), _ptr(v), _ptr(out), _ptr(workspace),
                                      workspace.numel(), _stream(dev)))
     return out
 

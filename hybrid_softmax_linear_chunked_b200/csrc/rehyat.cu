@@ -442,14 +442,37 @@ int rehyat_forward_states(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
                             reinterpret_cast<float*>(ws + pl.Zc), st);
 }
 
-int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
-                          const void* q, const void* k, const void* v, const float* Wq,
-                          const float* bq, void* out, const void* workspace, size_t ws_bytes,
-                          void* stream) {
+int rehyat_forward_phiq(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                        const void* q, const float* Wq, const float* bq, void* workspace,
+                        size_t ws_bytes, void* stream) {
   g_msg[0] = 0;
   ForwardPlan pl;
   RH_TRY(forward_common_checks(d, dt, T, L, Tc, To, workspace, ws_bytes, &pl));
-  if (!q || !k || !v || !Wq || !out) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!q || !Wq) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(q)) return fail(REHYAT_ERR_ALIGN, "q not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const long long N = (long long)T * L;
+  if (dt == REHYAT_BF16) {
+    CUtensorMap mw;
+    RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mw, st));
+    // phi_q of every query row whose chunk has a linear region: chunks c >= To / Tc + 1
+    const long long row_lin = (long long)(To / Tc + 1) * Tc * L;
+    if (row_lin < N)
+      RH_TRY(launch_featmap_tc(d, q, (int)N, (int)row_lin, (int)(N - row_lin), mw, bq,
+                               reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16), st));
+    return REHYAT_OK;
+  }
+  return launch_featmap(d, REHYAT_F32, (int)N, q, Wq, bq, ws + pl.phiq, st);
+}
+
+int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                          const void* q, const void* k, const void* v, void* out,
+                          const void* workspace, size_t ws_bytes, void* stream) {
+  g_msg[0] = 0;
+  ForwardPlan pl;
+  RH_TRY(forward_common_checks(d, dt, T, L, Tc, To, workspace, ws_bytes, &pl));
+  if (!q || !k || !v || !out) return fail(REHYAT_ERR_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(REHYAT_ERR_ALIGN, "q/k/v/out not 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -458,37 +481,28 @@ int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
   const long long N = (long long)T * L;
   const int rows_per_chunk = (Tc < T ? Tc : T) * L;
   if (dt == REHYAT_BF16) {
-    CUtensorMap mq, mk, mv, ms, mw;
+    CUtensorMap mq, mk, mv, ms, mphi;
     RH_TRY(make_map(&mq, q, d.D, N, BH));
     RH_TRY(make_map(&mk, k, d.D, N, BH));
     RH_TRY(make_map(&mv, v, d.D, N, BH));
     RH_TRY(make_map(&ms, ws + pl.St, d.F, d.D, (long long)BH * pl.C));
-    RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mw, st));
-    // phi_q of every query row whose chunk has a linear region: chunks c >= To / Tc + 1
-    __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
-    const long long c_lin = To / Tc + 1;
-    const long long row_lin = c_lin * Tc * L;
-    if (row_lin < N)
-      RH_TRY(launch_featmap_tc(d, q, (int)N, (int)row_lin, (int)(N - row_lin), mw, bq, phiq, st));
-    CUtensorMap mphi;
-    RH_TRY(make_map(&mphi, phiq, d.F, N, BH));
+    RH_TRY(make_map(&mphi, ws + pl.phiq_bf16, d.F, N, BH));
     rehyat::attn::Params ap{};
     ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
     ap.H = d.H; ap.P = d.P; ap.n_states = pl.C; ap.nq_rows = (int)N;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
-    ap.bq = bq; ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
+    ap.bq = nullptr;  // phi_q comes finished from the workspace
+    ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
     ap.out = static_cast<__nv_bfloat16*>(out);
     dim3 grid((rows_per_chunk + 255) / 256, pl.C, BH);
-    return launch_attn_bf16<true>(mq, mk, mv, ms, mw, mphi, ap, grid, st);
+    return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, grid, st);
   }
-  float* phiq = reinterpret_cast<float*>(ws + pl.phiq);
-  RH_TRY(launch_featmap(d, REHYAT_F32, (int)N, q, Wq, bq, phiq, st));
   rehyat::fp32::AttnParams ap{};
   ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
   ap.D = d.D; ap.F = d.F; ap.nq_rows = (int)N; ap.nkv_rows = (int)N; ap.n_states = pl.C;
   ap.scale = (float)(1.0 / std::sqrt((double)d.D));
   ap.q = static_cast<const float*>(q); ap.k = static_cast<const float*>(k);
-  ap.v = static_cast<const float*>(v); ap.phiq = phiq;
+  ap.v = static_cast<const float*>(v); ap.phiq = reinterpret_cast<const float*>(ws + pl.phiq);
   ap.S = reinterpret_cast<const float*>(ws + pl.Sc);
   ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
   ap.out = static_cast<float*>(out);
@@ -508,8 +522,8 @@ int rehyat_forward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(REHYAT_ERR_ALIGN, "q/k/v/out not 16-byte aligned");
   RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, workspace, ws_bytes, stream));
-  return rehyat_forward_attend(d, dt, T, L, Tc, To, q, k, v, Wq, bq, out, workspace, ws_bytes,
-                               stream);
+  RH_TRY(rehyat_forward_phiq(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream));
+  return rehyat_forward_attend(d, dt, T, L, Tc, To, q, k, v, out, workspace, ws_bytes, stream);
 }
 
 int rehyat_chunk_workspace_size(rehyat_dims d, rehyat_dtype dt, int frame_tokens,

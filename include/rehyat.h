@@ -96,20 +96,23 @@ int rehyat_forward(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int 
                    const float* Wk, const float* bk, void* out, void* workspace,
                    size_t ws_bytes, void* stream);
 
-/* rehyat_forward in two phases on the same workspace (rehyat_forward is exactly
- * rehyat_forward_states followed by rehyat_forward_attend):
+/* rehyat_forward in three phases on the same workspace (rehyat_forward is exactly
+ * rehyat_forward_states, rehyat_forward_phiq, rehyat_forward_attend in that order):
  *   _states: the §2.3 folds of every chunk and their prefix sums (the state each chunk reads),
  *            written into the workspace; reads k, v and phi_k's parameters;
- *   _attend: the hybrid output of every chunk from q, k, v and the workspace states.
- * The workspace must not change between the two calls.  Useful to reuse the states of one
- * (k, v) across several query sets, and to time the phases separately. */
+ *   _phiq:   phi_q of every query row whose chunk reads a linear state, into the workspace;
+ *   _attend: the hybrid output of every chunk from q, k, v and the workspace.
+ * The workspace must not change between the calls.  Useful to reuse the states of one (k, v)
+ * across several query sets, and to time the phases separately. */
 int rehyat_forward_states(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
                           const void* k, const void* v, const float* Wk, const float* bk,
                           void* workspace, size_t ws_bytes, void* stream);
+int rehyat_forward_phiq(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
+                        const void* q, const float* Wq, const float* bq, void* workspace,
+                        size_t ws_bytes, void* stream);
 int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
-                          const void* q, const void* k, const void* v, const float* Wq,
-                          const float* bq, void* out, const void* workspace, size_t ws_bytes,
-                          void* stream);
+                          const void* q, const void* k, const void* v, void* out,
+                          const void* workspace, size_t ws_bytes, void* stream);
 
 /* Workspace bytes rehyat_chunk_forward needs for one chunk of chunk_frames frames. */
 int rehyat_chunk_workspace_size(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
