@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 from hybrid_softmax_linear_chunked_b200 import binding as rb  # noqa: E402
 from hybrid_softmax_linear_chunked_b200 import configs as C  # noqa: E402
 from hybrid_softmax_linear_chunked_b200.inputs import make_inputs  # noqa: E402
+from hybrid_softmax_linear_chunked_b200.replicas import Replicas, job_throughput  # noqa: E402
 
 METRIC = "hybrid-attn query tokens/s (12 heads, D=128); % of dense BF16 tensor peak"
 UNIT = "tokens/s"
@@ -251,24 +252,17 @@ def workload_config(w: C.Workload, n_gpus: int):
 
 def main():
     args = parse_args()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        run_reference(args, rank)
+        run_reference(args, int(os.environ.get("RANK", "0")))
         return
 
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    rep = Replicas.from_env("nccl")
+    rank, world, local = rep.rank, rep.world, rep.local_rank
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     rb.load()
     w = WORKLOAD
-    inp = make_inputs(w, seed=w.seed + rank)
+    inp = make_inputs(w, seed=rep.seed(w.seed))
     q, k, v = (x.to(dev) for x in (inp.q, inp.k, inp.v))
     Wq, bq, Wk, bk = (x.to(dev) for x in (inp.Wq, inp.bq, inp.Wk, inp.bk))
     kw = dict(P=w.P, frame_tokens=w.frame_tokens, Tc=w.Tc, To=w.To)
@@ -288,10 +282,6 @@ def main():
         if ev_end is not None:
             ev_end.record(stream)
 
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
     for _ in range(max(3, args.warmup)):
         step()
     rb.sync_status(dev)
@@ -302,24 +292,21 @@ def main():
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(device_index_for_smi(dev))
     with sampler:
-        barrier()
+        rep.barrier()
         torch.cuda.synchronize(dev)
         start.record(stream)
         for i in range(K):
             step(mids[i], ends[i])
         stop.record(stream)
         torch.cuda.synchronize(dev)
-        barrier()
+        rep.barrier()
     rb.sync_status(dev)
     elapsed_ms = start.elapsed_time(stop)
     attn_ms = statistics.mean(mids[i].elapsed_time(ends[i]) for i in range(K))
     # states + phi_q phases of step i run between the end of step i-1 (or start) and mid of step i
     state_ms = statistics.mean((ends[i - 1].elapsed_time(mids[i]) if i else
                                 start.elapsed_time(mids[0])) for i in range(K))
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = rep.max(elapsed_ms, dev)
 
     # ---- end to end through the public API: pinned host inputs in, result out ----
     host = [x.pin_memory() for x in (inp.q, inp.k, inp.v, inp.Wq, inp.bq, inp.Wk, inp.bk)]
@@ -336,30 +323,26 @@ def main():
         e2e_step()
     E = args.e2e_steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
+    rep.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
     for _ in range(E):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    barrier()
+    rep.barrier()
     rb.sync_status(dev)
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = rep.max(e2e_ms, dev)
 
     if rank == 0:
         peaks = read_peaks()
-        tokens_per_step = w.B * w.N * world
         ms_per_step = elapsed_ms / K
         flops_attn = w.attn_tensor_flops()
         achieved = flops_attn / (attn_ms * 1e-3) / 1e12
         line = {
             "metric": METRIC,
-            "value": tokens_per_step / (ms_per_step * 1e-3),
+            "value": job_throughput(w.B * w.N, world, ms_per_step),
             "unit": UNIT,
             "n_gpus": world,
             "steps": K,
@@ -381,7 +364,7 @@ def main():
                          "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
                                                if peaks.get("bf16_tflops_sustained") else None),
                          "traffic": read_traffic()},
-            "e2e": {"value": tokens_per_step / (e2e_ms / E * 1e-3), "unit": UNIT,
+            "e2e": {"value": job_throughput(w.B * w.N, world, e2e_ms / E), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 6 * K,  # per step: 2 weight preps, fold, scan, phi_q, attention
             "clocks": sampler.summary(),
@@ -389,9 +372,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp, w)
         print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    rep.close()
 
 
 if __name__ == "__main__":

@@ -23,7 +23,7 @@ EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_forward_workspace_size", "rehyat_forward", "rehyat_forward_states",
             "rehyat_forward_phiq", "rehyat_forward_attend", "rehyat_chunk_workspace_size",
             "rehyat_chunk_forward", "rehyat_chunk_forward_static", "rehyat_chunk_states",
-            "rehyat_sync_status"]
+            "rehyat_selftest_wait_timeout", "rehyat_sync_status"]
 
 
 class RehyatError(RuntimeError):
@@ -77,6 +77,7 @@ def load() -> ctypes.CDLL:
                                               P, P, P, P, P, P, P]
     L.rehyat_chunk_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
                                       P, c_size_t, P]
+    L.rehyat_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
     L.rehyat_sync_status.argtypes = [P]
     for name in EXPORTED:
         if name not in ("rehyat_last_error",):
@@ -279,6 +280,13 @@ def chunk_forward_static(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, frame
                                            _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(S),
                                            _ptr(Z), _ptr(out), _stream(dev)))
     return out
+
+
+def selftest_wait_timeout(limit_ns: int = 20_000_000, device: torch.device | None = None) -> None:
+    """Enqueue the bounded-wait failure self test; the next sync_status() then raises
+    RehyatError with status REHYAT_ERR_TIMEOUT."""
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    _check(load().rehyat_selftest_wait_timeout(ctypes.c_longlong(int(limit_ns)), _stream(dev)))
 
 
 def sync_status(device: torch.device | None = None) -> None:

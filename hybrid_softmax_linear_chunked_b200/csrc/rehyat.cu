@@ -378,6 +378,23 @@ int static_scratch_for_current_device(void** out) {
   return REHYAT_OK;
 }
 
+// Exercises the error path of the bounded mbarrier wait: every warp waits on a barrier that
+// nothing arrives on.  The first wait to pass `limit_ns` raises the CTA's abort flag and sets
+// the device error word; the other warps see the flag and return too.
+__global__ void __launch_bounds__(64) wait_timeout_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_sh;
+  if (threadIdx.x == 0) {
+    rehyat::sm100::mbar_init(&bar, 1);
+    abort_sh = 0;
+    rehyat::sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abort_flag = &abort_sh;
+  rehyat::sm100::mbar_wait(&bar, 0, abort_flag, limit_ns);
+  __syncthreads();
+}
+
 }  // namespace
 
 // =============================================================================================
@@ -717,6 +734,15 @@ int rehyat_chunk_states(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, in
     return forward_states_bf16(d, T, L, Tc, To, k, v, Wk, bk, pl, ws, nullptr, nullptr, S_out,
                                Z_out, st);
   return forward_states_f32(d, T, L, Tc, To, k, v, Wk, bk, pl, ws, S_out, Z_out, st);
+}
+
+int rehyat_selftest_wait_timeout(long long limit_ns, void* stream) {
+  g_msg[0] = 0;
+  if (limit_ns < 1000 || limit_ns > 2000000000LL)
+    return fail(REHYAT_ERR_ARG, "limit_ns %lld outside [1e3, 2e9]", limit_ns);
+  wait_timeout_selftest_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_ns));
+  return cuda_check(cudaGetLastError(), "wait_timeout_selftest_kernel launch");
 }
 
 int rehyat_sync_status(void* stream) {

@@ -165,6 +165,14 @@ int rehyat_chunk_states(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens,
                         float* S_out, float* Z_out, void* workspace, size_t ws_bytes,
                         void* stream);
 
+/* Failure-path self test (no counterpart on the pages): enqueue on `stream` one small kernel whose
+ * warps wait on an mbarrier that nothing arrives on, with the same bounded wait the other
+ * kernels use but a limit of `limit_ns` nanoseconds (1e3 .. 2e9).  The wait gives up, the kernel
+ * sets the device error word and returns, so the next rehyat_sync_status() on that stream
+ * returns REHYAT_ERR_TIMEOUT (and clears the word); the context stays usable.  Returns
+ * REHYAT_ERR_ARG for a limit out of range, REHYAT_ERR_CUDA if the launch fails. */
+int rehyat_selftest_wait_timeout(long long limit_ns, void* stream);
+
 /* Synchronise `stream` and report device-side failures of earlier calls: REHYAT_ERR_TIMEOUT if
  * a kernel's bounded wait gave up (the error word is then cleared), REHYAT_ERR_CUDA if the
  * stream reports a CUDA error, else REHYAT_OK. */

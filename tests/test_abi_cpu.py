@@ -93,3 +93,9 @@ def test_chunk_forward_rejects_bad_arguments(lib):
     st = lib.rehyat_chunk_forward(d, rb.REHYAT_BF16, 64, 3, 3, 1, FAKE, FAKE, FAKE, FAKE, None,
                                   FAKE, None, FAKE, FAKE, FAKE, FAKE, 8, None)
     assert st == -4
+
+
+def test_selftest_rejects_limits_out_of_range(lib):
+    for bad in (0, 999, 2_000_000_001):
+        assert lib.rehyat_selftest_wait_timeout(bad, None) == -1
+        assert "limit_ns" in lib.rehyat_last_error().decode()
