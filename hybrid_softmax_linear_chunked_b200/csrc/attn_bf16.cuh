@@ -92,6 +92,32 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// ---- paired fp32 arithmetic (one instruction for two lanes of a 64-bit register pair) ----
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+
 // K-major SW128 descriptor of the kk-th 16-wide K step of a 128-row, 128-wide bf16 tile.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_addr, int kk) {
   return sdesc_sw128(tile_addr + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
@@ -419,9 +445,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(rr[i]);
 #pragma unroll
-          for (int i = 8; i < kBN; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(rr[i]));
-          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          for (int i = 8; i < kBN; i += 16)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              m8[e] = max3(m8[e], __uint_as_float(rr[i + e]), __uint_as_float(rr[i + 8 + e]));
+          mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         }
         const float m_tile = mx * sl2;
         const float m_new = (m_tile > m + 8.f) ? m_tile : m;
@@ -449,20 +477,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         m = m_new;
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        // Column pairs go through paired fp32 instructions (x = s * scale - m for two columns in
+        // one FMA, the row sum in two paired accumulators); 2^x on the MUFU; bf16 pack.
+        // 16 probabilities -> 8 packed columns per TMEM store.
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m, -m);
+        uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-        for (int hh = 0; hh < kBN / 16; ++hh) {  // 16 probabilities -> 8 packed columns per store
+        for (int hh = 0; hh < kBN / 16; ++hh) {
           uint32_t pr[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float a = ex2(fmaf(__uint_as_float(rr[hh * 16 + 2 * i]), sl2, -m));
-            const float b = ex2(fmaf(__uint_as_float(rr[hh * 16 + 2 * i + 1]), sl2, -m));
-            rs[i & 3] += a + b;
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(rr[hh * 16 + 2 * i]),
+                                               __uint_as_float(rr[hh * 16 + 2 * i + 1])),
+                                       sl2x2, negm2);
+            float xa, xb;
+            f2_unpack(x2, xa, xb);
+            const uint64_t p2 = f2_pack(ex2(xa), ex2(xb));
+            rs2[i & 1] = f2_add(rs2[i & 1], p2);
+            float a, b;
+            f2_unpack(p2, a, b);
             pr[i] = pack_bf16x2(a, b);
           }
           tmem_st8(tS + hh * 8, pr);
         }
-        const float rowsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        float rowsum;
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(rs2[0], a0, a1);
+          f2_unpack(rs2[1], b0, b1);
+          rowsum = (a0 + a1) + (b0 + b1);
+        }
         l += rowsum;
         tmem_st_wait();
         tc_fence_before();
