@@ -48,6 +48,9 @@ __all__ = [
     "softplus",
     "part_sizes",
     "feature_map",
+    "elu1",
+    "PHI_POLY",
+    "PHI_ELU1",
     "chunk_bounds",
     "rehyat_mask",
     "hybrid_attention_masked",
@@ -86,8 +89,22 @@ def part_sizes(F: int, P: int) -> list[int]:
     return [base + 1 if p < extra else base for p in range(P)]
 
 
-def feature_map(x: np.ndarray, W: np.ndarray, bias: np.ndarray | None, P: int) -> np.ndarray:
-    """Polynomial feature map phi(x) of ReHyAt overview §2.2.2.
+PHI_POLY = "poly"   # softplus parts raised to powers 1..P (ReHyAt overview §2.2.2)
+PHI_ELU1 = "elu1"   # elu(u) + 1, the linear-attention feature map of ReHyAt overview §2.1.2
+
+
+def elu1(u: np.ndarray) -> np.ndarray:
+    """elu(u) + 1: u + 1 for u > 0, e^u otherwise (continuous at 0, always > 0)."""
+    u = np.asarray(u, dtype=np.float64)
+    return np.where(u > 0, u + 1.0, np.exp(np.minimum(u, 0.0)))
+
+
+def feature_map(x: np.ndarray, W: np.ndarray, bias: np.ndarray | None, P: int,
+                kind: str = PHI_POLY) -> np.ndarray:
+    """Feature map phi(x): the polynomial map of ReHyAt overview §2.2.2 (kind "poly"), or the
+    elu(.) + 1 map of the linear attention in §2.1.2 (kind "elu1") applied after the same
+    grouped linear; with identity weights (G = D, W all ones, no bias) "elu1" is elu(x) + 1 of
+    the raw token, as printed there.
 
     x    : [n, D] tokens of one head.
     W    : [G, F/G, D/G] weights of the grouped 1x1 linear ("light MLP of grouped 1x1 convs"):
@@ -95,7 +112,7 @@ def feature_map(x: np.ndarray, W: np.ndarray, bias: np.ndarray | None, P: int) -
            [g*F/G, (g+1)*F/G) as u_g = x_g W[g]^T.
     bias : [F] or None.
     P    : number of parts; part p (1-based) of u is mapped to softplus(u_p) ** p, and the parts
-           are concatenated back in order.
+           are concatenated back in order (kind "poly"; ignored for "elu1").
     Returns phi [n, F], every entry > 0.
     """
     x = np.asarray(x, dtype=np.float64)
@@ -110,6 +127,10 @@ def feature_map(x: np.ndarray, W: np.ndarray, bias: np.ndarray | None, P: int) -
         u[:, g * Fg:(g + 1) * Fg] = x[:, g * Dg:(g + 1) * Dg] @ W[g].T
     if bias is not None:
         u = u + np.asarray(bias, dtype=np.float64)[None, :]
+    if kind == PHI_ELU1:
+        return elu1(u)
+    if kind != PHI_POLY:
+        raise ValueError(f"unknown feature map kind {kind!r}")
     out = np.empty_like(u)
     start = 0
     for p, size in enumerate(part_sizes(F, P), start=1):
@@ -193,7 +214,7 @@ def hybrid_attention_quadratic(q, k, v, phi_q, phi_k, frame_tokens: int, Tc: int
 
 
 def hybrid_attention_rows(q, k, v, Wq, bq, Wk, bk, P: int, frame_tokens: int, Tc: int, To: int,
-                          rows) -> np.ndarray:
+                          rows, kind: str = PHI_POLY) -> np.ndarray:
     """The quadratic form evaluated for selected query rows only (for sequences too long to
     evaluate whole): row i of chunk c = (i // L) // Tc weighs keys [w_c L, e_c L) by
     exp(q.k/sqrt(D)) and keys [0, w_c L) by phi_q(q).phi_k(k), shifted by the row max of the
@@ -205,9 +226,9 @@ def hybrid_attention_rows(q, k, v, Wq, bq, Wk, bk, P: int, frame_tokens: int, Tc
     bounds = chunk_bounds(T, Tc, To)
     rows = np.asarray(rows, dtype=np.int64)
     out = np.empty((len(rows), v.shape[1]))
-    phi_q = feature_map(q[rows], Wq, bq, P)
+    phi_q = feature_map(q[rows], Wq, bq, P, kind)
     need = max(bounds[(int(r) // L) // Tc][0] for r in rows) * L
-    phi_k = feature_map(k[:need], Wk, bk, P) if need > 0 else None
+    phi_k = feature_map(k[:need], Wk, bk, P, kind) if need > 0 else None
     for a, r in enumerate(rows):
         w, s, e = bounds[(int(r) // L) // Tc]
         logits = k[w * L:e * L] @ q[r] / math.sqrt(D)
@@ -274,10 +295,11 @@ def hybrid_attention_recurrent(q, k, v, phi_q, phi_k, frame_tokens: int, Tc: int
     return out
 
 
-def prefix_states(k, v, Wk, bk, P: int, frame_tokens: int, Tc: int, To: int):
+def prefix_states(k, v, Wk, bk, P: int, frame_tokens: int, Tc: int, To: int,
+                  kind: str = PHI_POLY):
     """Closed form of the state every chunk reads: S_c = phi_k[0:w_c]^T V[0:w_c],
     Z_c = phi_k[0:w_c]^T 1 (the linear region of chunk c, summed directly)."""
-    phi_k = feature_map(k, Wk, bk, P)
+    phi_k = feature_map(k, Wk, bk, P, kind)
     v = np.asarray(v, np.float64)
     T = k.shape[0] // frame_tokens
     Ss, Zs = [], []
@@ -289,7 +311,7 @@ def prefix_states(k, v, Wk, bk, P: int, frame_tokens: int, Tc: int, To: int):
 
 
 def chunk_forward(q_c, k_win, v_win, Wq, bq, Wk, bk, P: int, S, Z, frame_tokens: int,
-                  frames_before: int, chunk_frames: int, To: int):
+                  frames_before: int, chunk_frames: int, To: int, kind: str = PHI_POLY):
     """One streaming step (ReHyAt overview §5.2 loop, states per §2.3).
 
     q_c   : [chunk_frames*L, D] queries of the chunk that starts at frame `frames_before`.
@@ -304,8 +326,8 @@ def chunk_forward(q_c, k_win, v_win, Wq, bq, Wk, bk, P: int, S, Z, frame_tokens:
     w = frames_before - o
     if k_win.shape[0] != (o + chunk_frames) * L or q_c.shape[0] != chunk_frames * L:
         raise ValueError("window or chunk size does not match frames_before/chunk_frames/To")
-    phi_q = feature_map(q_c, Wq, bq, P)
-    phi_k = feature_map(k_win, Wk, bk, P)
+    phi_q = feature_map(q_c, Wq, bq, P, kind)
+    phi_k = feature_map(k_win, Wk, bk, P, kind)
     out = _window_output(np.asarray(q_c, np.float64), np.asarray(k_win, np.float64),
                          np.asarray(v_win, np.float64), phi_q, np.asarray(S, np.float64),
                          np.asarray(Z, np.float64), has_linear=w > 0)
@@ -321,7 +343,7 @@ def chunk_forward(q_c, k_win, v_win, Wq, bq, Wk, bk, P: int, S, Z, frame_tokens:
 # ---------------------------------------------------------------------------------------------
 
 def hybrid_attention_bruteforce(q, k, v, Wq, bq, Wk, bk, P: int, frame_tokens: int, Tc: int,
-                                To: int) -> np.ndarray:
+                                To: int, kind: str = PHI_POLY) -> np.ndarray:
     """Pure-Python loops.  For every query token i (frame t_i, chunk c = t_i // Tc) and every key
     token j (frame t_j): future chunks (t_j >= end of chunk c) are skipped; frames inside
     [max(0, c*Tc - To), end of chunk c) contribute exp(q.k/sqrt(D)); earlier frames contribute
@@ -343,6 +365,8 @@ def hybrid_attention_bruteforce(q, k, v, Wq, bq, Wk, bk, P: int, frame_tokens: i
             for d in range(Dg):
                 acc += float(W[g][r][d]) * x[g * Dg + d]
             u.append(acc)
+        if kind == PHI_ELU1:
+            return [a + 1.0 if a > 0 else math.exp(a) for a in u]
         res, f = [], 0
         for p, size in enumerate(part_sizes(F, P), start=1):
             for _ in range(size):

@@ -4,6 +4,9 @@ What pins what:
 * hand-derived worked examples (tests/golden/worked_examples.json) -> the output formula, the
   window/linear split, the overlap, the part powers, bidirectional softmax inside a chunk;
 * torch conv1d(groups=G) + torch softplus                             -> the feature map;
+* torch elu + 1 on the raw token (identity grouped linear)           -> the elu+1 feature map;
+* the linear attention of the pages' §2.1.2 (phi = elu + 1, no chunks)
+  and a scalar brute force with elu + 1                              -> the elu+1 hybrid;
 * torch scaled_dot_product_attention (float64)                       -> the single-chunk case;
 * normalised linear attention written with cumulative sums           -> the empty-window case;
 * scalar brute force (own phi, own frame classification)             -> everything, tiny sizes;
@@ -199,8 +202,48 @@ def check_rows_form(mod):
         np.testing.assert_allclose(got, quad[rows], rtol=1e-12, atol=1e-12)
 
 
+def check_elu1_featmap(mod):
+    """kind "elu1" with identity weights (G = D groups of 1 x 1) and no bias is elu(x) + 1 of the
+    raw token, as in the linear attention of ReHyAt overview §2.1.2; with general weights it is
+    elu(u) + 1 of the same grouped linear u as the polynomial map."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((40, 16)) * 2.0
+    eye = np.ones((16, 1, 1))
+    got = mod.feature_map(x, eye, None, 1, mod.PHI_ELU1)
+    want = (torch.nn.functional.elu(torch.from_numpy(x)) + 1.0).numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-14, atol=1e-15)
+    _, _, _, W, b, _, _ = _rand_problem(rng, 1, 1, 16, 8, 4, bias=0.3)
+    u = torch.nn.functional.conv1d(torch.from_numpy(x).T[None], torch.from_numpy(W).reshape(8, 4, 1),
+                                   bias=torch.from_numpy(b), groups=4)[0].T
+    want = (torch.nn.functional.elu(u) + 1.0).numpy()
+    np.testing.assert_allclose(mod.feature_map(x, W, b, 3, mod.PHI_ELU1), want, rtol=1e-13, atol=1e-14)
+
+
+def check_elu1_hybrid(mod):
+    """With phi = elu + 1: one chunk with no window is the pages' linear attention
+    phi(Q) (phi(K)^T V) normalised; the chunked hybrid matches the scalar brute force."""
+    rng = np.random.default_rng(12)
+    T, L, D = 4, 3, 8
+    q, k, v, _, _, _, _ = _rand_problem(rng, T, L, D, 8, 2)
+    eye = np.ones((D, 1, 1))
+    pq, pk = mod.feature_map(q, eye, None, 1, mod.PHI_ELU1), mod.feature_map(k, eye, None, 1, mod.PHI_ELU1)
+    M = np.full((T, T), mod.SET_LINEAR, dtype=np.int8)
+    got = mod.hybrid_attention_masked(q, k, v, pq, pk, L, M)
+    eq = np.where(q > 0, q + 1, np.exp(q)); ek = np.where(k > 0, k + 1, np.exp(k))
+    want = (eq @ (ek.T @ v)) / (eq @ ek.sum(axis=0))[:, None]
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    for (T, L, Tc, To) in [(6, 2, 2, 1), (5, 3, 3, 0), (7, 1, 1, 2)]:
+        q, k, v, Wq, bq, Wk, bk = _rand_problem(rng, T, L, 4, 4, 2, bias=0.2)
+        pq = mod.feature_map(q, Wq, bq, 1, mod.PHI_ELU1)
+        pk = mod.feature_map(k, Wk, bk, 1, mod.PHI_ELU1)
+        quad = mod.hybrid_attention_quadratic(q, k, v, pq, pk, L, Tc, To)
+        brute = mod.hybrid_attention_bruteforce(q, k, v, Wq, bq, Wk, bk, 1, L, Tc, To, mod.PHI_ELU1)
+        np.testing.assert_allclose(quad, brute, rtol=1e-11, atol=1e-12)
+
+
 PINS = [check_rows_form, check_golden, check_featmap_conv1d, check_single_chunk_is_softmax, check_linear_only,
-        check_bruteforce, check_recurrent_and_streaming, check_invariants]
+        check_bruteforce, check_recurrent_and_streaming, check_invariants, check_elu1_featmap,
+        check_elu1_hybrid]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -238,6 +281,10 @@ MUTATIONS = [
     ("bias dropped", "u = u + np.asarray(bias, dtype=np.float64)[None, :]", "u = u"),
     ("linear normaliser dropped in the recurrent form",
      "den = den + shift * (phi_q_c @ Z)[:, None]", "den = den"),
+    ("elu + 1 linear for negative inputs", "np.where(u > 0, u + 1.0, np.exp(np.minimum(u, 0.0)))",
+     "np.where(u > 0, u + 1.0, u + 1.0)"),
+    ("elu + 1 without the + 1", "np.where(u > 0, u + 1.0, np.exp(np.minimum(u, 0.0)))",
+     "np.where(u > 0, u, np.exp(np.minimum(u, 0.0)) - 1.0)"),
     ("streaming fold uses the chunk's own To twice",
      "w_next = max(0, frames_before + chunk_frames - To)",
      "w_next = max(0, frames_before + chunk_frames - 2 * To)"),
