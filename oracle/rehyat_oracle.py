@@ -53,6 +53,8 @@ __all__ = [
     "PHI_ELU1",
     "chunk_bounds",
     "rehyat_mask",
+    "schedule_bounds",
+    "schedule_mask",
     "hybrid_attention_masked",
     "hybrid_attention_quadratic",
     "hybrid_attention_recurrent",
@@ -156,6 +158,31 @@ def chunk_bounds(T: int, Tc: int, To: int) -> list[tuple[int, int, int]]:
         w = max(0, s - To)
         out.append((w, s, e))
     return out
+
+
+def schedule_bounds(chunk_frames, overlaps) -> list[tuple[int, int, int]]:
+    """(w_c, s_c, e_c) of a variable schedule (ReHyAt overview §5.2: a longer chunk for key
+    frames such as the first, more overlap where motion is strong): chunk c owns the next
+    chunk_frames[c] frames and its softmax window reaches overlaps[c] frames back."""
+    if len(chunk_frames) != len(overlaps) or not chunk_frames:
+        raise ValueError("one overlap per chunk")
+    out, s = [], 0
+    for cf, o in zip(chunk_frames, overlaps):
+        if cf < 1 or o < 0:
+            raise ValueError("need chunk_frames >= 1 and overlaps >= 0")
+        out.append((max(0, s - o), s, s + cf))
+        s += cf
+    return out
+
+
+def schedule_mask(bounds) -> np.ndarray:
+    """Frame-level set assignment of any chunk schedule given as (w_c, s_c, e_c) triples."""
+    T = bounds[-1][2]
+    M = np.full((T, T), SET_NONE, dtype=np.int8)
+    for (w, s, e) in bounds:
+        M[s:e, w:e] = SET_SOFTMAX
+        M[s:e, 0:w] = SET_LINEAR
+    return M
 
 
 def rehyat_mask(T: int, Tc: int, To: int) -> np.ndarray:
@@ -311,7 +338,8 @@ def prefix_states(k, v, Wk, bk, P: int, frame_tokens: int, Tc: int, To: int,
 
 
 def chunk_forward(q_c, k_win, v_win, Wq, bq, Wk, bk, P: int, S, Z, frame_tokens: int,
-                  frames_before: int, chunk_frames: int, To: int, kind: str = PHI_POLY):
+                  frames_before: int, chunk_frames: int, To: int, kind: str = PHI_POLY,
+                  To_next: int | None = None):
     """One streaming step (ReHyAt overview §5.2 loop, states per §2.3).
 
     q_c   : [chunk_frames*L, D] queries of the chunk that starts at frame `frames_before`.
@@ -319,8 +347,9 @@ def chunk_forward(q_c, k_win, v_win, Wq, bq, Wk, bk, P: int, S, Z, frame_tokens:
             followed by the chunk's own frames (the softmax window).
     S, Z  : states holding every frame before the window.
     Returns (out, S_new, Z_new).  After the output is formed, the window frames that the next
-    chunk (same To) no longer sees, [w_c, w_{c+1}) with w_{c+1} = max(0, frames_before +
-    chunk_frames - To), are folded into the returned states."""
+    chunk no longer sees, [w_c, w_{c+1}) with w_{c+1} = max(0, frames_before + chunk_frames -
+    To_next), are folded into the returned states; To_next is the next chunk's overlap (the
+    same To unless the schedule varies it)."""
     L = frame_tokens
     o = min(To, frames_before)
     w = frames_before - o
@@ -331,7 +360,11 @@ def chunk_forward(q_c, k_win, v_win, Wq, bq, Wk, bk, P: int, S, Z, frame_tokens:
     out = _window_output(np.asarray(q_c, np.float64), np.asarray(k_win, np.float64),
                          np.asarray(v_win, np.float64), phi_q, np.asarray(S, np.float64),
                          np.asarray(Z, np.float64), has_linear=w > 0)
-    w_next = max(0, frames_before + chunk_frames - To)
+    if To_next is None:
+        To_next = To
+    w_next = max(0, frames_before + chunk_frames - To_next)
+    if w_next < w:
+        raise ValueError("the next chunk's overlap reaches frames already folded into S")
     nd = (w_next - w) * L
     S_new = np.asarray(S, np.float64) + phi_k[:nd].T @ np.asarray(v_win, np.float64)[:nd]
     Z_new = np.asarray(Z, np.float64) + phi_k[:nd].sum(axis=0)

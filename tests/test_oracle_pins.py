@@ -241,9 +241,39 @@ def check_elu1_hybrid(mod):
         np.testing.assert_allclose(quad, brute, rtol=1e-11, atol=1e-12)
 
 
+def check_variable_schedule(mod):
+    """A variable schedule (longer first chunk, per-chunk overlap) streamed with the recurrent
+    step, each call folding what the next chunk's window no longer holds, equals the quadratic
+    form under the schedule's frame mask; a uniform schedule gives the standard mask."""
+    rng = np.random.default_rng(13)
+    assert (mod.schedule_mask(mod.schedule_bounds([3, 3, 3, 1], [1, 1, 1, 1]))
+            == mod.rehyat_mask(10, 3, 1)).all()
+    L = 2
+    for cfs, ovs in [([5, 3, 3, 2], [0, 1, 2, 1]), ([1, 2, 4, 1, 3], [0, 1, 2, 2, 1]),
+                     ([4, 4], [0, 4])]:
+        T = sum(cfs)
+        q, k, v, Wq, bq, Wk, bk = _rand_problem(rng, T, L, 8, 8, 2, bias=0.1)
+        pq, pk = mod.feature_map(q, Wq, bq, 2), mod.feature_map(k, Wk, bk, 2)
+        bounds = mod.schedule_bounds(cfs, ovs)
+        want = mod.hybrid_attention_masked(q, k, v, pq, pk, L, mod.schedule_mask(bounds))
+        S, Z = np.zeros((8, 8)), np.zeros(8)
+        got = []
+        for c, (w, s0, e) in enumerate(bounds):
+            nxt = ovs[c + 1] if c + 1 < len(ovs) else ovs[c]
+            o, S, Z = mod.chunk_forward(q[s0 * L:e * L], k[w * L:e * L], v[w * L:e * L], Wq, bq,
+                                        Wk, bk, 2, S, Z, L, s0, e - s0, ovs[c], To_next=nxt)
+            got.append(o)
+        np.testing.assert_allclose(np.concatenate(got), want, rtol=1e-12, atol=1e-12)
+    # a next overlap reaching past the current window needs frames already folded: refused
+    q, k, v, Wq, bq, Wk, bk = _rand_problem(rng, 4, L, 8, 8, 2)
+    with pytest.raises(ValueError):
+        mod.chunk_forward(q[2 * L:3 * L], k[L:3 * L], v[L:3 * L], Wq, bq, Wk, bk, 2, np.zeros((8, 8)),
+                          np.zeros(8), L, 2, 1, 1, To_next=3)
+
+
 PINS = [check_rows_form, check_golden, check_featmap_conv1d, check_single_chunk_is_softmax, check_linear_only,
         check_bruteforce, check_recurrent_and_streaming, check_invariants, check_elu1_featmap,
-        check_elu1_hybrid]
+        check_elu1_hybrid, check_variable_schedule]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -285,9 +315,12 @@ MUTATIONS = [
      "np.where(u > 0, u + 1.0, u + 1.0)"),
     ("elu + 1 without the + 1", "np.where(u > 0, u + 1.0, np.exp(np.minimum(u, 0.0)))",
      "np.where(u > 0, u, np.exp(np.minimum(u, 0.0)) - 1.0)"),
+    ("streaming fold ignores the next chunk's overlap",
+     "w_next = max(0, frames_before + chunk_frames - To_next)",
+     "w_next = max(0, frames_before + chunk_frames - To)"),
     ("streaming fold uses the chunk's own To twice",
-     "w_next = max(0, frames_before + chunk_frames - To)",
-     "w_next = max(0, frames_before + chunk_frames - 2 * To)"),
+     "w_next = max(0, frames_before + chunk_frames - To_next)",
+     "w_next = max(0, frames_before + chunk_frames - 2 * To_next)"),
 ]
 
 
@@ -301,6 +334,6 @@ def test_planted_mistake_is_caught(desc, old, new):
     for pin in PINS:
         try:
             pin(mod)
-        except (AssertionError, ValueError, IndexError):
+        except (AssertionError, ValueError, IndexError, pytest.fail.Exception):
             failed.append(pin.__name__)
     assert failed, f"no pin caught: {desc}"
