@@ -15,6 +15,8 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "li
 
 REHYAT_F32 = 0
 REHYAT_BF16 = 1
+PHI_POLY = 0   # softplus parts raised to powers 1..P
+PHI_ELU1 = 1   # elu(u) + 1
 
 STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_SHAPE", -3: "ERR_DTYPE", -4: "ERR_WORKSPACE",
           -5: "ERR_CUDA", -6: "ERR_TIMEOUT", -7: "ERR_ALIGN"}
@@ -22,7 +24,7 @@ STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_SHAPE", -3: "ERR_DTYPE", -4: "ERR_WOR
 EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_forward_workspace_size", "rehyat_forward", "rehyat_forward_states",
             "rehyat_forward_phiq", "rehyat_forward_attend", "rehyat_chunk_workspace_size",
-            "rehyat_chunk_forward", "rehyat_chunk_forward_static", "rehyat_chunk_states",
+            "rehyat_chunk_forward", "rehyat_chunk_forward_sched", "rehyat_chunk_forward_static", "rehyat_chunk_states",
             "rehyat_selftest_wait_timeout", "rehyat_sync_status"]
 
 
@@ -34,7 +36,7 @@ class RehyatError(RuntimeError):
 
 class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("D", ctypes.c_int), ("F", ctypes.c_int),
-                ("G", ctypes.c_int), ("P", ctypes.c_int)]
+                ("G", ctypes.c_int), ("P", ctypes.c_int), ("phi", ctypes.c_int)]
 
 
 _lib = None
@@ -73,6 +75,8 @@ def load() -> ctypes.CDLL:
                                               ctypes.POINTER(c_size_t)]
     L.rehyat_chunk_forward.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
                                        P, P, P, P, P, c_size_t, P]
+    L.rehyat_chunk_forward_sched.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, c_int, P, P,
+                                             P, P, P, P, P, P, P, P, P, c_size_t, P]
     L.rehyat_chunk_forward_static.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P,
                                               P, P, P, P, P, P, P]
     L.rehyat_chunk_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
@@ -125,25 +129,26 @@ def _weights(W: torch.Tensor, b: torch.Tensor | None):
     return W, b
 
 
-def dims_of(x: torch.Tensor, W: torch.Tensor, P: int) -> Dims:
-    """Dims from x [B,H,n,D] and W [H,G,F/G,D/G]."""
+def dims_of(x: torch.Tensor, W: torch.Tensor, P: int, phi: int = 0) -> Dims:
+    """Dims from x [B,H,n,D] and W [H,G,F/G,D/G]; phi is PHI_POLY or PHI_ELU1."""
     B, H, _, D = x.shape
     Hw, G, Fg, _ = W.shape
     if Hw != H:
         raise ValueError("W has a different head count than x")
-    return Dims(B, H, D, G * Fg, G, P)
+    return Dims(B, H, D, G * Fg, G, P, phi)
 
 
 def version() -> int:
     return load().rehyat_version()
 
 
-def featmap(x: torch.Tensor, W: torch.Tensor, bias: torch.Tensor | None, P: int) -> torch.Tensor:
+def featmap(x: torch.Tensor, W: torch.Tensor, bias: torch.Tensor | None, P: int,
+            phi: int = 0) -> torch.Tensor:
     """phi(x) for x [B,H,n,D] -> [B,H,n,F] (same dtype as x)."""
     L = load()
     dev = _dev(x, W, bias)
     _weights(W, bias)
-    d = dims_of(x, W, P)
+    d = dims_of(x, W, P, phi)
     phi = torch.empty(x.shape[0], x.shape[1], x.shape[2], d.F, dtype=x.dtype, device=dev)
     _check(L.rehyat_featmap(d, _dtype_code(x), x.shape[2], _ptr(x), _ptr(W), _ptr(bias),
                             _ptr(phi), _stream(dev)))
@@ -169,13 +174,13 @@ def _workspace(nbytes: int, dev: torch.device, workspace: torch.Tensor | None) -
     return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
 
 
-def forward(q, k, v, Wq, bq, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
+def forward(q, k, v, Wq, bq, Wk, bk, *, P: int, phi: int = 0, frame_tokens: int, Tc: int, To: int,
             out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
     """Hybrid attention over a whole sequence: q, k, v [B,H,T*frame_tokens,D] -> out."""
     lib = load()
     dev = _dev(q, k, v, Wq, bq, Wk, bk)
     _weights(Wq, bq), _weights(Wk, bk)
-    d = dims_of(q, Wq, P)
+    d = dims_of(q, Wq, P, phi)
     N = q.shape[2]
     if N % frame_tokens:
         raise ValueError("sequence length is not a multiple of frame_tokens")
@@ -190,12 +195,12 @@ def forward(q, k, v, Wq, bq, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: 
     return out
 
 
-def forward_states(k, v, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
+def forward_states(k, v, Wk, bk, *, P: int, phi: int = 0, frame_tokens: int, Tc: int, To: int,
                    workspace: torch.Tensor) -> torch.Tensor:
     """First phase of `forward`: fills `workspace` with the state every chunk reads."""
     lib = load()
     dev = _dev(k, v, Wk, bk, workspace)
-    d = dims_of(k, Wk, P)
+    d = dims_of(k, Wk, P, phi)
     T = k.shape[2] // frame_tokens
     _check(lib.rehyat_forward_states(d, _dtype_code(k), T, frame_tokens, Tc, To, _ptr(k), _ptr(v),
                                      _ptr(Wk), _ptr(bk), _ptr(workspace), workspace.numel(),
@@ -203,12 +208,12 @@ def forward_states(k, v, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
     return workspace
 
 
-def forward_phiq(q, Wq, bq, *, P: int, frame_tokens: int, Tc: int, To: int,
+def forward_phiq(q, Wq, bq, *, P: int, phi: int = 0, frame_tokens: int, Tc: int, To: int,
                  workspace: torch.Tensor) -> torch.Tensor:
     """Second phase of `forward`: phi_q of the query rows that read a state, into `workspace`."""
     lib = load()
     dev = _dev(q, Wq, bq, workspace)
-    d = dims_of(q, Wq, P)
+    d = dims_of(q, Wq, P, phi)
     T = q.shape[2] // frame_tokens
     _check(lib.rehyat_forward_phiq(d, _dtype_code(q), T, frame_tokens, Tc, To, _ptr(q), _ptr(Wq),
                                    _ptr(bq), _ptr(workspace), workspace.numel(), _stream(dev)))
@@ -227,12 +232,12 @@ def forward_attend(q, k, v, *, dims: Dims, frame_tokens: int, Tc: int, To: int,
     return out
 
 
-def chunk_states(k, v, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
+def chunk_states(k, v, Wk, bk, *, P: int, phi: int = 0, frame_tokens: int, Tc: int, To: int,
                  workspace: torch.Tensor | None = None):
     """States each chunk of `forward` reads: S [B,H,C,F,D], Z [B,H,C,F] (fp32)."""
     lib = load()
     dev = _dev(k, v, Wk, bk)
-    d = dims_of(k, Wk, P)
+    d = dims_of(k, Wk, P, phi)
     N = k.shape[2]
     T = N // frame_tokens
     C = -(-T // Tc)
@@ -246,32 +251,37 @@ def chunk_states(k, v, Wk, bk, *, P: int, frame_tokens: int, Tc: int, To: int,
     return S, Z
 
 
-def chunk_forward(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, frame_tokens: int,
-                  frames_before: int, To: int, out: torch.Tensor | None = None,
-                  workspace: torch.Tensor | None = None):
-    """One streaming step; S [B,H,F,D] and Z [B,H,F] (fp32) are updated in place."""
+def chunk_forward(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, phi: int = 0, frame_tokens: int,
+                  frames_before: int, To: int, To_next: int | None = None,
+                  out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """One streaming step; S [B,H,F,D] and Z [B,H,F] (fp32) are updated in place.  To_next (the
+    overlap of the next call, for a variable schedule) defaults to To."""
     lib = load()
     dev = _dev(q, k_win, v_win, Wq, bq, Wk, bk, S, Z)
-    d = dims_of(q, Wq, P)
+    d = dims_of(q, Wq, P, phi)
     chunk_frames = q.shape[2] // frame_tokens
     code = _dtype_code(q)
     ws = _workspace(chunk_workspace_size(d, code, frame_tokens, chunk_frames, To), dev, workspace)
     if out is None:
         out = torch.empty_like(q)
-    _check(lib.rehyat_chunk_forward(d, code, frame_tokens, frames_before, chunk_frames, To,
-                                    _ptr(q), _ptr(k_win), _ptr(v_win), _ptr(Wq), _ptr(bq),
-                                    _ptr(Wk), _ptr(bk), _ptr(S), _ptr(Z), _ptr(out), _ptr(ws),
-                                    ws.numel(), _stream(dev)))
+    args = (_ptr(q), _ptr(k_win), _ptr(v_win), _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(S),
+            _ptr(Z), _ptr(out), _ptr(ws), ws.numel(), _stream(dev))
+    if To_next is None:
+        _check(lib.rehyat_chunk_forward(d, code, frame_tokens, frames_before, chunk_frames, To,
+                                        *args))
+    else:
+        _check(lib.rehyat_chunk_forward_sched(d, code, frame_tokens, frames_before, chunk_frames,
+                                              To, To_next, *args))
     return out
 
 
-def chunk_forward_static(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, frame_tokens: int,
+def chunk_forward_static(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, phi: int = 0, frame_tokens: int,
                          frames_before: int, To: int, out: torch.Tensor | None = None):
     """chunk_forward without a workspace: the library's own fixed device scratch is used (for
     callers that cannot allocate); bf16 only."""
     lib = load()
     dev = _dev(q, k_win, v_win, Wq, bq, Wk, bk, S, Z)
-    d = dims_of(q, Wq, P)
+    d = dims_of(q, Wq, P, phi)
     chunk_frames = q.shape[2] // frame_tokens
     if out is None:
         out = torch.empty_like(q)

@@ -23,6 +23,8 @@ class Workload:
     bias           : constant filled into the feature-map biases (0 in the standard workloads).
     seed           : generator seed.
     mode           : "full" (one call over the sequence) or "stream" (chunk-by-chunk calls).
+    phi            : feature map after the grouped linear: "poly" (softplus parts raised to
+                     powers 1..P) or "elu1" (elu + 1).
     """
     name: str
     B: int
@@ -41,6 +43,12 @@ class Workload:
     bias: float = 0.0
     seed: int = 0
     mode: str = "full"
+    phi: str = "poly"
+
+    @property
+    def phi_code(self) -> int:
+        """The rehyat_phi value of `phi` (0 polynomial, 1 elu + 1)."""
+        return {"poly": 0, "elu1": 1}[self.phi]
 
     @property
     def frame_tokens(self) -> int:

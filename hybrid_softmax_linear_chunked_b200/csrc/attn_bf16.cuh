@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid < 256 && has_linear) {
     for (int i = tid; i < kFD; i += 256) {
-      sPw[i] = static_cast<uint8_t>(part_power(i, kFD, p.P));
+      sPw[i] = static_cast<uint8_t>(feature_power(i, kFD, p.P));
       sB[i] = p.bq ? p.bq[(size_t)h * kFD + i] : 0.f;
       sZ[i] = p.Z[((size_t)bh * p.n_states + c) * kFD + i];
     }

@@ -21,6 +21,16 @@ __host__ __device__ __forceinline__ int part_power(int f, int F, int P) {
   return p + 1;
 }
 
+// Entry of the per-feature table the kernels keep: the part power, or 0 for the elu + 1 map
+// (kernels receive P = 0 for it; a power of 0 never occurs in the polynomial map).
+__host__ __device__ __forceinline__ int feature_power(int f, int F, int P) {
+  return P == 0 ? 0 : part_power(f, F, P);
+}
+
+// elu(u) + 1: u + 1 for u > 0, e^u otherwise.
+__device__ __forceinline__ float elu1_fast(float u) { return u > 0.f ? u + 1.f : __expf(u); }
+__device__ __forceinline__ float elu1_accurate(float u) { return u > 0.f ? u + 1.f : expf(u); }
+
 __device__ __forceinline__ float int_pow(float x, int p) {
   float r = x;
   for (int i = 1; i < p; ++i) r *= x;
@@ -59,9 +69,16 @@ __device__ __forceinline__ float softplus_fast(float u) {
 __device__ __forceinline__ void phi16(const uint32_t* u, int f0, const float* bias,
                                       const uint8_t* pw, float scale, uint32_t* packed) {
   float ph[16];
+  const int p_first = pw[f0], p_last = pw[f0 + 15];
+  if (p_last == 0) {  // elu + 1 map (the whole table is 0)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) ph[i] = elu1_fast(__uint_as_float(u[i]) + bias[f0 + i]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(ph[2 * i] * scale, ph[2 * i + 1] * scale);
+    return;
+  }
 #pragma unroll
   for (int i = 0; i < 16; ++i) ph[i] = softplus_fast(__uint_as_float(u[i]) + bias[f0 + i]);
-  const int p_first = pw[f0], p_last = pw[f0 + 15];
   if (p_first == p_last) {
     if (p_first == 2) {
 #pragma unroll
@@ -140,8 +157,12 @@ __global__ void __launch_bounds__(128) featmap_kernel(const Tin* __restrict__ x,
       const float* w = sW + (g * Fg + o) * Dg;
       float u = sB[f];
       for (int i = 0; i < Dg; ++i) u = fmaf(w[i], xr[g * Dg + i], u);
-      const float sp = kAccurate ? softplus_accurate(u) : softplus_fast(u);
-      out[f] = from_f32<Tout>(int_pow(sp, part_power(f, F, P)));
+      if (P == 0) {
+        out[f] = from_f32<Tout>(kAccurate ? elu1_accurate(u) : elu1_fast(u));
+      } else {
+        const float sp = kAccurate ? softplus_accurate(u) : softplus_fast(u);
+        out[f] = from_f32<Tout>(int_pow(sp, part_power(f, F, P)));
+      }
     }
   }
 }

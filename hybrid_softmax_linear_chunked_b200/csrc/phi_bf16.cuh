@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   for (int i = tid; i < kFD; i += kThreads) {
     sB[i] = p.bias ? p.bias[(size_t)h * kFD + i] : 0.f;
-    sPw[i] = static_cast<uint8_t>(part_power(i, kFD, p.P));
+    sPw[i] = static_cast<uint8_t>(feature_power(i, kFD, p.P));
   }
   tc_fence_before();
   __syncthreads();

@@ -47,6 +47,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// The kernels take the part count P with P = 0 standing for the elu + 1 map.
+int kernel_P(const rehyat_dims& d) { return d.phi == REHYAT_PHI_ELU1 ? 0 : d.P; }
+
 int check_dims(const rehyat_dims& d, rehyat_dtype dt) {
   if (d.B < 1 || d.H < 1 || d.D < 1 || d.F < 1 || d.G < 1 || d.P < 1)
     return fail(REHYAT_ERR_ARG, "dims must be positive (B=%d H=%d D=%d F=%d G=%d P=%d)", d.B, d.H,
@@ -54,6 +57,8 @@ int check_dims(const rehyat_dims& d, rehyat_dtype dt) {
   if (d.D % d.G || d.F % d.G)
     return fail(REHYAT_ERR_ARG, "G=%d must divide D=%d and F=%d", d.G, d.D, d.F);
   if (d.P > d.F) return fail(REHYAT_ERR_ARG, "P=%d exceeds F=%d", d.P, d.F);
+  if (d.phi != REHYAT_PHI_POLY && d.phi != REHYAT_PHI_ELU1)
+    return fail(REHYAT_ERR_ARG, "unknown feature map kind phi=%d", d.phi);
   if (dt != REHYAT_F32 && dt != REHYAT_BF16) return fail(REHYAT_ERR_DTYPE, "unknown dtype %d", (int)dt);
   return REHYAT_OK;
 }
@@ -180,14 +185,14 @@ struct ChunkPlan {
 };
 
 ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_before,
-                     int chunk_frames, int To) {
+                     int chunk_frames, int To, int To_next) {
   ChunkPlan p{};
   const size_t BH = (size_t)d.B * d.H;
   p.o = To < frames_before ? To : frames_before;
   p.nq = chunk_frames * L;
   p.nkv = (p.o + chunk_frames) * L;
   const int w = frames_before - p.o;
-  int w_next = frames_before + chunk_frames - To;
+  int w_next = frames_before + chunk_frames - To_next;
   if (w_next < 0) w_next = 0;
   p.fold_rows = (w_next - w) * L;
   if (p.fold_rows < 0) p.fold_rows = 0;
@@ -228,12 +233,12 @@ int launch_featmap(const rehyat_dims& d, rehyat_dtype dt, int n, const void* x, 
     auto k = rehyat::featmap_kernel<__nv_bfloat16, __nv_bfloat16, false>;
     RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), "featmap attr"));
     k<<<grid, 128, smem, st>>>(static_cast<const __nv_bfloat16*>(x), W, b,
-                               static_cast<__nv_bfloat16*>(phi), n, d.H, d.D, d.F, d.G, d.P);
+                               static_cast<__nv_bfloat16*>(phi), n, d.H, d.D, d.F, d.G, kernel_P(d));
   } else {
     auto k = rehyat::featmap_kernel<float, float, true>;
     RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem), "featmap attr"));
     k<<<grid, 128, smem, st>>>(static_cast<const float*>(x), W, b, static_cast<float*>(phi), n,
-                               d.H, d.D, d.F, d.G, d.P);
+                               d.H, d.D, d.F, d.G, kernel_P(d));
   }
   return cuda_check(cudaGetLastError(), "featmap launch");
 }
@@ -265,7 +270,7 @@ int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int 
   if (per_cta > n_tiles) per_cta = n_tiles;
   rehyat::phi::Params pp{};
   pp.row0 = row0; pp.n_rows = n_rows; pp.rows_per_bh = rows_per_bh; pp.tiles_per_cta = per_cta;
-  pp.H = d.H; pp.P = d.P; pp.bias = bias; pp.phi = phi;
+  pp.H = d.H; pp.P = kernel_P(d); pp.bias = bias; pp.phi = phi;
   auto k = rehyat::phi::featmap_tc_kernel;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)rehyat::phi::kSmemBytes),
@@ -319,7 +324,7 @@ int forward_states_bf16(const rehyat_dims& d, int T, int L, int Tc, int To, cons
     RH_TRY(make_map(&mv, v, d.D, N, BH));
     RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mw, st));
     rehyat::state::FoldParams fp{};
-    fp.L = L; fp.H = d.H; fp.P = d.P; fp.T = T; fp.Tc = Tc; fp.To = To; fp.kv_frame0 = 0;
+    fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.T = T; fp.Tc = Tc; fp.To = To; fp.kv_frame0 = 0;
     fp.single_rows = -1; fp.n_fold = pl.n_fold; fp.splits = pl.splits;
     fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
     RH_TRY(launch_fold_bf16(mk, mv, mw, fp, dim3(pl.splits, pl.n_fold, BH), st));
@@ -404,7 +409,7 @@ extern "C" {
 
 const char* rehyat_last_error(void) { return g_msg; }
 
-int rehyat_version(void) { return 100; }
+int rehyat_version(void) { return 101; }
 
 int rehyat_featmap(rehyat_dims d, rehyat_dtype dt, int n_tokens, const void* x, const float* W,
                    const float* bias, void* phi, void* stream) {
@@ -506,7 +511,7 @@ int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
     RH_TRY(make_map(&mphi, ws + pl.phiq_bf16, d.F, N, BH));
     rehyat::attn::Params ap{};
     ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
-    ap.H = d.H; ap.P = d.P; ap.n_states = pl.C; ap.nq_rows = (int)N;
+    ap.H = d.H; ap.P = kernel_P(d); ap.n_states = pl.C; ap.nq_rows = (int)N;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
     ap.bq = nullptr;  // phi_q comes finished from the workspace
     ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
@@ -550,7 +555,7 @@ int rehyat_chunk_workspace_size(rehyat_dims d, rehyat_dtype dt, int frame_tokens
   RH_TRY(check_path_shape(d, dt));
   RH_TRY(check_sched(chunk_frames, frame_tokens, 1, To));
   if (!bytes) return fail(REHYAT_ERR_ARG, "null bytes pointer");
-  *bytes = plan_chunk(d, dt, frame_tokens, To, chunk_frames, To).total;
+  *bytes = plan_chunk(d, dt, frame_tokens, To, chunk_frames, To, To).total;
   return REHYAT_OK;
 }
 
@@ -559,17 +564,37 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int L, int frames_befor
                          const void* v_win, const float* Wq, const float* bq, const float* Wk,
                          const float* bk, float* S, float* Z, void* out, void* workspace,
                          size_t ws_bytes, void* stream) {
+  return rehyat_chunk_forward_sched(d, dt, L, frames_before, chunk_frames, To, To, q, k_win,
+                                    v_win, Wq, bq, Wk, bk, S, Z, out, workspace, ws_bytes,
+                                    stream);
+}
+
+int rehyat_chunk_forward_sched(rehyat_dims d, rehyat_dtype dt, int L, int frames_before,
+                               int chunk_frames, int To, int To_next, const void* q,
+                               const void* k_win, const void* v_win, const float* Wq,
+                               const float* bq, const float* Wk, const float* bk, float* S,
+                               float* Z, void* out, void* workspace, size_t ws_bytes,
+                               void* stream) {
   g_msg[0] = 0;
   RH_TRY(check_dims(d, dt));
   RH_TRY(check_path_shape(d, dt));
   RH_TRY(check_sched(chunk_frames, L, 1, To));
   if (frames_before < 0) return fail(REHYAT_ERR_ARG, "frames_before must be >= 0");
+  if (To_next < 0) return fail(REHYAT_ERR_ARG, "To_next must be >= 0");
+  {
+    const int o = To < frames_before ? To : frames_before;
+    const int seen = frames_before + chunk_frames;
+    if ((To_next < seen ? To_next : seen) > o + chunk_frames)
+      return fail(REHYAT_ERR_ARG,
+                  "To_next=%d reaches before this window (%d frames): those frames are already "
+                  "folded into S", To_next, o + chunk_frames);
+  }
   if (!q || !k_win || !v_win || !Wq || !Wk || !S || !Z || !out)
     return fail(REHYAT_ERR_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k_win) || !aligned16(v_win) || !aligned16(out))
     return fail(REHYAT_ERR_ALIGN, "q/k_win/v_win/out not 16-byte aligned");
-  const ChunkPlan pl = plan_chunk(d, dt, L, frames_before, chunk_frames, To);
-  const size_t need = plan_chunk(d, dt, L, To, chunk_frames, To).total;
+  const ChunkPlan pl = plan_chunk(d, dt, L, frames_before, chunk_frames, To, To_next);
+  const size_t need = plan_chunk(d, dt, L, To, chunk_frames, To, To).total;
   if (!workspace || ws_bytes < need || ws_bytes < pl.total)
     return fail(REHYAT_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, ws_bytes);
   if (!aligned16(workspace)) return fail(REHYAT_ERR_ALIGN, "workspace not 16-byte aligned");
@@ -597,7 +622,7 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int L, int frames_befor
     rehyat::attn::Params ap{};
     ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
     ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
-    ap.H = d.H; ap.P = d.P; ap.n_states = 1; ap.nq_rows = pl.nq;
+    ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
     ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
     RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
@@ -605,7 +630,7 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int L, int frames_befor
     if (pl.fold_rows > 0) {
       RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
       rehyat::state::FoldParams fp{};
-      fp.L = L; fp.H = d.H; fp.P = d.P; fp.single_rows = pl.fold_rows; fp.n_fold = 1;
+      fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.single_rows = pl.fold_rows; fp.n_fold = 1;
       fp.splits = pl.splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
       RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(pl.splits, 1, BH), st));
       rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
@@ -660,7 +685,7 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   if (!aligned16(q) || !aligned16(k_win) || !aligned16(v_win) || !aligned16(out))
     return fail(REHYAT_ERR_ALIGN, "q/k_win/v_win/out not 16-byte aligned");
   // Same plan as rehyat_chunk_forward, with the fold split count lowered until the scratch fits.
-  ChunkPlan pl = plan_chunk(d, dt, L, frames_before, chunk_frames, To);
+  ChunkPlan pl = plan_chunk(d, dt, L, frames_before, chunk_frames, To, To);
   const size_t BH = (size_t)d.B * d.H;
   const size_t st_bytes = round_up(BH * d.D * d.F * 2, 256);
   const size_t wbd_bytes = round_up((size_t)d.H * 2 * d.F * d.D * 2, 256);
@@ -697,7 +722,7 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   rehyat::attn::Params ap{};
   ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
   ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
-  ap.H = d.H; ap.P = d.P; ap.n_states = 1; ap.nq_rows = pl.nq;
+  ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
   RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3((pl.nq + 255) / 256, 1, nbh),
@@ -705,7 +730,7 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   if (pl.fold_rows > 0) {
     RH_TRY(prepare_blockdiag(d, Wk, Wkbd, &mwk, st));
     rehyat::state::FoldParams fp{};
-    fp.L = L; fp.H = d.H; fp.P = d.P; fp.single_rows = pl.fold_rows; fp.n_fold = 1;
+    fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.single_rows = pl.fold_rows; fp.n_fold = 1;
     fp.splits = splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
     RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(splits, 1, nbh), st));
     rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, nbh), 256, 0, st>>>(

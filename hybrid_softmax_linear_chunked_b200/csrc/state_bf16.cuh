@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   for (int i = tid; i < kFD; i += kThreads) {
     sB[i] = p.bk ? p.bk[(size_t)h * kFD + i] : 0.f;
-    sPw[i] = static_cast<uint8_t>(part_power(i, kFD, p.P));
+    sPw[i] = static_cast<uint8_t>(feature_power(i, kFD, p.P));
   }
   {
     uint32_t* ones = reinterpret_cast<uint32_t*>(sm + kOffOnes);

@@ -63,10 +63,20 @@ typedef enum {
 
 typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
 
+/* Which feature map phi follows the grouped linear u = x W_g^T + b:
+ *   REHYAT_PHI_POLY: split u into P contiguous parts, part p (1-based) -> softplus(u_p)^p
+ *                    (the polynomial map of the "ReHyAt overview" page §2.2.2);
+ *   REHYAT_PHI_ELU1: elu(u) + 1 (the linear-attention map of the same page §2.1.2; with
+ *                    G = D groups of 1 x 1 weights all 1 and no bias it is elu(x) + 1 of the
+ *                    raw token, as printed there).  P is then ignored. */
+typedef enum { REHYAT_PHI_POLY = 0, REHYAT_PHI_ELU1 = 1 } rehyat_phi;
+
 /* Problem dimensions shared by all calls: batch B, heads H, head dim D, feature count F of phi,
- * group count G of its grouped linear (D % G == 0, F % G == 0), polynomial parts P (1..F). */
+ * group count G of its grouped linear (D % G == 0, F % G == 0), polynomial parts P (1..F), and
+ * the feature map kind `phi` (a rehyat_phi; 0, the polynomial map, when zero-initialised). */
 typedef struct {
   int B, H, D, F, G, P;
+  int phi;
 } rehyat_dims;
 
 /* Message for the last non-OK status returned on this host thread ("" if none). */
@@ -135,6 +145,23 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int frame_tokens, int f
                          const void* v_win, const float* Wq, const float* bq, const float* Wk,
                          const float* bk, float* S, float* Z, void* out, void* workspace,
                          size_t ws_bytes, void* stream);
+
+/* rehyat_chunk_forward for a variable chunk schedule ("ReHyAt overview" page §5.2: a longer
+ * chunk for key frames such as the first, more overlap where motion is strong): chunk_frames
+ * and To may change from call to call, and To_next is the overlap the NEXT call will use.
+ * After the output, the window frames that the next window no longer holds, [w_c, w_{c+1}) with
+ * w_c = frames_before - min(To, frames_before) and w_{c+1} = max(0, frames_before +
+ * chunk_frames - To_next), are folded into S and Z.  REHYAT_ERR_ARG if To_next < 0 or if the
+ * next window would reach frames this call's window does not hold (min(To_next,
+ * frames_before + chunk_frames) > min(To, frames_before) + chunk_frames: they were folded
+ * before).  The workspace must have the size rehyat_chunk_workspace_size gives for the largest
+ * chunk_frames and To of the schedule.  rehyat_chunk_forward is this call with To_next = To. */
+int rehyat_chunk_forward_sched(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
+                               int frames_before, int chunk_frames, int To, int To_next,
+                               const void* q, const void* k_win, const void* v_win,
+                               const float* Wq, const float* bq, const float* Wk,
+                               const float* bk, float* S, float* Z, void* out, void* workspace,
+                               size_t ws_bytes, void* stream);
 
 /* rehyat_chunk_forward for callers that cannot allocate device memory: no workspace argument.
  * The pages have no counterpart of this call; it exists for callers such as a plugin inside a

@@ -32,14 +32,14 @@ def test_header_declares_the_binding_surface():
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.rehyat_version() == 100
+    assert lib.rehyat_version() == 101
 
 
 FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced: checks come first
 
 
-def dims(B=1, H=2, D=128, F=128, G=8, P=2):
-    return rb.Dims(B, H, D, F, G, P)
+def dims(B=1, H=2, D=128, F=128, G=8, P=2, phi=0):
+    return rb.Dims(B, H, D, F, G, P, phi)
 
 
 def call_forward(lib, d, dt=rb.REHYAT_BF16, T=7, L=64, Tc=3, To=1, ws_bytes=1 << 40, **ptrs):
@@ -53,6 +53,8 @@ def call_forward(lib, d, dt=rb.REHYAT_BF16, T=7, L=64, Tc=3, To=1, ws_bytes=1 <<
     (dict(d=dims(B=0)), -1),
     (dict(d=dims(G=3)), -1),
     (dict(d=dims(P=200)), -1),
+    (dict(d=dims(phi=2)), -1),
+    (dict(d=dims(phi=-1)), -1),
     (dict(d=dims(D=64, F=64)), -2),
     (dict(d=dims(F=64)), -2),
     (dict(d=dims(), dt=7), -3),
@@ -99,3 +101,24 @@ def test_selftest_rejects_limits_out_of_range(lib):
     for bad in (0, 999, 2_000_000_001):
         assert lib.rehyat_selftest_wait_timeout(bad, None) == -1
         assert "limit_ns" in lib.rehyat_last_error().decode()
+
+
+def test_abi_version_and_dims_layout(lib):
+    assert lib.rehyat_version() == 101
+    assert ctypes.sizeof(rb.Dims) == 7 * 4
+    # the elu + 1 kind passes validation (workspace queries need no device)
+    n = ctypes.c_size_t(0)
+    assert lib.rehyat_forward_workspace_size(dims(phi=rb.PHI_ELU1), rb.REHYAT_BF16, 7, 64, 3, 1,
+                                             ctypes.byref(n)) == 0 and n.value > 0
+
+
+def test_chunk_forward_sched_rejects_overlap_into_folded_frames(lib):
+    d = dims()
+    # window of frames [2, 4) (To = 1 after 3 frames, 1-frame chunk): a next overlap of 3 would
+    # need frame 1, already folded into S
+    st = lib.rehyat_chunk_forward_sched(d, rb.REHYAT_BF16, 64, 3, 1, 1, 3, FAKE, FAKE, FAKE, FAKE,
+                                        None, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert st == -1 and "folded" in lib.rehyat_last_error().decode()
+    st = lib.rehyat_chunk_forward_sched(d, rb.REHYAT_BF16, 64, 3, 1, 1, -1, FAKE, FAKE, FAKE, FAKE,
+                                        None, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert st == -1

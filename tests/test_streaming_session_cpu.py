@@ -19,11 +19,13 @@ def oracle_step(monkeypatch):
     rb.load()
     calls = []
 
-    def fake(q, kw, vw, Wq, bq, Wk, bk, S, Z, *, P, frame_tokens, frames_before, To, out=None,
-             workspace=None):
+    def fake(q, kw, vw, Wq, bq, Wk, bk, S, Z, *, P, frame_tokens, frames_before, To, phi=0,
+             To_next=None, out=None, workspace=None):
+        kind = O.PHI_ELU1 if phi == rb.PHI_ELU1 else O.PHI_POLY
         B, H, n, D = q.shape
         cf = n // frame_tokens
         calls.append((frames_before, cf, kw.shape[2] // frame_tokens))
+        nxt = To if To_next is None else To_next
         out = torch.empty_like(q) if out is None else out
         for b in range(B):
             for h in range(H):
@@ -32,7 +34,7 @@ def oracle_step(monkeypatch):
                                             bq[h].double().numpy(), Wk[h].double().numpy(),
                                             bk[h].double().numpy(), P, S[b, h].double().numpy(),
                                             Z[b, h].double().numpy(), frame_tokens, frames_before,
-                                            cf, To)
+                                            cf, To, kind, To_next=nxt)
                 out[b, h] = torch.from_numpy(o)
                 S[b, h] = torch.from_numpy(Sn)
                 Z[b, h] = torch.from_numpy(Zn)
@@ -85,3 +87,29 @@ def test_resume_from_host_state(oracle_step):
     again.load_state_dict(ck)
     part2 = feed(again, inp, W.chunk_bounds()[2:])
     assert all(torch.equal(a, b) for a, b in zip(whole, part1 + part2))
+
+
+def test_variable_schedule(oracle_step):
+    """Longer first chunk and per-chunk overlaps (session capacity Tc = 4, To = 2)."""
+    w = C.Workload("session-sched", B=1, H=1, D=32, T=11, frame_h=2, frame_w=2, Tc=4, To=2, P=2,
+                   F=32, G=4, dtype="f32", seed=6)
+    inp = make_inputs(w)
+    cfs, ovs = [4, 2, 3, 1, 1], [0, 1, 2, 2, 0]
+    s = streaming.ChunkStream(inp.Wq, inp.bq, inp.Wk, inp.bk, B=1, P=2, frame_tokens=4, Tc=4,
+                              To=2, dtype=torch.float32, device=torch.device("cpu"))
+    bounds = O.schedule_bounds(cfs, ovs)
+    outs = []
+    for c, (_, a, e) in enumerate(bounds):
+        sl = slice(a * 4, e * 4)
+        nxt = ovs[c + 1] if c + 1 < len(ovs) else ovs[c]
+        outs.append(s.step(inp.q[:, :, sl].contiguous(), inp.k[:, :, sl].contiguous(),
+                           inp.v[:, :, sl].contiguous(), To=ovs[c], To_next=nxt).clone())
+    got = torch.cat(outs, dim=2)[0, 0].double().numpy()
+    q, k, v = (x[0, 0].double().numpy() for x in (inp.q, inp.k, inp.v))
+    pq = O.feature_map(q, inp.Wq[0].double().numpy(), inp.bq[0].double().numpy(), 2)
+    pk = O.feature_map(k, inp.Wk[0].double().numpy(), inp.bk[0].double().numpy(), 2)
+    want = O.hybrid_attention_masked(q, k, v, pq, pk, 4, O.schedule_mask(bounds))
+    assert np.linalg.norm(got - want) / np.linalg.norm(want) <= 1e-6
+    with pytest.raises(ValueError):
+        s.step(inp.q[:, :, :4].contiguous(), inp.k[:, :, :4].contiguous(),
+               inp.v[:, :, :4].contiguous(), To=3)

@@ -119,3 +119,36 @@ def test_session_rejects_bad_chunks_and_states(dev, data):
     st["shape"] = (9,) + tuple(st["shape"][1:])
     with pytest.raises(ValueError):
         new_session(t).load_state_dict(st)
+
+
+def test_variable_schedule(dev):
+    """A longer first chunk and per-chunk overlaps (ReHyAt overview §5.2), bf16, against the
+    quadratic form under the schedule's frame mask."""
+    w = C.Workload("sched", B=1, H=2, D=128, T=13, frame_h=6, frame_w=11, Tc=5, To=2, P=2,
+                   F=128, G=8, dtype="bf16", seed=35)
+    inp = make_inputs(w)
+    t = [x.to(dev) for x in (inp.q, inp.k, inp.v, inp.Wq, inp.bq, inp.Wk, inp.bk)]
+    q, k, v = t[:3]
+    cfs, ovs = [5, 3, 3, 2], [0, 1, 2, 1]
+    bounds = O.schedule_bounds(cfs, ovs)
+    sess = new_session(t, w)
+    L = w.frame_tokens
+    outs = []
+    for c, (_, s, e) in enumerate(bounds):
+        sl = slice(s * L, e * L)
+        nxt = ovs[c + 1] if c + 1 < len(ovs) else ovs[c]
+        outs.append(sess.step(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(),
+                              v[:, :, sl].contiguous(), To=ovs[c], To_next=nxt).clone())
+    rb.sync_status(dev)
+    out = torch.cat(outs, dim=2)
+    M = O.schedule_mask(bounds)
+    for h in range(2):
+        qh, kh, vh = f64(inp.q[0, h]), f64(inp.k[0, h]), f64(inp.v[0, h])
+        want = O.hybrid_attention_masked(qh, kh, vh,
+                                         O.feature_map(qh, f64(inp.Wq[h]), f64(inp.bq[h]), w.P),
+                                         O.feature_map(kh, f64(inp.Wk[h]), f64(inp.bk[h]), w.P),
+                                         L, M)
+        got = f64(out[0, h])
+        assert np.isfinite(got).all()
+        assert np.abs(got - want).max() <= 2e-2
+        assert np.linalg.norm(got - want) / np.linalg.norm(want) <= 5e-3
