@@ -3,9 +3,16 @@
 
 One step = one whole-sequence forward of the 480x832 5 s workload (B=1, 12 heads, D=128,
 21 frames x 1560 tokens, Tc=3, To=1, P=2, F=128, G=8, bf16): the state folds with phi_k, their
-prefix scan, and the fused softmax + linear attention with phi_q, through the C ABI.
+prefix scan, phi_q, and the fused softmax + linear attention, through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload 480p5s|480p10s|720p5s|480p20s-stream] [--phi poly|elu1]
+                    [--schedule FRAMES/OVERLAP,...]
+
+The other workloads and options measure the remaining configurations: the streaming workload's
+step is the whole chunk-by-chunk pass (27 calls per sequence, both sequences of the batch at
+once) through the streaming session; --schedule gives it a variable chunk schedule (the first
+entry once, the others cyclically, e.g. 5/0,3/1,3/2); --phi elu1 swaps the feature map.
 
 N > 1 runs under torchrun: every rank runs its own replica of the workload (weak scaling, no
 collective on the data path; NCCL only for the timing barrier and the max over ranks).
@@ -15,6 +22,7 @@ workload instead (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -33,10 +41,12 @@ from hybrid_softmax_linear_chunked_b200 import binding as rb  # noqa: E402
 from hybrid_softmax_linear_chunked_b200 import configs as C  # noqa: E402
 from hybrid_softmax_linear_chunked_b200.inputs import make_inputs  # noqa: E402
 from hybrid_softmax_linear_chunked_b200.replicas import Replicas, job_throughput  # noqa: E402
+from hybrid_softmax_linear_chunked_b200.streaming import ChunkStream  # noqa: E402
 
 METRIC = "hybrid-attn query tokens/s (12 heads, D=128); % of dense BF16 tensor peak"
 UNIT = "tokens/s"
-WORKLOAD = C.WAN_480P_5S
+WORKLOADS = {"480p5s": C.WAN_480P_5S, "480p10s": C.WAN_480P_10S, "720p5s": C.WAN_720P_5S,
+             "480p20s-stream": C.WAN_480P_20S_STREAM}
 L2_BYTES = 126 * 1024 * 1024
 ATTN_SOURCES = ["hybrid_softmax_linear_chunked_b200/csrc/attn_bf16.cuh",
                 "hybrid_softmax_linear_chunked_b200/csrc/sm100.cuh",
@@ -52,7 +62,33 @@ def parse_args():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="480p5s")
+    ap.add_argument("--phi", choices=["poly", "elu1"], default="poly")
+    ap.add_argument("--schedule", default=None,
+                    help="streaming only: FRAMES/OVERLAP entries, first once, rest cyclic")
     return ap.parse_args()
+
+
+def pick_workload(args) -> C.Workload:
+    w = WORKLOADS[args.workload]
+    if args.phi != "poly":
+        w = dataclasses.replace(w, phi=args.phi, P=1, name=w.name + ", elu+1 feature map")
+    return w
+
+
+def parse_schedule(spec: str | None, w: C.Workload):
+    """(chunk_frames, overlap) per chunk covering w.T frames; None -> the uniform Tc / To."""
+    if not spec:
+        return [(e - s, w.To) for (_, s, e) in w.chunk_bounds()]
+    items = [tuple(int(x) for x in it.split("/")) for it in spec.split(",")]
+    out, t, i = [], 0, 0
+    while t < w.T:
+        cf, ov = items[i] if i == 0 or len(items) == 1 else items[1 + (i - 1) % (len(items) - 1)]
+        cf = min(cf, w.T - t)
+        out.append((cf, ov))
+        t += cf
+        i += 1
+    return out
 
 
 def read_peaks():
@@ -195,7 +231,7 @@ def run_reference(args, rank: int):
     if rank != 0:
         return
     import oracle.rehyat_oracle as O
-    w = WORKLOAD
+    w = pick_workload(args)
     inp = make_inputs(w)
     rng = np.random.default_rng(0)
     cache = {}
@@ -207,7 +243,8 @@ def run_reference(args, rank: int):
                                          inp.bq[h], inp.Wk[h], inp.bk[h])]
         q, k, v, Wq, bq, Wk, bk = cache[h]
         rows = rng.integers(0, w.N, size=n_rows)
-        O.hybrid_attention_rows(q, k, v, Wq, bq, Wk, bk, w.P, w.frame_tokens, w.Tc, w.To, rows)
+        O.hybrid_attention_rows(q, k, v, Wq, bq, Wk, bk, w.P, w.frame_tokens, w.Tc, w.To, rows,
+                                O.PHI_ELU1 if w.phi == "elu1" else O.PHI_POLY)
 
     # size a step so that warm-up + timed steps take about two minutes in all
     t = time.perf_counter()
@@ -261,12 +298,112 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     rb.load()
-    w = WORKLOAD
+    w = pick_workload(args)
     inp = make_inputs(w, seed=rep.seed(w.seed))
+    run = (stream_runner if w.mode == "stream" else full_runner)(w, inp, dev, args)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(max(3, args.warmup)):
+        run.step()
+    rb.sync_status(dev)
+
+    K = args.steps
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(device_index_for_smi(dev))
+    with sampler:
+        rep.barrier()
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for i in range(K):
+            run.step(mids[i], ends[i])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        rep.barrier()
+    rb.sync_status(dev)
+    elapsed_ms = start.elapsed_time(stop)
+    # the attention launch of step i runs between its mid and end events; the phases before it
+    # between the end of step i-1 (or start) and the mid of step i
+    attn_ms = statistics.mean(mids[i].elapsed_time(ends[i]) for i in range(K))
+    pre_ms = statistics.mean((ends[i - 1].elapsed_time(mids[i]) if i else
+                              start.elapsed_time(mids[0])) for i in range(K))
+    elapsed_ms = rep.max(elapsed_ms, dev)
+
+    # ---- end to end through the public API: pinned host inputs in, result out ----
+    for _ in range(3):
+        run.e2e_step()
+    E = args.e2e_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    rep.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(E):
+        run.e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    rep.barrier()
+    rb.sync_status(dev)
+    e2e_ms = rep.max(e0.elapsed_time(e1), dev)
+
+    if rank == 0:
+        peaks = read_peaks()
+        ms_per_step = elapsed_ms / K
+        kernel_time = attn_ms if run.attn_isolated else ms_per_step
+        achieved = run.attn_flops / (kernel_time * 1e-3) / 1e12
+        cfg = workload_config(w, world)
+        cfg.update(run.config)
+        line = {
+            "metric": METRIC,
+            "value": job_throughput(w.B * w.N, world, ms_per_step),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": cfg,
+            "tflops": run.step_flops * world / (ms_per_step * 1e-3) / 1e12,
+            "frac_of_bf16_peak_step": run.step_flops / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "kernel_ms": ({"attention": attn_ms, "states_and_phiq": pre_ms} if run.attn_isolated
+                          else {"step": ms_per_step}),
+            "roofline": {"kernel": run.roofline_kernel, "bound": "tensor",
+                         "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"],
+                         "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                         "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                               if peaks.get("bf16_tflops_sustained") else None),
+                         "traffic": read_traffic() if run.attn_isolated and args.workload == "480p5s"
+                                    and w.phi == "poly" else None},
+            "e2e": {"value": job_throughput(w.B * w.N, world, e2e_ms / E), "unit": UNIT,
+                    "h2d_bytes_per_step": run.h2d, "d2h_bytes_per_step": run.d2h},
+            "gpu_launches": run.launches_per_step * K,
+            "clocks": sampler.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(inp, w)
+        print(json.dumps(line), flush=True)
+    rep.close()
+
+
+class _Run:
+    """What one timed step does, for one workload mode."""
+    attn_isolated = True
+    roofline_kernel = "hybrid_attn_bf16_kernel"
+    config: dict = {}
+
+
+def full_runner(w: C.Workload, inp, dev, args) -> _Run:
+    """One whole-sequence forward: states, phi_q, then the attention (events around it)."""
+    r = _Run()
     q, k, v = (x.to(dev) for x in (inp.q, inp.k, inp.v))
     Wq, bq, Wk, bk = (x.to(dev) for x in (inp.Wq, inp.bq, inp.Wk, inp.bk))
-    kw = dict(P=w.P, frame_tokens=w.frame_tokens, Tc=w.Tc, To=w.To)
-    d = rb.dims_of(q, Wq, w.P)
+    kw = dict(P=w.P, phi=w.phi_code, frame_tokens=w.frame_tokens, Tc=w.Tc, To=w.To)
+    d = rb.dims_of(q, Wq, w.P, w.phi_code)
     ws = torch.empty(rb.forward_workspace_size(d, rb.REHYAT_BF16, w.T, w.frame_tokens, w.Tc,
                                                w.To), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
@@ -282,97 +419,93 @@ def main():
         if ev_end is not None:
             ev_end.record(stream)
 
-    for _ in range(max(3, args.warmup)):
-        step()
-    rb.sync_status(dev)
-
-    K = args.steps
-    mids = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(device_index_for_smi(dev))
-    with sampler:
-        rep.barrier()
-        torch.cuda.synchronize(dev)
-        start.record(stream)
-        for i in range(K):
-            step(mids[i], ends[i])
-        stop.record(stream)
-        torch.cuda.synchronize(dev)
-        rep.barrier()
-    rb.sync_status(dev)
-    elapsed_ms = start.elapsed_time(stop)
-    attn_ms = statistics.mean(mids[i].elapsed_time(ends[i]) for i in range(K))
-    # states + phi_q phases of step i run between the end of step i-1 (or start) and mid of step i
-    state_ms = statistics.mean((ends[i - 1].elapsed_time(mids[i]) if i else
-                                start.elapsed_time(mids[0])) for i in range(K))
-    elapsed_ms = rep.max(elapsed_ms, dev)
-
-    # ---- end to end through the public API: pinned host inputs in, result out ----
     host = [x.pin_memory() for x in (inp.q, inp.k, inp.v, inp.Wq, inp.bq, inp.Wk, inp.bk)]
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in host)
-    d2h = out_h.numel() * out_h.element_size()
 
     def e2e_step():
         qd, kd, vd, Wqd, bqd, Wkd, bkd = (x.to(dev, non_blocking=True) for x in host)
         o = rb.forward(qd, kd, vd, Wqd, bqd, Wkd, bkd, workspace=ws, **kw)
         out_h.copy_(o, non_blocking=True)
 
-    for _ in range(3):
-        e2e_step()
-    E = args.e2e_steps
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    rep.barrier()
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(E):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    rep.barrier()
-    rb.sync_status(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = rep.max(e2e_ms, dev)
+    r.step, r.e2e_step = step, e2e_step
+    r.h2d = sum(x.numel() * x.element_size() for x in host)
+    r.d2h = out_h.numel() * out_h.element_size()
+    r.attn_flops = w.attn_tensor_flops()
+    r.step_flops = w.flops(streaming=False)
+    r.launches_per_step = 6  # 2 weight preps, fold, scan, phi_q, attention
+    return r
 
-    if rank == 0:
-        peaks = read_peaks()
-        ms_per_step = elapsed_ms / K
-        flops_attn = w.attn_tensor_flops()
-        achieved = flops_attn / (attn_ms * 1e-3) / 1e12
-        line = {
-            "metric": METRIC,
-            "value": job_throughput(w.B * w.N, world, ms_per_step),
-            "unit": UNIT,
-            "n_gpus": world,
-            "steps": K,
-            "warmup": args.warmup,
-            "ms_per_step": ms_per_step,
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "bf16",
-            "data": "synthetic",
-            "config": workload_config(w, world),
-            "tflops": w.flops() * world / (ms_per_step * 1e-3) / 1e12,
-            "frac_of_bf16_peak_step": w.flops() / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
-            "kernel_ms": {"attention": attn_ms, "states_and_phiq": state_ms},
-            "roofline": {"kernel": "hybrid_attn_bf16_kernel", "bound": "tensor",
-                         "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / peaks["bf16_tflops"],
-                         "peak_source": f"{peaks['source']} bf16 dense (burst)",
-                         "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
-                                               if peaks.get("bf16_tflops_sustained") else None),
-                         "traffic": read_traffic()},
-            "e2e": {"value": job_throughput(w.B * w.N, world, e2e_ms / E), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 6 * K,  # per step: 2 weight preps, fold, scan, phi_q, attention
-            "clocks": sampler.summary(),
-        }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(inp, w)
-        print(json.dumps(line), flush=True)
-    rep.close()
+
+def sched_bounds(sched):
+    """(w, s, e, overlap, next overlap) per chunk of a (frames, overlap) schedule."""
+    out, s = [], 0
+    for c, (cf, ov) in enumerate(sched):
+        nxt = sched[c + 1][1] if c + 1 < len(sched) else ov
+        out.append((max(0, s - ov), s, s + cf, ov, nxt))
+        s += cf
+    return out
+
+
+def stream_runner(w: C.Workload, inp, dev, args) -> _Run:
+    """The whole sequence fed chunk by chunk through the streaming session (every sequence of
+    the batch at once); the inputs sit in HBM already split into chunks."""
+    r = _Run()
+    r.attn_isolated = False
+    sched = parse_schedule(args.schedule, w)
+    bounds = sched_bounds(sched)
+    L = w.frame_tokens
+    Wq, bq, Wk, bk = (x.to(dev) for x in (inp.Wq, inp.bq, inp.Wk, inp.bk))
+    chunks = [[x[:, :, s * L:e * L].contiguous().to(dev) for x in (inp.q, inp.k, inp.v)]
+              for (_, s, e, _, _) in bounds]
+    outs = [torch.empty_like(c[0]) for c in chunks]
+    sess = ChunkStream(Wq, bq, Wk, bk, B=w.B, P=w.P, phi=w.phi_code, frame_tokens=L,
+                       Tc=max(cf for cf, _ in sched), To=max(ov for _, ov in sched))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev_mid=None, ev_end=None):
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        sess.reset()
+        for c, (_, _, _, ov, nxt) in enumerate(bounds):
+            sess.step(*chunks[c], out=outs[c], To=ov, To_next=nxt)
+        if ev_end is not None:
+            ev_end.record(stream)
+
+    host = [[x[:, :, s * L:e * L].contiguous().pin_memory() for x in (inp.q, inp.k, inp.v)]
+            for (_, s, e, _, _) in bounds]
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+
+    def e2e_step():
+        sess.reset()
+        for c, (_, _, _, ov, nxt) in enumerate(bounds):
+            qd, kd, vd = (x.to(dev, non_blocking=True) for x in host[c])
+            o = sess.step(qd, kd, vd, To=ov, To_next=nxt)
+            host_out[c].copy_(o, non_blocking=True)
+
+    # algorithmic work of the schedule: softmax over each window, readout of chunks with a linear
+    # region, every fold (the streaming calls fold after every chunk), and the feature maps
+    D, F = w.D, w.F
+    attn = step_f = 0.0
+    launches = 0
+    for (wf, s, e, ov, nxt) in bounds:
+        nq, nw = (e - s) * L, (e - wf) * L
+        attn += 4.0 * nq * nw * D + (2.0 * nq * F * D if wf > 0 else 0.0)
+        fold = max(0, max(0, e - nxt) - wf) * L
+        step_f += (2.0 * nq * F + (2.0 * nq * D * F / w.G) if wf > 0 else 0.0)
+        step_f += fold * (2.0 * F * D + F + 2.0 * D * F / w.G)
+        launches += 5 + (1 if wf > 0 else 0) + (3 if fold > 0 else 0)
+    r.attn_flops = attn * w.B * w.H
+    r.step_flops = (attn + step_f) * w.B * w.H
+    r.step, r.e2e_step = step, e2e_step
+    r.h2d = sum(x.numel() * x.element_size() for c in host for x in c)
+    r.d2h = sum(o.numel() * o.element_size() for o in host_out)
+    # per call: K and V window gathers, S transpose, W_q block-diagonal, [phi_q], attention,
+    # [W_k block-diagonal, fold, state add]
+    r.launches_per_step = launches
+    r.roofline_kernel = "whole streaming step (attention FLOPs / step time)"
+    r.config = {"mode": "stream", "calls_per_step": len(bounds),
+                "schedule": [[cf, ov] for cf, ov in sched]}
+    return r
 
 
 if __name__ == "__main__":

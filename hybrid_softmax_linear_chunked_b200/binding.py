@@ -24,7 +24,8 @@ STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_SHAPE", -3: "ERR_DTYPE", -4: "ERR_WOR
 EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_forward_workspace_size", "rehyat_forward", "rehyat_forward_states",
             "rehyat_forward_phiq", "rehyat_forward_attend", "rehyat_chunk_workspace_size",
-            "rehyat_chunk_forward", "rehyat_chunk_forward_sched", "rehyat_chunk_forward_static", "rehyat_chunk_states",
+            "rehyat_chunk_forward", "rehyat_chunk_forward_sched", "rehyat_chunk_carry_workspace_size",
+            "rehyat_chunk_forward_carry", "rehyat_chunk_forward_static", "rehyat_chunk_states",
             "rehyat_selftest_wait_timeout", "rehyat_sync_status"]
 
 
@@ -77,6 +78,10 @@ def load() -> ctypes.CDLL:
                                        P, P, P, P, P, c_size_t, P]
     L.rehyat_chunk_forward_sched.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, c_int, P, P,
                                              P, P, P, P, P, P, P, P, P, c_size_t, P]
+    L.rehyat_chunk_carry_workspace_size.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int,
+                                                    ctypes.POINTER(c_size_t)]
+    L.rehyat_chunk_forward_carry.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                             P, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P]
     L.rehyat_chunk_forward_static.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P,
                                               P, P, P, P, P, P, P]
     L.rehyat_chunk_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
@@ -272,6 +277,39 @@ def chunk_forward(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, phi: int = 0
     else:
         _check(lib.rehyat_chunk_forward_sched(d, code, frame_tokens, frames_before, chunk_frames,
                                               To, To_next, *args))
+    return out
+
+
+def chunk_carry_workspace_size(d: Dims, dtype_code: int, L_: int, chunk_frames: int, To: int,
+                               carry_frames: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().rehyat_chunk_carry_workspace_size(d, dtype_code, L_, chunk_frames, To,
+                                                    carry_frames, ctypes.byref(n)))
+    return n.value
+
+
+def chunk_forward_carry(q, k, v, Wq, bq, Wk, bk, S, Z, k_carry, v_carry, *, P: int, phi: int = 0,
+                        frame_tokens: int, frames_before: int, To: int,
+                        To_next: int | None = None, out: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None):
+    """Streaming step on the chunk alone; S, Z and the carried frames k_carry, v_carry
+    [B,H,carry_frames*L,D] are updated in place."""
+    lib = load()
+    dev = _dev(q, k, v, Wq, bq, Wk, bk, S, Z, k_carry, v_carry)
+    d = dims_of(q, Wq, P, phi)
+    chunk_frames = q.shape[2] // frame_tokens
+    carry_frames = k_carry.shape[2] // frame_tokens
+    code = _dtype_code(q)
+    ws = _workspace(chunk_carry_workspace_size(d, code, frame_tokens, chunk_frames, To,
+                                               carry_frames), dev, workspace)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.rehyat_chunk_forward_carry(d, code, frame_tokens, frames_before, chunk_frames, To,
+                                          To if To_next is None else To_next, carry_frames,
+                                          _ptr(q), _ptr(k), _ptr(v), _ptr(Wq), _ptr(bq),
+                                          _ptr(Wk), _ptr(bk), _ptr(S), _ptr(Z), _ptr(k_carry),
+                                          _ptr(v_carry), _ptr(out), _ptr(ws), ws.numel(),
+                                          _stream(dev)))
     return out
 
 

@@ -19,6 +19,7 @@
 #include "phi_bf16.cuh"
 #include "sm100.cuh"
 #include "state_bf16.cuh"
+#include "stream_carry.cuh"
 
 namespace {
 
@@ -215,6 +216,27 @@ ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_be
     p.dS = cv.take(BH * d.F * d.D * 4);
     p.dZ = cv.take(BH * d.F * 4);
   }
+  p.total = cv.off;
+  return p;
+}
+
+// Streaming with carried frames: the chunk step's own workspace, then the assembled K and V
+// windows and the next carry of K and V.
+struct CarryPlan {
+  size_t step, kwin, vwin, kcar, vcar, total;
+};
+
+CarryPlan plan_carry(const rehyat_dims& d, rehyat_dtype dt, int L, int chunk_frames, int To,
+                     int cap) {
+  CarryPlan p{};
+  const size_t es = dt == REHYAT_BF16 ? 2 : 4;
+  const size_t BH = (size_t)d.B * d.H;
+  Carve cv;
+  p.step = cv.take(plan_chunk(d, dt, L, To, chunk_frames, To, To).total);
+  p.kwin = cv.take(BH * (size_t)(To + chunk_frames) * L * d.D * es);
+  p.vwin = cv.take(BH * (size_t)(To + chunk_frames) * L * d.D * es);
+  p.kcar = cv.take(BH * (size_t)cap * L * d.D * es);
+  p.vcar = cv.take(BH * (size_t)cap * L * d.D * es);
   p.total = cv.off;
   return p;
 }
@@ -665,6 +687,74 @@ int rehyat_chunk_forward_sched(rehyat_dims d, rehyat_dtype dt, int L, int frames
     rehyat::fp32::state_add_f32_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
         dS, dZ, d.F, d.D, S, Z);
     RH_TRY(cuda_check(cudaGetLastError(), "state add f32 launch"));
+  }
+  return REHYAT_OK;
+}
+
+int rehyat_chunk_carry_workspace_size(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
+                                      int chunk_frames, int To, int carry_frames,
+                                      size_t* bytes) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(chunk_frames, frame_tokens, 1, To));
+  if (carry_frames < To) return fail(REHYAT_ERR_ARG, "carry_frames %d < To %d", carry_frames, To);
+  if (!bytes) return fail(REHYAT_ERR_ARG, "null bytes pointer");
+  *bytes = plan_carry(d, dt, frame_tokens, chunk_frames, To, carry_frames).total;
+  return REHYAT_OK;
+}
+
+int rehyat_chunk_forward_carry(rehyat_dims d, rehyat_dtype dt, int L, int frames_before,
+                               int chunk_frames, int To, int To_next, int carry_frames,
+                               const void* q, const void* k, const void* v, const float* Wq,
+                               const float* bq, const float* Wk, const float* bk, float* S,
+                               float* Z, void* k_carry, void* v_carry, void* out,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(chunk_frames, L, 1, To));
+  if (frames_before < 0) return fail(REHYAT_ERR_ARG, "frames_before must be >= 0");
+  if (carry_frames < To) return fail(REHYAT_ERR_ARG, "carry_frames %d < To %d", carry_frames, To);
+  if (!k || !v || (carry_frames > 0 && (!k_carry || !v_carry)))
+    return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_carry) || !aligned16(v_carry))
+    return fail(REHYAT_ERR_ALIGN, "k/v/k_carry/v_carry not 16-byte aligned");
+  // the window and the step's workspace are sized for this call's To; the caller's workspace
+  // comes from rehyat_chunk_carry_workspace_size with the largest chunk_frames and To
+  const CarryPlan pl = plan_carry(d, dt, L, chunk_frames, To, carry_frames);
+  if (!workspace || ws_bytes < pl.total)
+    return fail(REHYAT_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", pl.total, ws_bytes);
+  if (!aligned16(workspace)) return fail(REHYAT_ERR_ALIGN, "workspace not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int BH = d.B * d.H;
+  const int ov = To < frames_before ? To : frames_before;
+  const size_t es = dt == REHYAT_BF16 ? 2 : 4;
+  rehyat::carry::Params cp{};
+  cp.L = L; cp.ov = ov; cp.cf = chunk_frames; cp.cap = carry_frames;
+  cp.row_vec = (int)(d.D * es / 16);
+  const long long vecs = ((long long)(ov + chunk_frames) + carry_frames) * L * cp.row_vec;
+  long long gx = (vecs + 255) / 256;
+  const long long max_gx = (8LL * 148 + BH - 1) / BH;
+  if (gx > max_gx) gx = max_gx;
+  for (int t = 0; t < 2; ++t) {
+    cp.carry = static_cast<const uint4*>(t ? v_carry : k_carry);
+    cp.chunk = static_cast<const uint4*>(t ? v : k);
+    cp.window = reinterpret_cast<uint4*>(ws + (t ? pl.vwin : pl.kwin));
+    cp.carry_new = reinterpret_cast<uint4*>(ws + (t ? pl.vcar : pl.kcar));
+    rehyat::carry::gather_kernel<<<dim3((unsigned)gx, BH), 256, 0, st>>>(cp);
+    RH_TRY(cuda_check(cudaGetLastError(), "window gather launch"));
+  }
+  RH_TRY(rehyat_chunk_forward_sched(d, dt, L, frames_before, chunk_frames, To, To_next, q,
+                                    ws + pl.kwin, ws + pl.vwin, Wq, bq, Wk, bk, S, Z, out,
+                                    ws + pl.step, pl.kwin - pl.step, stream));
+  const size_t car_bytes = (size_t)BH * carry_frames * L * d.D * es;
+  if (car_bytes) {
+    RH_TRY(cuda_check(cudaMemcpyAsync(k_carry, ws + pl.kcar, car_bytes, cudaMemcpyDeviceToDevice, st),
+                      "carry copy"));
+    RH_TRY(cuda_check(cudaMemcpyAsync(v_carry, ws + pl.vcar, car_bytes, cudaMemcpyDeviceToDevice, st),
+                      "carry copy"));
   }
   return REHYAT_OK;
 }

@@ -146,6 +146,26 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int frame_tokens, int f
                          const float* bk, float* S, float* Z, void* out, void* workspace,
                          size_t ws_bytes, void* stream);
 
+/* The streaming step with the overlap frames kept by the library's own copy kernel: the caller
+ * passes only the chunk (k, v [B,H,chunk_frames*L,D]) and a carry buffer per tensor
+ * (k_carry, v_carry [B,H,carry_frames*L,D], inout, same dtype): the last carry_frames frames of
+ * K and V seen so far, right-aligned (after f frames, only the last min(f, carry_frames) are
+ * meaningful).  The call builds the window [the last min(To, frames_before) carried frames |
+ * the chunk] in the workspace, runs rehyat_chunk_forward_sched on it (To_next as there), and
+ * updates the carry to the last carry_frames frames of (carry ++ chunk).  Needs To <=
+ * carry_frames; a zero-initialised carry is fine for the first call.  The state between calls
+ * is then S, Z and the carry: the method's recurrent state (page §2.3).  Workspace:
+ * rehyat_chunk_carry_workspace_size with the largest chunk_frames and To of the stream. */
+int rehyat_chunk_carry_workspace_size(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
+                                      int chunk_frames, int To, int carry_frames, size_t* bytes);
+int rehyat_chunk_forward_carry(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
+                               int frames_before, int chunk_frames, int To, int To_next,
+                               int carry_frames, const void* q, const void* k, const void* v,
+                               const float* Wq, const float* bq, const float* Wk,
+                               const float* bk, float* S, float* Z, void* k_carry,
+                               void* v_carry, void* out, void* workspace, size_t ws_bytes,
+                               void* stream);
+
 /* rehyat_chunk_forward for a variable chunk schedule ("ReHyAt overview" page §5.2: a longer
  * chunk for key frames such as the first, more overlap where motion is strong): chunk_frames
  * and To may change from call to call, and To_next is the overlap the NEXT call will use.

@@ -122,3 +122,20 @@ def test_chunk_forward_sched_rejects_overlap_into_folded_frames(lib):
     st = lib.rehyat_chunk_forward_sched(d, rb.REHYAT_BF16, 64, 3, 1, 1, -1, FAKE, FAKE, FAKE, FAKE,
                                         None, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
     assert st == -1
+
+
+def test_chunk_forward_carry_checks(lib):
+    d = dims()
+    n = ctypes.c_size_t(0)
+    assert lib.rehyat_chunk_carry_workspace_size(d, rb.REHYAT_BF16, 64, 3, 2, 1, ctypes.byref(n)) == -1
+    assert lib.rehyat_chunk_carry_workspace_size(d, rb.REHYAT_BF16, 64, 3, 1, 1, ctypes.byref(n)) == 0
+    # carry shorter than the overlap
+    st = lib.rehyat_chunk_forward_carry(d, rb.REHYAT_BF16, 64, 3, 3, 2, 2, 1, FAKE, FAKE, FAKE,
+                                        FAKE, None, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                        FAKE, 1 << 30, None)
+    assert st == -1 and "carry_frames" in lib.rehyat_last_error().decode()
+    # workspace too small
+    st = lib.rehyat_chunk_forward_carry(d, rb.REHYAT_BF16, 64, 3, 3, 1, 1, 1, FAKE, FAKE, FAKE,
+                                        FAKE, None, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                        FAKE, 16, None)
+    assert st == -4

@@ -1,6 +1,7 @@
-"""Host logic of the streaming session on CPU: the window / overlap bookkeeping, the frame
-counter and checkpoint / resume, with the C call replaced by the oracle's streaming step (the
-GPU path of the same session is covered by the gpu-marked tests)."""
+"""Host logic of the streaming session on CPU: the frame counter, the overlaps passed per step,
+and checkpoint / resume, with the C call replaced by a host restatement of its carry contract
+around the oracle's streaming step (the GPU path of the same session, where the library builds
+the window, is covered by the gpu-marked tests)."""
 import numpy as np
 import pytest
 import torch
@@ -19,12 +20,19 @@ def oracle_step(monkeypatch):
     rb.load()
     calls = []
 
-    def fake(q, kw, vw, Wq, bq, Wk, bk, S, Z, *, P, frame_tokens, frames_before, To, phi=0,
-             To_next=None, out=None, workspace=None):
+    def fake(q, k, v, Wq, bq, Wk, bk, S, Z, k_carry, v_carry, *, P, frame_tokens,
+             frames_before, To, phi=0, To_next=None, out=None, workspace=None):
+        """The carry contract of rehyat_chunk_forward_carry, restated on the host: window =
+        [last min(To, frames_before) carried frames | chunk]; carry <- last cap frames of
+        (carry ++ chunk), right-aligned; the step itself is the oracle's."""
         kind = O.PHI_ELU1 if phi == rb.PHI_ELU1 else O.PHI_POLY
+        L = frame_tokens
         B, H, n, D = q.shape
-        cf = n // frame_tokens
-        calls.append((frames_before, cf, kw.shape[2] // frame_tokens))
+        cf, cap = n // L, k_carry.shape[2] // L
+        ov = min(To, frames_before)
+        kw = torch.cat([k_carry[:, :, (cap - ov) * L:], k], dim=2)
+        vw = torch.cat([v_carry[:, :, (cap - ov) * L:], v], dim=2)
+        calls.append((frames_before, cf, kw.shape[2] // L))
         nxt = To if To_next is None else To_next
         out = torch.empty_like(q) if out is None else out
         for b in range(B):
@@ -33,14 +41,17 @@ def oracle_step(monkeypatch):
                                             vw[b, h].double().numpy(), Wq[h].double().numpy(),
                                             bq[h].double().numpy(), Wk[h].double().numpy(),
                                             bk[h].double().numpy(), P, S[b, h].double().numpy(),
-                                            Z[b, h].double().numpy(), frame_tokens, frames_before,
+                                            Z[b, h].double().numpy(), L, frames_before,
                                             cf, To, kind, To_next=nxt)
                 out[b, h] = torch.from_numpy(o)
                 S[b, h] = torch.from_numpy(Sn)
                 Z[b, h] = torch.from_numpy(Zn)
+        if cap:
+            k_carry.copy_(torch.cat([k_carry, k], dim=2)[:, :, -cap * L:])
+            v_carry.copy_(torch.cat([v_carry, v], dim=2)[:, :, -cap * L:])
         return out
 
-    monkeypatch.setattr(streaming.rb, "chunk_forward", fake)
+    monkeypatch.setattr(streaming.rb, "chunk_forward_carry", fake)
     return calls
 
 
