@@ -26,7 +26,7 @@ EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_forward_phiq", "rehyat_forward_attend", "rehyat_chunk_workspace_size",
             "rehyat_chunk_forward", "rehyat_chunk_forward_sched", "rehyat_chunk_carry_workspace_size",
             "rehyat_chunk_forward_carry", "rehyat_chunk_forward_static", "rehyat_chunk_states",
-            "rehyat_selftest_wait_timeout", "rehyat_sync_status"]
+            "rehyat_gemm_bf16", "rehyat_selftest_wait_timeout", "rehyat_sync_status"]
 
 
 class RehyatError(RuntimeError):
@@ -86,6 +86,9 @@ def load() -> ctypes.CDLL:
                                               P, P, P, P, P, P, P]
     L.rehyat_chunk_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
                                       P, c_size_t, P]
+    LL = ctypes.c_longlong
+    L.rehyat_gemm_bf16.argtypes = [c_int, c_int, c_int, c_int, P, LL, LL, c_int, P, LL, LL, c_int,
+                                   P, LL, LL, c_int, c_int, ctypes.c_float, P]
     L.rehyat_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
     L.rehyat_sync_status.argtypes = [P]
     for name in EXPORTED:
@@ -327,6 +330,26 @@ def chunk_forward_static(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, phi: 
                                            chunk_frames, To, _ptr(q), _ptr(k_win), _ptr(v_win),
                                            _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(S),
                                            _ptr(Z), _ptr(out), _stream(dev)))
+    return out
+
+
+def gemm(A: torch.Tensor, B: torch.Tensor, *, a_mn: bool = False, b_mn: bool = False,
+         out: torch.Tensor | None = None, accumulate: bool = False, alpha: float = 1.0,
+         out_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    """Batched bf16 GEMM on the tensor cores.  A [batch, M, K] (or [batch, K, M] with a_mn),
+    B [batch, N, K] (or [batch, K, N] with b_mn), both contiguous bf16; returns C [batch, M, N]
+    = alpha A B (added to `out` with accumulate)."""
+    dev = _dev(A, B)
+    batch = A.shape[0]
+    M, K = (A.shape[2], A.shape[1]) if a_mn else (A.shape[1], A.shape[2])
+    N = B.shape[2] if b_mn else B.shape[1]
+    if out is None:
+        out = torch.empty(batch, M, N, dtype=out_dtype, device=dev)
+    _check(load().rehyat_gemm_bf16(M, N, K, batch, _ptr(A), A.shape[2], A.shape[1] * A.shape[2],
+                                   int(a_mn), _ptr(B), B.shape[2], B.shape[1] * B.shape[2],
+                                   int(b_mn), _ptr(out), out.shape[2], out.shape[1] * out.shape[2],
+                                   int(out.dtype == torch.bfloat16), int(accumulate),
+                                   ctypes.c_float(alpha), _stream(dev)))
     return out
 
 

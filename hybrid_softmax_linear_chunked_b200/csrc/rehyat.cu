@@ -16,6 +16,7 @@
 #include "attn_bf16.cuh"
 #include "featmap.cuh"
 #include "fp32_path.cuh"
+#include "gemm_bf16.cuh"
 #include "phi_bf16.cuh"
 #include "sm100.cuh"
 #include "state_bf16.cuh"
@@ -119,6 +120,59 @@ int make_map(CUtensorMap* m, const void* base, int cols, long long rows, long lo
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(REHYAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return REHYAT_OK;
+}
+
+// bf16 [outer][rows][cols] tensor with explicit strides (elements), box {box_cols, box_rows, 1}.
+int make_map_strided(CUtensorMap* m, const void* base, long long cols, long long rows,
+                     long long outer, long long row_stride, long long outer_stride, int box_cols,
+                     int box_rows) {
+  EncodeTiledFn enc;
+  RH_TRY(get_encoder(&enc));
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)outer_stride * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(REHYAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return REHYAT_OK;
+}
+
+// A bf16 matrix operand of a batched GEMM: element (i, j) of batch b at
+// ptr + b * batch_stride + i * ld + j, i.e. ld is the stride of the leading (non-contiguous)
+// index, in elements.
+struct Operand {
+  const void* ptr;
+  long long ld, batch_stride;
+  bool mn;  // false: K contiguous; true: M (for A) or N (for B) contiguous
+};
+
+// C[b] (+)= alpha A[b] B[b] with A M x K, B K x N (layouts per Operand::mn), C [M][N] with row
+// stride ldc.  Strides and bases must be 16-byte aligned (multiples of 8 elements).
+int launch_gemm(int M, int N, int K, int batch, const Operand& A, const Operand& B, void* C,
+                long long ldc, long long c_batch, bool c_bf16, bool accumulate, float alpha,
+                cudaStream_t st) {
+  if (M < 1 || N < 1 || K < 1 || batch < 1) return fail(REHYAT_ERR_ARG, "empty GEMM");
+  if ((A.ld | A.batch_stride | B.ld | B.batch_stride) & 7)
+    return fail(REHYAT_ERR_ALIGN, "GEMM operand strides must be multiples of 8 elements");
+  if (!aligned16(A.ptr) || !aligned16(B.ptr) || !aligned16(C) || (!c_bf16 && ((ldc | c_batch) & 3)))
+    return fail(REHYAT_ERR_ALIGN, "GEMM pointers must be 16-byte aligned");
+  CUtensorMap ma, mb;
+  if (A.mn) RH_TRY(make_map_strided(&ma, A.ptr, M, K, batch, A.ld, A.batch_stride, 64, 64));
+  else RH_TRY(make_map_strided(&ma, A.ptr, K, M, batch, A.ld, A.batch_stride, 64, 128));
+  if (B.mn) RH_TRY(make_map_strided(&mb, B.ptr, N, K, batch, B.ld, B.batch_stride, 64, 64));
+  else RH_TRY(make_map_strided(&mb, B.ptr, K, N, batch, B.ld, B.batch_stride, 64, 128));
+  rehyat::gemm::Params gp{};
+  gp.M = M; gp.N = N; gp.K = K; gp.a_mn = A.mn; gp.b_mn = B.mn;
+  gp.C = C; gp.ldc = ldc; gp.c_batch = c_batch; gp.c_bf16 = c_bf16; gp.accumulate = accumulate;
+  gp.alpha = alpha;
+  auto k = rehyat::gemm::gemm_bf16_kernel;
+  RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)rehyat::gemm::kSmemBytes), "gemm attr"));
+  dim3 grid((N + 127) / 128, (M + 127) / 128, batch);
+  k<<<grid, rehyat::gemm::kThreads, rehyat::gemm::kSmemBytes, st>>>(ma, mb, gp);
+  return cuda_check(cudaGetLastError(), "gemm launch");
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -849,6 +903,17 @@ int rehyat_chunk_states(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, in
     return forward_states_bf16(d, T, L, Tc, To, k, v, Wk, bk, pl, ws, nullptr, nullptr, S_out,
                                Z_out, st);
   return forward_states_f32(d, T, L, Tc, To, k, v, Wk, bk, pl, ws, S_out, Z_out, st);
+}
+
+int rehyat_gemm_bf16(int M, int N, int K, int batch, const void* A, long long lda,
+                     long long a_batch, int a_mn, const void* B, long long ldb, long long b_batch,
+                     int b_mn, void* C, long long ldc, long long c_batch, int c_bf16,
+                     int accumulate, float alpha, void* stream) {
+  g_msg[0] = 0;
+  if (!A || !B || !C) return fail(REHYAT_ERR_ARG, "null pointer");
+  return launch_gemm(M, N, K, batch, Operand{A, lda, a_batch, a_mn != 0},
+                     Operand{B, ldb, b_batch, b_mn != 0}, C, ldc, c_batch, c_bf16 != 0,
+                     accumulate != 0, alpha, static_cast<cudaStream_t>(stream));
 }
 
 int rehyat_selftest_wait_timeout(long long limit_ns, void* stream) {

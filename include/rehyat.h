@@ -212,6 +212,21 @@ int rehyat_chunk_states(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens,
                         float* S_out, float* Z_out, void* workspace, size_t ws_bytes,
                         void* stream);
 
+/* Batched bf16 GEMM on the tensor cores (the building block of the backward pass; no
+ * counterpart on the pages): for b < batch, C[b] = alpha * A[b] B[b] (accumulate = 0) or
+ * C[b] += alpha * A[b] B[b] (accumulate = 1), fp32 accumulation, C fp32 (c_bf16 = 0) or bf16.
+ *   A is M x K: element (m, k) of batch b at A + b*a_batch + m*lda + k (a_mn = 0) or
+ *               A + b*a_batch + k*lda + m (a_mn = 1); bf16.
+ *   B is K x N: element (k, n) at B + b*b_batch + n*ldb + k (b_mn = 0) or
+ *               B + b*b_batch + k*ldb + n (b_mn = 1); bf16.
+ *   C [M][N] per batch: element (m, n) at C + b*c_batch + m*ldc + n.
+ * Strides in elements; A, B strides multiples of 8, fp32 ldc a multiple of 4, pointers 16-byte
+ * aligned (REHYAT_ERR_ALIGN otherwise).  Enqueued on `stream`; allocates nothing. */
+int rehyat_gemm_bf16(int M, int N, int K, int batch, const void* A, long long lda,
+                     long long a_batch, int a_mn, const void* B, long long ldb, long long b_batch,
+                     int b_mn, void* C, long long ldc, long long c_batch, int c_bf16,
+                     int accumulate, float alpha, void* stream);
+
 /* Failure-path self test (no counterpart on the pages): enqueue on `stream` one small kernel whose
  * warps wait on an mbarrier that nothing arrives on, with the same bounded wait the other
  * kernels use but a limit of `limit_ns` nanoseconds (1e3 .. 2e9).  The wait gives up, the kernel
