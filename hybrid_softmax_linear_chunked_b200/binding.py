@@ -26,6 +26,7 @@ EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_forward_phiq", "rehyat_forward_attend", "rehyat_chunk_workspace_size",
             "rehyat_chunk_forward", "rehyat_chunk_forward_sched", "rehyat_chunk_carry_workspace_size",
             "rehyat_chunk_forward_carry", "rehyat_chunk_forward_static", "rehyat_chunk_states",
+            "rehyat_forward_train", "rehyat_backward_workspace_size", "rehyat_backward",
             "rehyat_gemm_bf16", "rehyat_selftest_wait_timeout", "rehyat_sync_status"]
 
 
@@ -87,6 +88,11 @@ def load() -> ctypes.CDLL:
     L.rehyat_chunk_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
                                       P, c_size_t, P]
     LL = ctypes.c_longlong
+    L.rehyat_forward_train.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
+                                       P, P, P, P, c_size_t, P]
+    L.rehyat_backward_workspace_size.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int,
+                                                 ctypes.POINTER(c_size_t)]
+    L.rehyat_backward.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int] + [P] * 18 + [c_size_t, P]
     L.rehyat_gemm_bf16.argtypes = [c_int, c_int, c_int, c_int, P, LL, LL, c_int, P, LL, LL, c_int,
                                    P, LL, LL, c_int, c_int, ctypes.c_float, P]
     L.rehyat_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
@@ -331,6 +337,57 @@ def chunk_forward_static(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, phi: 
                                            _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(S),
                                            _ptr(Z), _ptr(out), _stream(dev)))
     return out
+
+
+def forward_train(q, k, v, Wq, bq, Wk, bk, *, P: int, phi: int = 0, frame_tokens: int, Tc: int,
+                  To: int, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """`forward` that also returns lse [B,H,N] fp32 (log2 of every row's denominator), which
+    `backward` needs.  bf16 only."""
+    lib = load()
+    dev = _dev(q, k, v, Wq, bq, Wk, bk)
+    _weights(Wq, bq), _weights(Wk, bk)
+    d = dims_of(q, Wq, P, phi)
+    N = q.shape[2]
+    T = N // frame_tokens
+    code = _dtype_code(q)
+    ws = _workspace(forward_workspace_size(d, code, T, frame_tokens, Tc, To), dev, workspace)
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[1], N, dtype=torch.float32, device=dev)
+    _check(lib.rehyat_forward_train(d, code, T, frame_tokens, Tc, To, _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(out), _ptr(lse),
+                                    _ptr(ws), ws.numel(), _stream(dev)))
+    return out, lse
+
+
+def backward_workspace_size(d: Dims, dtype_code: int, T: int, L_: int, Tc: int, To: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().rehyat_backward_workspace_size(d, dtype_code, T, L_, Tc, To, ctypes.byref(n)))
+    return n.value
+
+
+def backward(q, k, v, Wq, bq, Wk, bk, out, lse, dout, *, P: int, phi: int = 0,
+             frame_tokens: int, Tc: int, To: int, workspace: torch.Tensor | None = None) -> dict:
+    """Gradients of sum(dout * out) for every input: dict with dq, dk, dv [B,H,N,D], dWq, dWk
+    [H,G,F/G,D/G], dbq, dbk [H,F] (fp32)."""
+    lib = load()
+    dev = _dev(q, k, v, Wq, bq, Wk, bk, out, lse, dout)
+    d = dims_of(q, Wq, P, phi)
+    N = q.shape[2]
+    T = N // frame_tokens
+    code = _dtype_code(q)
+    ws = _workspace(backward_workspace_size(d, code, T, frame_tokens, Tc, To), dev, workspace)
+    g = {n: torch.empty(q.shape, dtype=torch.float32, device=dev) for n in ("dq", "dk", "dv")}
+    g["dWq"] = torch.empty(Wq.shape, dtype=torch.float32, device=dev)
+    g["dWk"] = torch.empty(Wk.shape, dtype=torch.float32, device=dev)
+    g["dbq"] = torch.empty(d.H, d.F, dtype=torch.float32, device=dev)
+    g["dbk"] = torch.empty(d.H, d.F, dtype=torch.float32, device=dev)
+    _check(lib.rehyat_backward(d, code, T, frame_tokens, Tc, To, _ptr(q), _ptr(k), _ptr(v),
+                               _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(out), _ptr(lse),
+                               _ptr(dout), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                               _ptr(g["dWq"]), _ptr(g["dbq"]), _ptr(g["dWk"]), _ptr(g["dbk"]),
+                               _ptr(ws), ws.numel(), _stream(dev)))
+    return g
 
 
 def gemm(A: torch.Tensor, B: torch.Tensor, *, a_mn: bool = False, b_mn: bool = False,

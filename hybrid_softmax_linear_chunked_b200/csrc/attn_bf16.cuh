@@ -80,6 +80,7 @@ struct Params {
   const float* bq;    // [H, F] or null
   const float* Z;     // [BH, n_states, F]
   __nv_bfloat16* out; // [BH, nq_rows, D]
+  float* lse;         // [BH, nq_rows] or null: log2 of each row's denominator (for the backward)
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -586,6 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row_in_chunk = tile_row0 + t * kBM + r;
         const bool row_valid = row_in_chunk < nq;
         const float inv = 1.f / l;
+        if (p.lse && row_valid)
+          p.lse[(size_t)bh * p.nq_rows + q_row0 + row_in_chunk] = m + log2f(l);
         __nv_bfloat16* orow = p.out + ((size_t)bh * p.nq_rows + q_row0 + row_in_chunk) * kHD;
 #pragma unroll
         for (int cc = 0; cc < kHD / 32; ++cc) {

@@ -16,6 +16,7 @@
 #include "attn_bf16.cuh"
 #include "featmap.cuh"
 #include "fp32_path.cuh"
+#include "backward.cuh"
 #include "gemm_bf16.cuh"
 #include "phi_bf16.cuh"
 #include "sm100.cuh"
@@ -481,6 +482,101 @@ __global__ void __launch_bounds__(64) wait_timeout_selftest_kernel(unsigned long
 // =============================================================================================
 // C ABI
 // =============================================================================================
+// ---------------------------------------------------------------------------------------------
+// Backward workspace: the forward's (states, phi_q), then the backward's own buffers.
+// ---------------------------------------------------------------------------------------------
+struct BackwardPlan {
+  ForwardPlan fwd;
+  int C, c_lin, nq_max, nw_max, nblk_r, nblk_b;
+  size_t fwd_off, fwd_bytes, phik, Drow, lam, SB, DPB, PB, DSB, GB, phis, dphiq, dphik, U, DU, RB,
+      Rt, rpart, rt, dWbd, dbpart, total;
+};
+
+BackwardPlan plan_backward(const rehyat_dims& d, int T, int L, int Tc, int To) {
+  BackwardPlan p{};
+  p.fwd = plan_forward(d, REHYAT_BF16, T, L, Tc, To);
+  const size_t BH = (size_t)d.B * d.H, N = (size_t)T * L, F = d.F, D = d.D;
+  p.C = (T + Tc - 1) / Tc;
+  p.c_lin = To / Tc + 1;  // first chunk with a linear region
+  p.nq_max = (Tc < T ? Tc : T) * L;
+  p.nw_max = ((Tc + To) < T ? (Tc + To) : T) * L;
+  p.nblk_r = (p.nq_max + 255) / 256;
+  p.nblk_b = (int)((N + 255) / 256);
+  Carve cv;
+  p.fwd_off = cv.take(p.fwd.total);
+  p.fwd_bytes = p.fwd.total;
+  p.phik = cv.take(BH * N * F * 2);
+  p.Drow = cv.take(BH * N * 4);
+  p.lam = cv.take(BH * N * 4);
+  const size_t SW = BH * (size_t)p.nq_max * p.nw_max;
+  p.SB = cv.take(SW * 4);
+  p.DPB = cv.take(SW * 4);
+  p.PB = cv.take(SW * 2);
+  p.DSB = cv.take(SW * 2);
+  p.GB = cv.take(BH * p.nq_max * F * 4);
+  p.phis = cv.take(BH * p.nq_max * F * 2);
+  p.dphiq = cv.take(BH * N * F * 4);
+  p.dphik = cv.take(BH * N * F * 4);
+  p.U = cv.take(BH * N * F * 4);
+  p.DU = cv.take(BH * N * F * 2);
+  p.RB = cv.take(BH * p.C * F * D * 4);
+  p.Rt = cv.take(BH * p.C * F * D * 2);
+  p.rpart = cv.take((size_t)p.C * BH * p.nblk_r * F * 4);
+  p.rt = cv.take(BH * p.C * F * 4);
+  p.dWbd = cv.take((size_t)d.H * F * D * 4);
+  p.dbpart = cv.take(BH * p.nblk_b * F * 4);
+  p.total = cv.off;
+  return p;
+}
+
+// Feature-map backward of rows [r0, r1) of every (b, h): U = x Wbd^T, du = (g - rsub) f'(U + b),
+// dx += du Wbd, dW += diag blocks of du^T x, db += column sums of du.
+int feature_backward(const rehyat_dims& d, long long N, long long r0, long long r1,
+                     const void* x, const __nv_bfloat16* Wbd, const float* bias, const float* g,
+                     const float* rsub, int C, int L, int Tc, int To, const BackwardPlan& pl,
+                     uint8_t* ws, float* dx, float* dW, float* db, cudaStream_t st) {
+  if (r1 <= r0) return REHYAT_OK;
+  const long long rows = r1 - r0, F = d.F, D = d.D;
+  const int H = d.H, BH = d.B * d.H;
+  float* U = reinterpret_cast<float*>(ws + pl.U);
+  __nv_bfloat16* DU = reinterpret_cast<__nv_bfloat16*>(ws + pl.DU);
+  float* dWbd = reinterpret_cast<float*>(ws + pl.dWbd);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  for (int b = 0; b < d.B; ++b) {
+    const long long bo = (long long)b * H * N;  // first row of batch b
+    for (int part = 0; part < 2; ++part)       // U = x Wbd_hi^T + x Wbd_lo^T
+      RH_TRY(launch_gemm((int)rows, (int)F, (int)D, H,
+                         Operand{xb + (bo + r0) * D, D, N * D, false},
+                         Operand{Wbd + part * F * D, D, 2 * F * D, false},
+                         U + (bo + r0) * F, F, N * F, false, part > 0, 1.f, st));
+  }
+  rehyat::bwd::feat_grad_kernel<<<dim3((unsigned)rows, BH), d.F, 0, st>>>(
+      U, bias, H, g, rsub, C, L, Tc, To, d.F, kernel_P(d), N, r0, DU);
+  RH_TRY(cuda_check(cudaGetLastError(), "feature gradient launch"));
+  RH_TRY(cuda_check(cudaMemsetAsync(dWbd, 0, (size_t)H * F * D * 4, st), "memset"));
+  for (int b = 0; b < d.B; ++b) {
+    const long long bo = (long long)b * H * N;
+    for (int part = 0; part < 2; ++part)       // dx += du Wbd_hi + du Wbd_lo
+      RH_TRY(launch_gemm((int)rows, (int)D, (int)F, H,
+                         Operand{DU + (bo + r0) * F, F, N * F, false},
+                         Operand{Wbd + part * F * D, D, 2 * F * D, true},
+                         dx + (bo + r0) * D, D, N * D, false, true, 1.f, st));
+    // dWbd += du^T x over this batch's rows
+    RH_TRY(launch_gemm((int)F, (int)D, (int)rows, H, Operand{DU + (bo + r0) * F, F, N * F, true},
+                       Operand{xb + (bo + r0) * D, D, N * D, true}, dWbd, D, F * D, false, true,
+                       1.f, st));
+  }
+  rehyat::bwd::blockdiag_grad_kernel<<<dim3((unsigned)((F * (D / d.G) + 255) / 256), H), 256, 0,
+                                       st>>>(dWbd, d.D, d.F, d.G, dW);
+  RH_TRY(cuda_check(cudaGetLastError(), "weight gradient launch"));
+  float* part = reinterpret_cast<float*>(ws + pl.dbpart);
+  const int nblk = (int)((rows + 255) / 256);
+  rehyat::bwd::colsum_part_kernel<<<dim3(nblk, BH), d.F, 0, st>>>(DU, d.F, N, r0, r1, part, nblk);
+  RH_TRY(cuda_check(cudaGetLastError(), "bias gradient launch"));
+  rehyat::bwd::bias_grad_kernel<<<H, d.F, 0, st>>>(part, d.B, H, d.F, nblk, db);
+  return cuda_check(cudaGetLastError(), "bias gradient launch");
+}
+
 extern "C" {
 
 const char* rehyat_last_error(void) { return g_msg; }
@@ -564,9 +660,21 @@ int rehyat_forward_phiq(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, in
   return launch_featmap(d, REHYAT_F32, (int)N, q, Wq, bq, ws + pl.phiq, st);
 }
 
+static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                               const void* q, const void* k, const void* v, void* out,
+                               float* lse, const void* workspace, size_t ws_bytes, void* stream);
+
 int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
                           const void* q, const void* k, const void* v, void* out,
                           const void* workspace, size_t ws_bytes, void* stream) {
+  return forward_attend_impl(d, dt, T, L, Tc, To, q, k, v, out, nullptr, workspace, ws_bytes,
+                             stream);
+}
+
+static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                               const void* q, const void* k, const void* v, void* out,
+                               float* lse, const void* workspace, size_t ws_bytes,
+                               void* stream) {
   g_msg[0] = 0;
   ForwardPlan pl;
   RH_TRY(forward_common_checks(d, dt, T, L, Tc, To, workspace, ws_bytes, &pl));
@@ -592,6 +700,7 @@ int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
     ap.bq = nullptr;  // phi_q comes finished from the workspace
     ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
     ap.out = static_cast<__nv_bfloat16*>(out);
+    ap.lse = lse;
     dim3 grid((rows_per_chunk + 255) / 256, pl.C, BH);
     return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, grid, st);
   }
@@ -622,6 +731,178 @@ int rehyat_forward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
   RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, workspace, ws_bytes, stream));
   RH_TRY(rehyat_forward_phiq(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream));
   return rehyat_forward_attend(d, dt, T, L, Tc, To, q, k, v, out, workspace, ws_bytes, stream);
+}
+
+int rehyat_forward_train(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                         const void* q, const void* k, const void* v, const float* Wq,
+                         const float* bq, const float* Wk, const float* bk, void* out, float* lse,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  g_msg[0] = 0;
+  if (dt != REHYAT_BF16) return fail(REHYAT_ERR_DTYPE, "the training forward is bf16 only");
+  ForwardPlan pl;
+  RH_TRY(forward_common_checks(d, dt, T, L, Tc, To, workspace, ws_bytes, &pl));
+  if (!q || !k || !v || !Wq || !Wk || !out || !lse) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(REHYAT_ERR_ALIGN, "q/k/v/out not 16-byte aligned");
+  RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, workspace, ws_bytes, stream));
+  RH_TRY(rehyat_forward_phiq(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream));
+  return forward_attend_impl(d, dt, T, L, Tc, To, q, k, v, out, lse, workspace, ws_bytes, stream);
+}
+
+int rehyat_backward_workspace_size(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                                   size_t* bytes) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  if (dt != REHYAT_BF16) return fail(REHYAT_ERR_DTYPE, "the backward pass is bf16 only");
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(T, L, Tc, To));
+  if (!bytes) return fail(REHYAT_ERR_ARG, "null bytes pointer");
+  *bytes = plan_backward(d, T, L, Tc, To).total;
+  return REHYAT_OK;
+}
+
+int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To, const void* q,
+                    const void* k, const void* v, const float* Wq, const float* bq,
+                    const float* Wk, const float* bk, const void* out, const float* lse,
+                    const void* dout, float* dq, float* dk, float* dv, float* dWq, float* dbq,
+                    float* dWk, float* dbk, void* workspace, size_t ws_bytes, void* stream) {
+  g_msg[0] = 0;
+  RH_TRY(check_dims(d, dt));
+  if (dt != REHYAT_BF16) return fail(REHYAT_ERR_DTYPE, "the backward pass is bf16 only");
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(T, L, Tc, To));
+  if (L % 8) return fail(REHYAT_ERR_SHAPE, "the backward needs frame_tokens %% 8 == 0 (got %d)", L);
+  if (!q || !k || !v || !Wq || !Wk || !out || !lse || !dout || !dq || !dk || !dv || !dWq ||
+      !dbq || !dWk || !dbk)
+    return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(REHYAT_ERR_ALIGN, "tensors must be 16-byte aligned");
+  const BackwardPlan pl = plan_backward(d, T, L, Tc, To);
+  if (!workspace || ws_bytes < pl.total)
+    return fail(REHYAT_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", pl.total, ws_bytes);
+  if (!aligned16(workspace)) return fail(REHYAT_ERR_ALIGN, "workspace not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* fw = ws + pl.fwd_off;
+  const int BH = d.B * d.H;
+  const long long N = (long long)T * L, F = d.F, D = d.D;
+  const int C = pl.C;
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
+  const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  auto b16 = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
+  const size_t ND = (size_t)BH * N * D * 4;
+  const size_t WB = (size_t)d.H * F * (D / d.G) * 4;
+  RH_TRY(cuda_check(cudaMemsetAsync(dq, 0, ND, st), "memset"));
+  RH_TRY(cuda_check(cudaMemsetAsync(dk, 0, ND, st), "memset"));
+  RH_TRY(cuda_check(cudaMemsetAsync(dv, 0, ND, st), "memset"));
+  RH_TRY(cuda_check(cudaMemsetAsync(dWq, 0, WB, st), "memset"));
+  RH_TRY(cuda_check(cudaMemsetAsync(dWk, 0, WB, st), "memset"));
+  RH_TRY(cuda_check(cudaMemsetAsync(dbq, 0, (size_t)d.H * F * 4, st), "memset"));
+  RH_TRY(cuda_check(cudaMemsetAsync(dbk, 0, (size_t)d.H * F * 4, st), "memset"));
+  RH_TRY(cuda_check(cudaMemsetAsync(ws + pl.RB, 0, (size_t)BH * C * F * D * 4, st), "memset"));
+  RH_TRY(cuda_check(cudaMemsetAsync(ws + pl.rpart, 0, (size_t)C * BH * pl.nblk_r * F * 4, st),
+                    "memset"));
+
+  // states S_c (transposed, bf16), Z_c and phi_q of the rows that read a state, as the forward
+  RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, fw, pl.fwd_bytes, stream));
+  RH_TRY(rehyat_forward_phiq(d, dt, T, L, Tc, To, q, Wq, bq, fw, pl.fwd_bytes, stream));
+  const __nv_bfloat16* St = reinterpret_cast<const __nv_bfloat16*>(fw + pl.fwd.St);
+  const float* Zc = reinterpret_cast<const float*>(fw + pl.fwd.Zc);
+  const __nv_bfloat16* phiq = reinterpret_cast<const __nv_bfloat16*>(fw + pl.fwd.phiq_bf16);
+  const __nv_bfloat16* Wqbd = reinterpret_cast<const __nv_bfloat16*>(fw + pl.fwd.Wqbd);
+  const __nv_bfloat16* Wkbd = reinterpret_cast<const __nv_bfloat16*>(fw + pl.fwd.Wkbd);
+  // the key rows that some later chunk reads linearly: [0, w_{C-1} L)
+  const long long wl = (long long)((C - 1) * Tc - To > 0 ? (C - 1) * Tc - To : 0) * L;
+  if (wl > 0) {
+    CUtensorMap mwk;
+    RH_TRY(make_map(&mwk, Wkbd, d.D, d.F, 2LL * d.H));
+    RH_TRY(launch_featmap_tc(d, k, (int)N, 0, (int)wl, mwk, bk, b16(pl.phik), st));
+  }
+  rehyat::bwd::rowstats_kernel<<<(unsigned)((BH * N + 7) / 8), 256, 0, st>>>(
+      dob, static_cast<const __nv_bfloat16*>(out), lse, BH * N, d.D, f32(pl.Drow), f32(pl.lam));
+  RH_TRY(cuda_check(cudaGetLastError(), "row statistics launch"));
+
+  const float sl2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
+  const float isd = (float)(1.0 / std::sqrt((double)d.D));
+  for (int c = 0; c < C; ++c) {
+    const int s = c * Tc, e = (s + Tc < T ? s + Tc : T), w = (s - To > 0 ? s - To : 0);
+    const long long nq = (long long)(e - s) * L, nw = (long long)(e - w) * L;
+    const long long r0 = (long long)s * L, k0 = (long long)w * L;
+    // S = Q_c K_w^T, dP = dO_c V_w^T (fp32)
+    RH_TRY(launch_gemm((int)nq, (int)nw, (int)D, BH, Operand{qb + r0 * D, D, N * D, false},
+                       Operand{kb + k0 * D, D, N * D, false}, f32(pl.SB), nw, nq * nw, false,
+                       false, 1.f, st));
+    RH_TRY(launch_gemm((int)nq, (int)nw, (int)D, BH, Operand{dob + r0 * D, D, N * D, false},
+                       Operand{vb + k0 * D, D, N * D, false}, f32(pl.DPB), nw, nq * nw, false,
+                       false, 1.f, st));
+    rehyat::bwd::softmax_grad_kernel<<<dim3((unsigned)nq, BH), 256, 0, st>>>(
+        f32(pl.SB), f32(pl.DPB), (int)nq, (int)nw, lse, f32(pl.Drow), N, r0, sl2, isd,
+        b16(pl.PB), b16(pl.DSB));
+    RH_TRY(cuda_check(cudaGetLastError(), "softmax gradient launch"));
+    // dq_c += dS K_w;  dk_w += dS^T Q_c;  dv_w += P^T dO_c
+    RH_TRY(launch_gemm((int)nq, (int)D, (int)nw, BH, Operand{b16(pl.DSB), nw, nq * nw, false},
+                       Operand{kb + k0 * D, D, N * D, true}, dq + r0 * D, D, N * D, false, true,
+                       1.f, st));
+    RH_TRY(launch_gemm((int)nw, (int)D, (int)nq, BH, Operand{b16(pl.DSB), nw, nq * nw, true},
+                       Operand{qb + r0 * D, D, N * D, true}, dk + k0 * D, D, N * D, false, true,
+                       1.f, st));
+    RH_TRY(launch_gemm((int)nw, (int)D, (int)nq, BH, Operand{b16(pl.PB), nw, nq * nw, true},
+                       Operand{dob + r0 * D, D, N * D, true}, dv + k0 * D, D, N * D, false, true,
+                       1.f, st));
+    if (w > 0) {
+      // G = dO_c S_c^T; dphi_q = lam (G - D Z_c); R_c = (lam phi_q)^T dO_c; r_c partials
+      RH_TRY(launch_gemm((int)nq, (int)F, (int)D, BH, Operand{dob + r0 * D, D, N * D, false},
+                         Operand{St + (long long)c * D * F, F, (long long)C * D * F, true},
+                         f32(pl.GB), F, nq * F, false, false, 1.f, st));
+      rehyat::bwd::phiq_grad_kernel<<<dim3((unsigned)nq, BH), d.F, 0, st>>>(
+          f32(pl.GB), (int)nq, d.F, N, r0, f32(pl.lam), f32(pl.Drow), Zc + (long long)c * F,
+          (long long)C * F, phiq, f32(pl.dphiq), b16(pl.phis));
+      RH_TRY(cuda_check(cudaGetLastError(), "phi_q gradient launch"));
+      RH_TRY(launch_gemm((int)F, (int)D, (int)nq, BH, Operand{b16(pl.phis), F, nq * F, true},
+                         Operand{dob + r0 * D, D, N * D, true},
+                         f32(pl.RB) + (long long)c * F * D, D, (long long)C * F * D, false, false,
+                         1.f, st));
+      const int nblk = (int)((nq + 255) / 256);
+      rehyat::bwd::rpart_kernel<<<dim3(nblk, BH), d.F, 0, st>>>(
+          (int)nq, d.F, N, r0, f32(pl.lam), f32(pl.Drow), phiq,
+          f32(pl.rpart) + (long long)c * BH * pl.nblk_r * F, pl.nblk_r);
+      RH_TRY(cuda_check(cudaGetLastError(), "r partial launch"));
+    }
+  }
+  if (wl > 0) {
+    rehyat::bwd::suffix_kernel<<<dim3((unsigned)((F * D + 255) / 256), BH), 256, 0, st>>>(
+        f32(pl.RB), f32(pl.rpart), C, pl.nblk_r, d.F, d.D, b16(pl.Rt), f32(pl.rt));
+    RH_TRY(cuda_check(cudaGetLastError(), "suffix launch"));
+    // keys folded after chunk c (frames [w_c, w_{c+1})) are read linearly from chunk c + 1 on
+    for (int c = 0; c + 1 < C; ++c) {
+      const int w0 = (c * Tc - To > 0 ? c * Tc - To : 0);
+      const int w1 = ((c + 1) * Tc - To > 0 ? (c + 1) * Tc - To : 0);
+      if (w1 <= w0) continue;
+      const long long g0 = (long long)w0 * L, ng = (long long)(w1 - w0) * L;
+      const __nv_bfloat16* Rt1 = b16(pl.Rt) + (long long)(c + 1) * F * D;
+      // dphi_k = V_g Rt^T (r~ is subtracted with the activation derivative); dv_g += phi_k Rt
+      RH_TRY(launch_gemm((int)ng, (int)F, (int)D, BH, Operand{vb + g0 * D, D, N * D, false},
+                         Operand{Rt1, D, (long long)C * F * D, false}, f32(pl.dphik) + g0 * F, F,
+                         N * F, false, false, 1.f, st));
+      RH_TRY(launch_gemm((int)ng, (int)D, (int)F, BH,
+                         Operand{b16(pl.phik) + g0 * F, F, N * F, false},
+                         Operand{Rt1, D, (long long)C * F * D, true}, dv + g0 * D, D, N * D,
+                         false, true, 1.f, st));
+    }
+  }
+  // through the feature maps: q rows of chunks with a linear region, k rows read linearly
+  const long long rq0 = (long long)pl.c_lin * Tc * L;
+  if (rq0 < N)
+    RH_TRY(feature_backward(d, N, rq0, N, q, Wqbd, bq, f32(pl.dphiq), nullptr, C, L, Tc, To, pl,
+                            ws, dq, dWq, dbq, st));
+  if (wl > 0)
+    RH_TRY(feature_backward(d, N, 0, wl, k, Wkbd, bk, f32(pl.dphik), f32(pl.rt), C, L, Tc, To,
+                            pl, ws, dk, dWk, dbk, st));
+  return REHYAT_OK;
 }
 
 int rehyat_chunk_workspace_size(rehyat_dims d, rehyat_dtype dt, int frame_tokens,

@@ -212,6 +212,32 @@ int rehyat_chunk_states(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens,
                         float* S_out, float* Z_out, void* workspace, size_t ws_bytes,
                         void* stream);
 
+/* ---- training: the forward that keeps its row statistics, and the backward pass ----
+ * The pages train the feature maps by distillation and then fine-tune ("ReHyAt overview" §3.1.1,
+ * §3.1.2); both need the gradients of the §2.2.1 output formula.  bf16 only (D = F = 128).
+ *
+ * rehyat_forward_train: rehyat_forward plus lse [B,H,T*L] fp32: for every query row, log2 of
+ *   its denominator (softmax sum plus linear term) in the units where key j weighs
+ *   2^(q.k_j log2(e) / sqrt(D)).  Same workspace as rehyat_forward.
+ * rehyat_backward: given q, k, v, the weights, the forward's out and lse, and dout = dL/dout
+ *   [B,H,T*L,D] bf16, writes dq, dk, dv [B,H,T*L,D] fp32, dWq, dWk [H,G,F/G,D/G] fp32 and dbq,
+ *   dbk [H,F] fp32 (summed over the batch; written even when bq / bk are NULL).  Needs
+ *   frame_tokens % 8 == 0 (REHYAT_ERR_SHAPE otherwise) and a workspace of
+ *   rehyat_backward_workspace_size bytes (it holds one chunk's score matrices: about
+ *   12 B * B*H * (Tc*L) * ((Tc+To)*L) plus O(B*H*T*L*F)). */
+int rehyat_forward_train(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
+                         const void* q, const void* k, const void* v, const float* Wq,
+                         const float* bq, const float* Wk, const float* bk, void* out, float* lse,
+                         void* workspace, size_t ws_bytes, void* stream);
+int rehyat_backward_workspace_size(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens,
+                                   int Tc, int To, size_t* bytes);
+int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
+                    const void* q, const void* k, const void* v, const float* Wq,
+                    const float* bq, const float* Wk, const float* bk, const void* out,
+                    const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                    float* dWq, float* dbq, float* dWk, float* dbk, void* workspace,
+                    size_t ws_bytes, void* stream);
+
 /* Batched bf16 GEMM on the tensor cores (the building block of the backward pass; no
  * counterpart on the pages): for b < batch, C[b] = alpha * A[b] B[b] (accumulate = 0) or
  * C[b] += alpha * A[b] B[b] (accumulate = 1), fp32 accumulation, C fp32 (c_bf16 = 0) or bf16.

@@ -139,3 +139,18 @@ def test_chunk_forward_carry_checks(lib):
                                         FAKE, None, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE,
                                         FAKE, 16, None)
     assert st == -4
+
+
+def test_backward_checks(lib):
+    d = dims()
+    n = ctypes.c_size_t(0)
+    assert lib.rehyat_backward_workspace_size(d, rb.REHYAT_F32, 7, 64, 3, 1, ctypes.byref(n)) == -3
+    assert lib.rehyat_backward_workspace_size(d, rb.REHYAT_BF16, 7, 64, 3, 1, ctypes.byref(n)) == 0
+    args = [FAKE] * 3 + [FAKE, None, FAKE, None] + [FAKE] * 3 + [FAKE] * 7 + [FAKE]
+    # frame_tokens not a multiple of 8
+    assert lib.rehyat_backward(d, rb.REHYAT_BF16, 7, 60, 3, 1, *args, 1 << 40, None) == -2
+    # workspace too small
+    assert lib.rehyat_backward(d, rb.REHYAT_BF16, 7, 64, 3, 1, *args, 16, None) == -4
+    # fp32 training forward refused
+    assert lib.rehyat_forward_train(d, rb.REHYAT_F32, 7, 64, 3, 1, FAKE, FAKE, FAKE, FAKE, None,
+                                    FAKE, None, FAKE, FAKE, FAKE, 1 << 40, None) == -3
