@@ -64,6 +64,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="480p5s")
     ap.add_argument("--phi", choices=["poly", "elu1"], default="poly")
+    ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
+                    help="backward: time the backward pass (the forward's out and row statistics "
+                         "are computed before the timed region)")
     ap.add_argument("--schedule", default=None,
                     help="streaming only: FRAMES/OVERLAP entries, first once, rest cyclic")
     return ap.parse_args()
@@ -300,7 +303,10 @@ def main():
     rb.load()
     w = pick_workload(args)
     inp = make_inputs(w, seed=rep.seed(w.seed))
-    run = (stream_runner if w.mode == "stream" else full_runner)(w, inp, dev, args)
+    if args.which == "backward":
+        run = backward_runner(w, inp, dev, args)
+    else:
+        run = (stream_runner if w.mode == "stream" else full_runner)(w, inp, dev, args)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(max(3, args.warmup)):
@@ -433,6 +439,58 @@ def full_runner(w: C.Workload, inp, dev, args) -> _Run:
     r.attn_flops = w.attn_tensor_flops()
     r.step_flops = w.flops(streaming=False)
     r.launches_per_step = 6  # 2 weight preps, fold, scan, phi_q, attention
+    return r
+
+
+def backward_runner(w: C.Workload, inp, dev, args) -> _Run:
+    """One backward pass over the whole sequence (dq, dk, dv, dW, db); the forward's output and
+    row statistics and a seeded dL/dout are in HBM before the timed region."""
+    r = _Run()
+    r.attn_isolated = False
+    q, k, v = (x.to(dev) for x in (inp.q, inp.k, inp.v))
+    Wq, bq, Wk, bk = (x.to(dev) for x in (inp.Wq, inp.bq, inp.Wk, inp.bk))
+    kw = dict(P=w.P, phi=w.phi_code, frame_tokens=w.frame_tokens, Tc=w.Tc, To=w.To)
+    out, lse = rb.forward_train(q, k, v, Wq, bq, Wk, bk, **kw)
+    dout = torch.randn(out.shape, generator=torch.Generator().manual_seed(w.seed + 1)).to(
+        torch.bfloat16).to(dev)
+    d = rb.dims_of(q, Wq, w.P, w.phi_code)
+    ws = torch.empty(rb.backward_workspace_size(d, rb.REHYAT_BF16, w.T, w.frame_tokens, w.Tc,
+                                                w.To), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev_mid=None, ev_end=None):
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        rb.backward(q, k, v, Wq, bq, Wk, bk, out, lse, dout, workspace=ws, **kw)
+        if ev_end is not None:
+            ev_end.record(stream)
+
+    host = [x.pin_memory() for x in (inp.q, inp.k, inp.v, inp.Wq, inp.bq, inp.Wk, inp.bk)]
+    host += [out.cpu().pin_memory(), lse.cpu().pin_memory(), dout.cpu().pin_memory()]
+    grads_h = {}
+
+    def e2e_step():
+        t = [x.to(dev, non_blocking=True) for x in host]
+        g = rb.backward(*t[:7], t[7], t[8], t[9], workspace=ws, **kw)
+        for name, x in g.items():
+            if name not in grads_h:
+                grads_h[name] = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+            grads_h[name].copy_(x, non_blocking=True)
+
+    r.step, r.e2e_step = step, e2e_step
+    r.h2d = sum(x.numel() * x.element_size() for x in host)
+    r.d2h = 3 * q.numel() * 4 + 2 * Wq.numel() * 4 + 2 * w.H * w.F * 4
+    r.attn_flops = w.backward_flops()
+    r.step_flops = w.backward_flops()
+    C_ = w.n_chunks
+    lin = sum(1 for (wf, _, _) in w.chunk_bounds() if wf > 0)
+    groups = sum(1 for c in range(C_ - 1) if w.chunk_bounds()[c + 1][0] > w.chunk_bounds()[c][0])
+    # phi_k, row stats, per chunk 2 GEMM + softmax-grad + 3 GEMM (+ linear: GEMM, phi_q grad,
+    # GEMM, r partials), suffix, per fold group 2 GEMM, two feature backwards (per batch 5 GEMM,
+    # feature grad, block-diagonal grad, column sums, bias grad), plus the forward states/phi_q
+    r.launches_per_step = (2 + 6 * C_ + 4 * lin + 1 + 2 * groups + 2 * (5 * w.B + 4) + 6)
+    r.roofline_kernel = "backward pass (all launches; algorithmic FLOPs / time)"
+    r.config = {"pass": "backward"}
     return r
 
 

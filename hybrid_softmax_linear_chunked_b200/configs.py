@@ -113,6 +113,26 @@ class Workload:
                 tot += 2.0 * nq * F * D
         return tot * self.B * self.H
 
+    def backward_flops(self) -> float:
+        """Algorithmic FLOPs of the backward over all (b, h): QK^T, dO V^T, dS K, dS^T Q and
+        P^T dO over each chunk's window; dO S_c^T and (lam phi_q)^T dO for chunks with a linear
+        region; V R~^T and phi_k R~ for the keys read linearly; and the grouped linear of each
+        feature map three times (u, dx, dW: 2 D F / G per token each)."""
+        L, D, F = self.frame_tokens, self.D, self.F
+        bounds = self.chunk_bounds()
+        tot = 0.0
+        q_rows = 0
+        for (w, s, e) in bounds:
+            nq, nw = (e - s) * L, (e - w) * L
+            tot += 10.0 * nq * nw * D
+            if w > 0:
+                tot += 4.0 * nq * D * F
+                q_rows += nq
+        k_rows = bounds[-1][0] * L
+        tot += 4.0 * k_rows * D * F
+        tot += 3 * 2.0 * (q_rows + k_rows) * D * F / self.G
+        return tot * self.B * self.H
+
     def io_bytes(self) -> float:
         """Algorithmic HBM bytes: q, k, v read once and the output written once."""
         el = 4 if self.dtype == "f32" else 2
