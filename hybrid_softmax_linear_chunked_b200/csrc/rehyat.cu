@@ -488,8 +488,8 @@ __global__ void __launch_bounds__(64) wait_timeout_selftest_kernel(unsigned long
 struct BackwardPlan {
   ForwardPlan fwd;
   int C, c_lin, nq_max, nw_max, nblk_r, nblk_b;
-  size_t fwd_off, fwd_bytes, phik, Drow, lam, SB, DPB, PB, DSB, GB, phis, dphiq, dphik, U, DU, RB,
-      Rt, rpart, rt, dWbd, dbpart, total;
+  size_t fwd_off, fwd_bytes, phik, Drow, lam, PB, DSB, GB, phis, dphiq, dphik, U, DU, RB, Rt,
+      rpart, rt, dWbd, dbpart, total;
 };
 
 BackwardPlan plan_backward(const rehyat_dims& d, int T, int L, int Tc, int To) {
@@ -509,8 +509,6 @@ BackwardPlan plan_backward(const rehyat_dims& d, int T, int L, int Tc, int To) {
   p.Drow = cv.take(BH * N * 4);
   p.lam = cv.take(BH * N * 4);
   const size_t SW = BH * (size_t)p.nq_max * p.nw_max;
-  p.SB = cv.take(SW * 4);
-  p.DPB = cv.take(SW * 4);
   p.PB = cv.take(SW * 2);
   p.DSB = cv.take(SW * 2);
   p.GB = cv.take(BH * p.nq_max * F * 4);
@@ -832,17 +830,24 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
     const int s = c * Tc, e = (s + Tc < T ? s + Tc : T), w = (s - To > 0 ? s - To : 0);
     const long long nq = (long long)(e - s) * L, nw = (long long)(e - w) * L;
     const long long r0 = (long long)s * L, k0 = (long long)w * L;
-    // S = Q_c K_w^T, dP = dO_c V_w^T (fp32)
-    RH_TRY(launch_gemm((int)nq, (int)nw, (int)D, BH, Operand{qb + r0 * D, D, N * D, false},
-                       Operand{kb + k0 * D, D, N * D, false}, f32(pl.SB), nw, nq * nw, false,
-                       false, 1.f, st));
-    RH_TRY(launch_gemm((int)nq, (int)nw, (int)D, BH, Operand{dob + r0 * D, D, N * D, false},
-                       Operand{vb + k0 * D, D, N * D, false}, f32(pl.DPB), nw, nq * nw, false,
-                       false, 1.f, st));
-    rehyat::bwd::softmax_grad_kernel<<<dim3((unsigned)nq, BH), 256, 0, st>>>(
-        f32(pl.SB), f32(pl.DPB), (int)nq, (int)nw, lse, f32(pl.Drow), N, r0, sl2, isd,
-        b16(pl.PB), b16(pl.DSB));
-    RH_TRY(cuda_check(cudaGetLastError(), "softmax gradient launch"));
+    // P and dS of the chunk's (query, window key) pairs, from S = Q_c K_w^T and dP = dO_c V_w^T
+    {
+      CUtensorMap mq, mk, mdo, mv;
+      RH_TRY(make_map_strided(&mq, qb + r0 * D, D, nq, BH, D, N * D, 64, 128));
+      RH_TRY(make_map_strided(&mk, kb + k0 * D, D, nw, BH, D, N * D, 64, 128));
+      RH_TRY(make_map_strided(&mdo, dob + r0 * D, D, nq, BH, D, N * D, 64, 128));
+      RH_TRY(make_map_strided(&mv, vb + k0 * D, D, nw, BH, D, N * D, 64, 128));
+      rehyat::bwd::ScoreParams sp{};
+      sp.nq = (int)nq; sp.nw = (int)nw; sp.stat_rows = N; sp.stat_row0 = r0;
+      sp.lse2 = lse; sp.Drow = f32(pl.Drow); sp.scale_log2 = sl2; sp.inv_sqrt_d = isd;
+      sp.P = b16(pl.PB); sp.dS = b16(pl.DSB);
+      auto kern = rehyat::bwd::score_grad_kernel;
+      RH_TRY(cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)rehyat::bwd::kScoreSmem), "score attr"));
+      kern<<<dim3((unsigned)((nw + 127) / 128), (unsigned)((nq + 127) / 128), BH),
+             rehyat::bwd::kScoreThreads, rehyat::bwd::kScoreSmem, st>>>(mq, mk, mdo, mv, sp);
+      RH_TRY(cuda_check(cudaGetLastError(), "score gradient launch"));
+    }
     // dq_c += dS K_w;  dk_w += dS^T Q_c;  dv_w += P^T dO_c
     RH_TRY(launch_gemm((int)nq, (int)D, (int)nw, BH, Operand{b16(pl.DSB), nw, nq * nw, false},
                        Operand{kb + k0 * D, D, N * D, true}, dq + r0 * D, D, N * D, false, true,
