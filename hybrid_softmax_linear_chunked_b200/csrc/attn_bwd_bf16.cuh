@@ -1,0 +1,433 @@
+// Fused softmax-window backward of the hybrid attention, FlashAttention style: the scores of a
+// (query tile, key tile) pair are recomputed in TMEM and never reach memory.  With the forward's
+// row statistics (lse2 = log2 of the row denominator, D = dO . O, both [BH][N] fp32):
+//   P = 2^(q.k log2(e)/sqrt(D) - lse2),   dS = P (dO . v - D) / sqrt(D)
+//   dV += P^T dO,  dK += dS^T Q          (dkdv_kernel: one CTA per key tile of a chunk's window,
+//                                          looping over the chunk's query tiles)
+//   dQ += dS K                           (dq_kernel: one CTA per query tile, looping over the
+//                                          window's key tiles)
+// The derivative is that of the "ReHyAt overview" page's §2.2.1 output formula; the linear
+// terms' gradients are separate (backward.cuh and tensor-core products).
+//
+// Both kernels: 192 threads.  Warps 0-3 compute (one TMEM lane = one row per thread), warp 4
+// loads by TMA (and allocates TMEM), warp 5 issues the MMAs.  Per loop step the MMA warp issues
+// the two score products (S and dP, SS), the compute warps turn them into packed bf16 P / dS
+// written back over the scores in TMEM, and the MMA warp issues the products that use them as
+// the A operand (TS).  Launch once per chunk (keys of the overlap frames belong to two chunks'
+// windows; the launches' += on dK, dV are ordered by the stream).
+#pragma once
+
+#include "attn_bf16.cuh"
+#include "sm100.cuh"
+
+namespace rehyat {
+namespace attn_bwd {
+
+using namespace sm100;
+using attn::kmajor_desc;
+using attn::mnmajor_desc;
+
+constexpr int kThreads = 192;
+constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 bf16 tile (two 128 x 64 boxes)
+constexpr uint32_t kStatBytes = 2 * 128 * 4;
+
+struct Params {
+  int L, T, Tc, To, c;   // frames per chunk etc.; c = the chunk of this launch
+  int N;                 // rows per (b, h)
+  const float* lse2;     // [BH][N]
+  const float* Drow;     // [BH][N]
+  float scale_log2, inv_sqrt_d;
+  float* dq;             // [BH][N][D] fp32, +=
+  float* dk;
+  float* dv;
+};
+
+struct Geometry {
+  int q_row0, nq, k_row0, nw;
+};
+
+__device__ __forceinline__ Geometry geometry(const Params& p) {
+  const int s = p.c * p.Tc;
+  const int e = min(s + p.Tc, p.T);
+  const int w = max(0, s - p.To);
+  return Geometry{s * p.L, (e - s) * p.L, w * p.L, (e - w) * p.L};
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                          int row, int bh) {
+  tma_load_3d(dst, map, bar, 0, row, bh);
+  tma_load_3d(dst + 128 * 128, map, bar, 64, row, bh);
+}
+
+// Adds 32 fp32 values (TMEM words) to a row of a fp32 [..][128] tensor.
+__device__ __forceinline__ void add_row32(float* dst, const uint32_t* r) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float4 o = d4[i];
+    o.x += __uint_as_float(r[4 * i]);
+    o.y += __uint_as_float(r[4 * i + 1]);
+    o.z += __uint_as_float(r[4 * i + 2]);
+    o.w += __uint_as_float(r[4 * i + 3]);
+    d4[i] = o;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// dK, dV: CTA = one 128-key tile of chunk c's window; loop over the chunk's query tiles.
+// TMEM: S^T [0,128) -> P^T, dP^T [128,256) -> dS^T, dV [256,384), dK [384,512).
+// smem: K, V (resident), Q and dO in 2 stages, the query tiles' lse2 and D in 2 stages.
+// ------------------------------------------------------------------------------------------
+constexpr uint32_t kKOffK = 0, kKOffV = kTile, kKOffQ = 2 * kTile, kKOffO = 4 * kTile;
+constexpr uint32_t kKOffStat = 6 * kTile;
+constexpr uint32_t kKSmem = kKOffStat + 2 * kStatBytes + 1024;
+enum KBar { kKvFull = 0, kQFull = 1, kQEmpty = 3, kSdFull = 5, kPdFull = 6, kKDone = 7, kKBars = 8 };
+
+// grid (ceil(nw / 128), 1, BH)
+__global__ void __launch_bounds__(kThreads, 1)
+    dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                const Params p) {
+  static_assert(kKSmem + 256 <= 232448, "shared memory over the limit");
+  const Geometry g = geometry(p);
+  const int bh = blockIdx.z;
+  const int key0 = blockIdx.x * 128;  // within the window
+  if (key0 >= g.nw) return;
+  const int n_q = (g.nq + 127) / 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  __shared__ __align__(8) uint64_t bars[kKBars];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  volatile int* abort_flag = &abort_sh;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (warp == 4) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kKBars; ++i) mbar_init(&bars[i], i == kPdFull ? 128 : 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  float* sStat = reinterpret_cast<float*>(sm + kKOffStat);  // [stage][lse 128 | D 128]
+
+  if (warp == 4) {
+    // ---- producer ----
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmO);
+      mbar_arrive_expect_tx(&bars[kKvFull], 2 * kTile);
+      load_tile(sm + kKOffK, &tmK, &bars[kKvFull], g.k_row0 + key0, bh);
+      load_tile(sm + kKOffV, &tmV, &bars[kKvFull], g.k_row0 + key0, bh);
+    }
+    __syncwarp();
+    bool ok = true;
+    int issued = 0;
+    for (int i = 0; i < n_q; ++i) {
+      const int s = i & 1;
+      if (i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQEmpty + s], ((i >> 1) - 1) & 1, abort_flag));
+      if (!ok) break;
+      // the query tile's statistics; rows past the chunk get lse2 = +inf, so P = dS = 0 there
+      float* st = sStat + s * 256;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int qi = i * 128 + lane * 4 + t;
+        const bool valid = qi < g.nq;
+        const long long idx = (long long)bh * p.N + g.q_row0 + (valid ? qi : 0);
+        st[lane * 4 + t] = valid ? p.lse2[idx] : INFINITY;
+        st[128 + lane * 4 + t] = valid ? p.Drow[idx] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars[kQFull + s], 2 * kTile);
+        load_tile(sm + kKOffQ + s * kTile, &tmQ, &bars[kQFull + s], g.q_row0 + i * 128, bh);
+        load_tile(sm + kKOffO + s * kTile, &tmO, &bars[kQFull + s], g.q_row0 + i * 128, bh);
+      }
+      __syncwarp();
+      ++issued;
+    }
+    if (!ok) {
+      mbar_wait_drain(&bars[kKvFull], 0);
+      for (int i = max(0, issued - 2); i < issued; ++i)
+        mbar_wait_drain(&bars[kQFull + (i & 1)], (i >> 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ---- MMA issuer ----
+    const uint32_t id_ss = idesc_bf16(128, 128, false, false);
+    const uint32_t id_ts = idesc_bf16(128, 128, false, true);
+    const uint32_t sK = smem_u32(sm + kKOffK), sV = smem_u32(sm + kKOffV);
+    auto wait = [&](int b, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, abort_flag));
+    };
+    bool ok = wait(kKvFull, 0);
+    for (int i = 0; i < n_q && ok; ++i) {
+      const int s = i & 1;
+      const uint32_t sQ = smem_u32(sm + kKOffQ + s * kTile), sO = smem_u32(sm + kKOffO + s * kTile);
+      ok = wait(kQFull + s, (i >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        for (int kk = 0; kk < 8; ++kk)  // S^T = K Q^T
+          mma_ss(tmem, kmajor_desc(sK, kk), kmajor_desc(sQ, kk), id_ss, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)  // dP^T = V dO^T
+          mma_ss(tmem + 128, kmajor_desc(sV, kk), kmajor_desc(sO, kk), id_ss, kk > 0 ? 1u : 0u);
+        mma_commit(&bars[kSdFull]);
+      }
+      __syncwarp();
+      ok = wait(kPdFull, i & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        for (int kk = 0; kk < 8; ++kk)  // dV += P^T dO
+          mma_ts(tmem + 256, tmem + kk * 8, mnmajor_desc(sO, kk), id_ts, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
+          mma_ts(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(sQ, kk), id_ts,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[kQEmpty + s]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) mma_commit(&bars[kKDone]);
+    __syncwarp();
+    mbar_wait_drain(&bars[kKDone], 0);
+    __syncwarp();
+  } else {
+    // ---- compute: thread = key row r of the tile ----
+    const int r = tid;  // 0..127, TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base, tD = tmem + lane_base + 128;
+    const float sl2 = p.scale_log2, isd = p.inv_sqrt_d;
+    bool ok = true;
+    for (int i = 0; i < n_q; ++i) {
+      const int s = i & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSdFull], i & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const float* lse = sStat + s * 256;
+      const float* Dq = lse + 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + c * 32, sv);
+        tmem_ld32(tD + c * 32, dv);
+        uint32_t pp[16], gg[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int q0 = c * 32 + 2 * e;
+          const float p0 = attn::ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -lse[q0]));
+          const float p1 = attn::ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -lse[q0 + 1]));
+          pp[e] = pack_bf16x2(p0, p1);
+          gg[e] = pack_bf16x2(p0 * (__uint_as_float(dv[2 * e]) - Dq[q0]) * isd,
+                              p1 * (__uint_as_float(dv[2 * e + 1]) - Dq[q0 + 1]) * isd);
+        }
+        // packed columns [16c, 16c + 16) hold scores already read (chunks c / 2 and c)
+        tmem_st16(tS + c * 16, pp);
+        tmem_st16(tD + c * 16, gg);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[kPdFull]);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKDone], 0, abort_flag)) && !*abort_flag;
+    if (ok) {
+      tc_fence_after();
+      const bool row_ok = key0 + r < g.nw;
+      const long long row = (long long)bh * p.N + g.k_row0 + key0 + r;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tmem + lane_base + 256 + cc * 32, a);
+        tmem_ld32(tmem + lane_base + 384 + cc * 32, b);
+        if (row_ok) {
+          add_row32(p.dv + row * 128 + cc * 32, a);
+          add_row32(p.dk + row * 128 + cc * 32, b);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// dQ: CTA = one 128-row query tile of chunk c; loop over the window's key tiles.
+// TMEM: S [0,128), dP [128,256) -> dS, dQ [256,384).  smem: Q, dO (resident), K and V in 2
+// stages.
+// ------------------------------------------------------------------------------------------
+constexpr uint32_t kQOffQ = 0, kQOffO = kTile, kQOffK = 2 * kTile, kQOffV = 4 * kTile;
+constexpr uint32_t kQSmem = 6 * kTile + 1024;
+enum QBar { kQoFull = 0, kKFull = 1, kKEmpty = 3, kSFull = 5, kDsFull = 6, kQDone = 7, kQBars = 8 };
+
+// grid (ceil(nq / 128), 1, BH)
+__global__ void __launch_bounds__(kThreads, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const Params p) {
+  static_assert(kQSmem + 256 <= 232448, "shared memory over the limit");
+  const Geometry g = geometry(p);
+  const int bh = blockIdx.z;
+  const int q0 = blockIdx.x * 128;  // within the chunk
+  if (q0 >= g.nq) return;
+  const int n_k = (g.nw + 127) / 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  __shared__ __align__(8) uint64_t bars[kQBars];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  volatile int* abort_flag = &abort_sh;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (warp == 4) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kQBars; ++i) mbar_init(&bars[i], i == kDsFull ? 128 : 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 4) {
+    // ---- producer ----
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bars[kQoFull], 2 * kTile);
+      load_tile(sm + kQOffQ, &tmQ, &bars[kQoFull], g.q_row0 + q0, bh);
+      load_tile(sm + kQOffO, &tmO, &bars[kQoFull], g.q_row0 + q0, bh);
+    }
+    __syncwarp();
+    bool ok = true;
+    int issued = 0;
+    for (int j = 0; j < n_k; ++j) {
+      const int s = j & 1;
+      if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty + s], ((j >> 1) - 1) & 1, abort_flag));
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars[kKFull + s], 2 * kTile);
+        load_tile(sm + kQOffK + s * kTile, &tmK, &bars[kKFull + s], g.k_row0 + j * 128, bh);
+        load_tile(sm + kQOffV + s * kTile, &tmV, &bars[kKFull + s], g.k_row0 + j * 128, bh);
+      }
+      __syncwarp();
+      ++issued;
+    }
+    if (!ok) {
+      mbar_wait_drain(&bars[kQoFull], 0);
+      for (int j = max(0, issued - 2); j < issued; ++j)
+        mbar_wait_drain(&bars[kKFull + (j & 1)], (j >> 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ---- MMA issuer ----
+    const uint32_t id_ss = idesc_bf16(128, 128, false, false);
+    const uint32_t id_ts = idesc_bf16(128, 128, false, true);
+    const uint32_t sQ = smem_u32(sm + kQOffQ), sO = smem_u32(sm + kQOffO);
+    auto wait = [&](int b, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, abort_flag));
+    };
+    bool ok = wait(kQoFull, 0);
+    for (int j = 0; j < n_k && ok; ++j) {
+      const int s = j & 1;
+      const uint32_t sK = smem_u32(sm + kQOffK + s * kTile), sV = smem_u32(sm + kQOffV + s * kTile);
+      ok = wait(kKFull + s, (j >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        for (int kk = 0; kk < 8; ++kk)  // S = Q K^T
+          mma_ss(tmem, kmajor_desc(sQ, kk), kmajor_desc(sK, kk), id_ss, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)  // dP = dO V^T
+          mma_ss(tmem + 128, kmajor_desc(sO, kk), kmajor_desc(sV, kk), id_ss, kk > 0 ? 1u : 0u);
+        mma_commit(&bars[kSFull]);
+      }
+      __syncwarp();
+      ok = wait(kDsFull, j & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        for (int kk = 0; kk < 8; ++kk)  // dQ += dS K
+          mma_ts(tmem + 256, tmem + 128 + kk * 8, mnmajor_desc(sK, kk), id_ts,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[kKEmpty + s]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) mma_commit(&bars[kQDone]);
+    __syncwarp();
+    mbar_wait_drain(&bars[kQDone], 0);
+    __syncwarp();
+  } else {
+    // ---- compute: thread = query row r of the tile ----
+    const int r = tid;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base, tD = tmem + lane_base + 128;
+    const float sl2 = p.scale_log2, isd = p.inv_sqrt_d;
+    const bool row_ok = q0 + r < g.nq;
+    const long long row = (long long)bh * p.N + g.q_row0 + q0 + r;
+    const float l2 = row_ok ? p.lse2[row] : INFINITY;
+    const float Di = row_ok ? p.Drow[row] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_k; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int valid = g.nw - j * 128;  // key columns of this tile inside the window
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + c * 32, sv);
+        tmem_ld32(tD + c * 32, dv);
+        uint32_t gg[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int k0 = c * 32 + 2 * e;
+          float p0 = attn::ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -l2));
+          float p1 = attn::ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -l2));
+          p0 = k0 < valid ? p0 : 0.f;
+          p1 = k0 + 1 < valid ? p1 : 0.f;
+          gg[e] = pack_bf16x2(p0 * (__uint_as_float(dv[2 * e]) - Di) * isd,
+                              p1 * (__uint_as_float(dv[2 * e + 1]) - Di) * isd);
+        }
+        tmem_st16(tD + c * 16, gg);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[kDsFull]);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQDone], 0, abort_flag)) && !*abort_flag;
+    if (ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_base + 256 + cc * 32, a);
+        if (row_ok) add_row32(p.dq + row * 128 + cc * 32, a);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace attn_bwd
+}  // namespace rehyat

@@ -182,147 +182,3 @@ __global__ void blockdiag_grad_kernel(const float* __restrict__ dWbd, int D, int
 }  // namespace bwd
 }  // namespace rehyat
 
-namespace rehyat {
-namespace bwd {
-
-using namespace sm100;
-
-// P and dS of one 128 x 128 tile of a chunk's (query, window key) pairs, straight from the
-// operands: S = Q K^T and dP = dO V^T (tcgen05, fp32 in TMEM columns [0, 128) and [128, 256)),
-// then per row (one thread per TMEM lane) P = 2^(S log2(e)/sqrt(D) - lse2) and
-// dS = P (dP - D_i) / sqrt(D), stored as bf16 [BH][nq][nw].  The score matrices never reach
-// memory in fp32.  Warp 0 loads the four 128 x 128 operand tiles (TMA, 8 boxes of 128 x 64),
-// warp 1 issues the 16 MMAs and owns TMEM, warps 2-5 compute and store.
-//   grid (ceil(nw / 128), ceil(nq / 128), BH), block 192, dynamic smem kScoreSmem.
-constexpr int kScoreThreads = 192;
-constexpr uint32_t kScoreTile = 128 * 64 * 2;  // one 128 x 64 box
-constexpr uint32_t kScoreSmem = 8 * kScoreTile + 1024;
-
-struct ScoreParams {
-  int nq, nw;
-  long long stat_rows, stat_row0;  // lse2 / Drow indexed [BH][stat_rows] from stat_row0
-  const float* lse2;
-  const float* Drow;
-  float scale_log2, inv_sqrt_d;
-  __nv_bfloat16* P;
-  __nv_bfloat16* dS;
-};
-
-__global__ void __launch_bounds__(kScoreThreads, 1)
-    score_grad_kernel(const __grid_constant__ CUtensorMap tmQ,
-                      const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmdO,
-                      const __grid_constant__ CUtensorMap tmV, const ScoreParams p) {
-  static_assert(kScoreSmem + 256 <= 232448, "shared memory over the limit");
-  const int n0 = blockIdx.x * 128, m0 = blockIdx.y * 128, bh = blockIdx.z;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[3];  // 0: Q, K loaded; 1: dO, V loaded; 2: MMAs done
-  __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_sh;
-  volatile int* abort_flag = &abort_sh;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (warp == 1) {
-    tmem_alloc(&tmem_base_sh, 256);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
-    abort_sh = 0;
-    fence_mbar_init();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base_sh;
-  // smem: [Q lo | Q hi | K lo | K hi | dO lo | dO hi | V lo | V hi], each 128 rows x 64 cols
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bars[0], 4 * kScoreTile);
-      for (int h = 0; h < 2; ++h) {
-        tma_load_3d(sm + (0 + h) * kScoreTile, &tmQ, &bars[0], h * 64, m0, bh);
-        tma_load_3d(sm + (2 + h) * kScoreTile, &tmK, &bars[0], h * 64, n0, bh);
-      }
-      mbar_arrive_expect_tx(&bars[1], 4 * kScoreTile);
-      for (int h = 0; h < 2; ++h) {
-        tma_load_3d(sm + (4 + h) * kScoreTile, &tmdO, &bars[1], h * 64, m0, bh);
-        tma_load_3d(sm + (6 + h) * kScoreTile, &tmV, &bars[1], h * 64, n0, bh);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    const uint32_t idesc = idesc_bf16(128, 128, false, false);
-    const uint32_t base = smem_u32(sm);
-    bool ok = true;
-    for (int pr = 0; pr < 2 && ok; ++pr) {  // pr 0: S = Q K^T; pr 1: dP = dO V^T
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[pr], 0, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t a = base + (4 * pr) * kScoreTile, b = base + (4 * pr + 2) * kScoreTile;
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kScoreTile + (kk & 3) * 32;
-          mma_ss(tmem + pr * 128, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(b + off, 16, 1024),
-                 idesc, kk > 0 ? 1u : 0u);
-        }
-      }
-      __syncwarp();
-    }
-    if (lane == 0) mma_commit(&bars[2]);
-    __syncwarp();
-    if (!ok) {
-      mbar_wait_drain(&bars[0], 0);
-      mbar_wait_drain(&bars[1], 0);
-    }
-    mbar_wait_drain(&bars[2], 0);
-  } else {
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[2], 0, abort_flag)) && !*abort_flag;
-    if (ok) {
-      tc_fence_after();
-      const int g = warp & 3;
-      const int i = m0 + g * 32 + lane;
-      const bool row_ok = i < p.nq;
-      const long long srow = (long long)bh * p.stat_rows + p.stat_row0 + (row_ok ? i : 0);
-      const float l2 = p.lse2[srow], Di = p.Drow[srow];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(g * 32) << 16);
-      const long long obase = ((long long)bh * p.nq + i) * p.nw;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t s[32], d[32];
-        tmem_ld32(taddr + c * 32, s);
-        tmem_ld32(taddr + 128 + c * 32, d);
-        const int col0 = n0 + c * 32;
-        if (!row_ok || col0 >= p.nw) continue;
-        uint32_t pp[16], gg[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = exp2f(fmaf(__uint_as_float(s[2 * e]), p.scale_log2, -l2));
-          const float p1 = exp2f(fmaf(__uint_as_float(s[2 * e + 1]), p.scale_log2, -l2));
-          pp[e] = pack_bf16x2(p0, p1);
-          gg[e] = pack_bf16x2(p0 * (__uint_as_float(d[2 * e]) - Di) * p.inv_sqrt_d,
-                              p1 * (__uint_as_float(d[2 * e + 1]) - Di) * p.inv_sqrt_d);
-        }
-        // nw is a multiple of 8: store whole 16-byte groups that lie inside the row
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          if (col0 + q4 * 8 < p.nw) {
-            *reinterpret_cast<uint4*>(p.P + obase + col0 + q4 * 8) =
-                make_uint4(pp[4 * q4], pp[4 * q4 + 1], pp[4 * q4 + 2], pp[4 * q4 + 3]);
-            *reinterpret_cast<uint4*>(p.dS + obase + col0 + q4 * 8) =
-                make_uint4(gg[4 * q4], gg[4 * q4 + 1], gg[4 * q4 + 2], gg[4 * q4 + 3]);
-          }
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 256);
-  }
-}
-
-}  // namespace bwd
-}  // namespace rehyat

@@ -14,6 +14,7 @@
 
 #include "../../include/rehyat.h"
 #include "attn_bf16.cuh"
+#include "attn_bwd_bf16.cuh"
 #include "featmap.cuh"
 #include "fp32_path.cuh"
 #include "backward.cuh"
@@ -488,8 +489,8 @@ __global__ void __launch_bounds__(64) wait_timeout_selftest_kernel(unsigned long
 struct BackwardPlan {
   ForwardPlan fwd;
   int C, c_lin, nq_max, nw_max, nblk_r, nblk_b;
-  size_t fwd_off, fwd_bytes, phik, Drow, lam, PB, DSB, GB, phis, dphiq, dphik, U, DU, RB, Rt,
-      rpart, rt, dWbd, dbpart, total;
+  size_t fwd_off, fwd_bytes, phik, Drow, lam, GB, phis, dphiq, dphik, U, DU, RB, Rt, rpart, rt,
+      dWbd, dbpart, total;
 };
 
 BackwardPlan plan_backward(const rehyat_dims& d, int T, int L, int Tc, int To) {
@@ -508,9 +509,6 @@ BackwardPlan plan_backward(const rehyat_dims& d, int T, int L, int Tc, int To) {
   p.phik = cv.take(BH * N * F * 2);
   p.Drow = cv.take(BH * N * 4);
   p.lam = cv.take(BH * N * 4);
-  const size_t SW = BH * (size_t)p.nq_max * p.nw_max;
-  p.PB = cv.take(SW * 2);
-  p.DSB = cv.take(SW * 2);
   p.GB = cv.take(BH * p.nq_max * F * 4);
   p.phis = cv.take(BH * p.nq_max * F * 2);
   p.dphiq = cv.take(BH * N * F * 4);
@@ -826,38 +824,35 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
 
   const float sl2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   const float isd = (float)(1.0 / std::sqrt((double)d.D));
+  CUtensorMap mq, mk, mv, mo;
+  RH_TRY(make_map(&mq, q, d.D, N, BH));
+  RH_TRY(make_map(&mk, k, d.D, N, BH));
+  RH_TRY(make_map(&mv, v, d.D, N, BH));
+  RH_TRY(make_map(&mo, dout, d.D, N, BH));
   for (int c = 0; c < C; ++c) {
     const int s = c * Tc, e = (s + Tc < T ? s + Tc : T), w = (s - To > 0 ? s - To : 0);
     const long long nq = (long long)(e - s) * L, nw = (long long)(e - w) * L;
     const long long r0 = (long long)s * L, k0 = (long long)w * L;
-    // P and dS of the chunk's (query, window key) pairs, from S = Q_c K_w^T and dP = dO_c V_w^T
+    // the softmax window's gradients, scores recomputed in TMEM: dK, dV per key tile, dQ per
+    // query tile
     {
-      CUtensorMap mq, mk, mdo, mv;
-      RH_TRY(make_map_strided(&mq, qb + r0 * D, D, nq, BH, D, N * D, 64, 128));
-      RH_TRY(make_map_strided(&mk, kb + k0 * D, D, nw, BH, D, N * D, 64, 128));
-      RH_TRY(make_map_strided(&mdo, dob + r0 * D, D, nq, BH, D, N * D, 64, 128));
-      RH_TRY(make_map_strided(&mv, vb + k0 * D, D, nw, BH, D, N * D, 64, 128));
-      rehyat::bwd::ScoreParams sp{};
-      sp.nq = (int)nq; sp.nw = (int)nw; sp.stat_rows = N; sp.stat_row0 = r0;
-      sp.lse2 = lse; sp.Drow = f32(pl.Drow); sp.scale_log2 = sl2; sp.inv_sqrt_d = isd;
-      sp.P = b16(pl.PB); sp.dS = b16(pl.DSB);
-      auto kern = rehyat::bwd::score_grad_kernel;
-      RH_TRY(cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)rehyat::bwd::kScoreSmem), "score attr"));
-      kern<<<dim3((unsigned)((nw + 127) / 128), (unsigned)((nq + 127) / 128), BH),
-             rehyat::bwd::kScoreThreads, rehyat::bwd::kScoreSmem, st>>>(mq, mk, mdo, mv, sp);
-      RH_TRY(cuda_check(cudaGetLastError(), "score gradient launch"));
+      rehyat::attn_bwd::Params bp{};
+      bp.L = L; bp.T = T; bp.Tc = Tc; bp.To = To; bp.c = c; bp.N = (int)N;
+      bp.lse2 = lse; bp.Drow = f32(pl.Drow); bp.scale_log2 = sl2; bp.inv_sqrt_d = isd;
+      bp.dq = dq; bp.dk = dk; bp.dv = dv;
+      auto kkv = rehyat::attn_bwd::dkdv_kernel;
+      auto kq = rehyat::attn_bwd::dq_kernel;
+      RH_TRY(cuda_check(cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)rehyat::attn_bwd::kKSmem), "dkdv attr"));
+      RH_TRY(cuda_check(cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)rehyat::attn_bwd::kQSmem), "dq attr"));
+      kkv<<<dim3((unsigned)((nw + 127) / 128), 1, BH), rehyat::attn_bwd::kThreads,
+            rehyat::attn_bwd::kKSmem, st>>>(mq, mk, mv, mo, bp);
+      RH_TRY(cuda_check(cudaGetLastError(), "dkdv launch"));
+      kq<<<dim3((unsigned)((nq + 127) / 128), 1, BH), rehyat::attn_bwd::kThreads,
+           rehyat::attn_bwd::kQSmem, st>>>(mq, mk, mv, mo, bp);
+      RH_TRY(cuda_check(cudaGetLastError(), "dq launch"));
     }
-    // dq_c += dS K_w;  dk_w += dS^T Q_c;  dv_w += P^T dO_c
-    RH_TRY(launch_gemm((int)nq, (int)D, (int)nw, BH, Operand{b16(pl.DSB), nw, nq * nw, false},
-                       Operand{kb + k0 * D, D, N * D, true}, dq + r0 * D, D, N * D, false, true,
-                       1.f, st));
-    RH_TRY(launch_gemm((int)nw, (int)D, (int)nq, BH, Operand{b16(pl.DSB), nw, nq * nw, true},
-                       Operand{qb + r0 * D, D, N * D, true}, dk + k0 * D, D, N * D, false, true,
-                       1.f, st));
-    RH_TRY(launch_gemm((int)nw, (int)D, (int)nq, BH, Operand{b16(pl.PB), nw, nq * nw, true},
-                       Operand{dob + r0 * D, D, N * D, true}, dv + k0 * D, D, N * D, false, true,
-                       1.f, st));
     if (w > 0) {
       // G = dO_c S_c^T; dphi_q = lam (G - D Z_c); R_c = (lam phi_q)^T dO_c; r_c partials
       RH_TRY(launch_gemm((int)nq, (int)F, (int)D, BH, Operand{dob + r0 * D, D, N * D, false},
