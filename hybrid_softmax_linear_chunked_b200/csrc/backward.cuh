@@ -65,16 +65,17 @@ __global__ void phiq_grad_kernel(const float* __restrict__ G, int nq, int F, lon
       __float2bfloat16_rn(lm * __bfloat162float(phiq[srow * F + f]));
 }
 
-// Partial sums of r_c = sum_i lam_i D_i phi_q_i over blocks of 256 rows of one chunk:
+// Partial sums of r_c = sum_i lam_i D_i phi_q_i over blocks of kRBlock rows of one chunk:
 // rpart [BH][nblk][F].  grid (nblk, BH), block F.
+constexpr int kRBlock = 64;
 __global__ void rpart_kernel(int nq, int F, long long N, long long row0,
                              const float* __restrict__ lam, const float* __restrict__ Drow,
                              const __nv_bfloat16* __restrict__ phiq, float* __restrict__ rpart,
                              int nblk) {
   const int blk = blockIdx.x, bh = blockIdx.y, f = threadIdx.x;
   float acc = 0.f;
-  const int i1 = min(nq, (blk + 1) * 256);
-  for (int i = blk * 256; i < i1; ++i) {
+  const int i1 = min(nq, (blk + 1) * kRBlock);
+  for (int i = blk * kRBlock; i < i1; ++i) {
     const long long srow = (long long)bh * N + row0 + i;
     acc = fmaf(lam[srow] * Drow[srow], __bfloat162float(phiq[srow * F + f]), acc);
   }
@@ -132,11 +133,11 @@ __global__ void feat_grad_kernel(const float* __restrict__ U, const float* __res
   }
   float fp;
   if (P == 0) {
-    fp = u > 0.f ? 1.f : expf(u);
+    fp = u > 0.f ? 1.f : __expf(u);
   } else {
     const int p = part_power(f, F, P);
-    const float sp = softplus_accurate(u);
-    const float sig = 1.f / (1.f + expf(-u));
+    const float sp = softplus_fast(u);
+    const float sig = __fdividef(1.f, 1.f + __expf(-u));
     fp = (float)p * int_pow(sp, p - 1 > 0 ? p - 1 : 1) * sig;
     if (p == 1) fp = sig;
   }

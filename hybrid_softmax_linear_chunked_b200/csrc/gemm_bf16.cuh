@@ -4,6 +4,8 @@
 // each with its operands in whichever layout the forward left them:
 //   A is M x K, stored K-contiguous ([M][K], a_mn = 0) or M-contiguous ([K][M], a_mn = 1);
 //   B is K x N, stored K-contiguous ([N][K], b_mn = 0) or N-contiguous ([K][N], b_mn = 1).
+// With split > 1 the K range is cut into `split` parts computed by separate CTAs that add their
+// partial tiles into C with fp32 atomics (C must hold the initial value; fp32 output only).
 // One CTA computes one 128 x 128 tile of C: warp 0 streams 64-deep K slices of A and B through a
 // 4-stage TMA ring (128-byte swizzle; rows, columns and K past the matrix read zeros), warp 1
 // issues four M128 N128 K16 MMAs per slice and owns the TMEM accumulator, warps 2-5 read the
@@ -35,6 +37,7 @@ struct Params {
   long long ldc, c_batch;  // elements
   int c_bf16, accumulate;
   float alpha;
+  int split;  // K parts (>= 1); blockIdx.z = batch * split + part
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -61,13 +64,17 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
   }
 }
 
-// grid (ceil(N / 128), ceil(M / 128), batch), block 192.
+// grid (ceil(N / 128), ceil(M / 128), batch * split), block 192.
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, const Params p) {
   static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
-  const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM, b = blockIdx.z;
-  const int num_k = (p.K + kBK - 1) / kBK;
+  const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
+  const int b = blockIdx.z / p.split, part = blockIdx.z - b * p.split;
+  const int k_slices = (p.K + kBK - 1) / kBK;
+  const int per_part = (k_slices + p.split - 1) / p.split;
+  const int kb0 = part * per_part;
+  const int num_k = max(0, min(k_slices, kb0 + per_part) - kb0);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ __align__(8) uint64_t bars[kNumBars];
@@ -107,8 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) {
         uint8_t* st = sm + s * kStageBytes;
         mbar_arrive_expect_tx(&bars[kFull + s], kStageBytes);
-        load_operand(st, &tmA, &bars[kFull + s], p.a_mn, m0, kb * kBK, b);
-        load_operand(st + kTileA, &tmB, &bars[kFull + s], p.b_mn, n0, kb * kBK, b);
+        load_operand(st, &tmA, &bars[kFull + s], p.a_mn, m0, (kb0 + kb) * kBK, b);
+        load_operand(st + kTileA, &tmB, &bars[kFull + s], p.b_mn, n0, (kb0 + kb) * kBK, b);
       }
       __syncwarp();
       ++issued;
@@ -157,7 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!row_ok || col0 >= p.N) continue;
         const long long base = (long long)b * p.c_batch + (long long)row * p.ldc + col0;
         const int ncol = min(32, p.N - col0);
-        if (p.c_bf16) {
+        if (p.split > 1) {
+          float* C = static_cast<float*>(p.C) + base;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < ncol) atomicAdd(C + i, __uint_as_float(r[i]) * p.alpha);
+        } else if (p.c_bf16) {
           __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + base;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {

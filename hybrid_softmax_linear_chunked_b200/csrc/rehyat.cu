@@ -154,7 +154,9 @@ struct Operand {
 // stride ldc.  Strides and bases must be 16-byte aligned (multiples of 8 elements).
 int launch_gemm(int M, int N, int K, int batch, const Operand& A, const Operand& B, void* C,
                 long long ldc, long long c_batch, bool c_bf16, bool accumulate, float alpha,
-                cudaStream_t st) {
+                cudaStream_t st, int split = 1) {
+  if (split < 1 || (split > 1 && (c_bf16 || !accumulate)))
+    return fail(REHYAT_ERR_ARG, "split-K GEMM needs fp32 output accumulated into C");
   if (M < 1 || N < 1 || K < 1 || batch < 1) return fail(REHYAT_ERR_ARG, "empty GEMM");
   if ((A.ld | A.batch_stride | B.ld | B.batch_stride) & 7)
     return fail(REHYAT_ERR_ALIGN, "GEMM operand strides must be multiples of 8 elements");
@@ -169,10 +171,11 @@ int launch_gemm(int M, int N, int K, int batch, const Operand& A, const Operand&
   gp.M = M; gp.N = N; gp.K = K; gp.a_mn = A.mn; gp.b_mn = B.mn;
   gp.C = C; gp.ldc = ldc; gp.c_batch = c_batch; gp.c_bf16 = c_bf16; gp.accumulate = accumulate;
   gp.alpha = alpha;
+  gp.split = split;
   auto k = rehyat::gemm::gemm_bf16_kernel;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)rehyat::gemm::kSmemBytes), "gemm attr"));
-  dim3 grid((N + 127) / 128, (M + 127) / 128, batch);
+  dim3 grid((N + 127) / 128, (M + 127) / 128, batch * split);
   k<<<grid, rehyat::gemm::kThreads, rehyat::gemm::kSmemBytes, st>>>(ma, mb, gp);
   return cuda_check(cudaGetLastError(), "gemm launch");
 }
@@ -501,7 +504,7 @@ BackwardPlan plan_backward(const rehyat_dims& d, int T, int L, int Tc, int To) {
   p.c_lin = To / Tc + 1;  // first chunk with a linear region
   p.nq_max = (Tc < T ? Tc : T) * L;
   p.nw_max = ((Tc + To) < T ? (Tc + To) : T) * L;
-  p.nblk_r = (p.nq_max + 255) / 256;
+  p.nblk_r = (p.nq_max + rehyat::bwd::kRBlock - 1) / rehyat::bwd::kRBlock;
   p.nblk_b = (int)((N + 255) / 256);
   Carve cv;
   p.fwd_off = cv.take(p.fwd.total);
@@ -560,7 +563,7 @@ int feature_backward(const rehyat_dims& d, long long N, long long r0, long long 
     // dWbd += du^T x over this batch's rows
     RH_TRY(launch_gemm((int)F, (int)D, (int)rows, H, Operand{DU + (bo + r0) * F, F, N * F, true},
                        Operand{xb + (bo + r0) * D, D, N * D, true}, dWbd, D, F * D, false, true,
-                       1.f, st));
+                       1.f, st, 16));
   }
   rehyat::bwd::blockdiag_grad_kernel<<<dim3((unsigned)((F * (D / d.G) + 255) / 256), H), 256, 0,
                                        st>>>(dWbd, d.D, d.F, d.G, dW);
@@ -864,9 +867,9 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
       RH_TRY(cuda_check(cudaGetLastError(), "phi_q gradient launch"));
       RH_TRY(launch_gemm((int)F, (int)D, (int)nq, BH, Operand{b16(pl.phis), F, nq * F, true},
                          Operand{dob + r0 * D, D, N * D, true},
-                         f32(pl.RB) + (long long)c * F * D, D, (long long)C * F * D, false, false,
-                         1.f, st));
-      const int nblk = (int)((nq + 255) / 256);
+                         f32(pl.RB) + (long long)c * F * D, D, (long long)C * F * D, false, true,
+                         1.f, st, 8));
+      const int nblk = (int)((nq + rehyat::bwd::kRBlock - 1) / rehyat::bwd::kRBlock);
       rehyat::bwd::rpart_kernel<<<dim3(nblk, BH), d.F, 0, st>>>(
           (int)nq, d.F, N, r0, f32(pl.lam), f32(pl.Drow), phiq,
           f32(pl.rpart) + (long long)c * BH * pl.nblk_r * F, pl.nblk_r);
