@@ -195,7 +195,8 @@ struct Carve {
 int fold_splits(int BH, int n_fold, long long rows_per_fold) {
   if (n_fold <= 0) return 1;
   const long long tiles = (rows_per_fold + 127) / 128;
-  long long want = (2LL * 148 + (long long)BH * n_fold - 1) / ((long long)BH * n_fold);
+  // one wave of the one-CTA-per-SM fold kernel: long loops amortise each CTA's set-up
+  long long want = 148LL / ((long long)BH * n_fold);
   long long s = want < 1 ? 1 : want;
   const long long max_s = tiles / 2 > 0 ? tiles / 2 : 1;
   if (s > max_s) s = max_s;
@@ -346,7 +347,9 @@ int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int 
   CUtensorMap mx;
   RH_TRY(make_map(&mx, x, d.D, rows_per_bh, BH));
   const int n_tiles = (n_rows + 127) / 128;
-  int per_cta = (int)(((long long)n_tiles * BH + 2 * 148 - 1) / (2 * 148));
+  // one wave (one CTA per SM): as many CTAs per (b, h) as fit in 148
+  const int ctas_per_bh = BH < 148 ? 148 / BH : 1;
+  int per_cta = (n_tiles + ctas_per_bh - 1) / ctas_per_bh;
   if (per_cta < 1) per_cta = 1;
   if (per_cta > n_tiles) per_cta = n_tiles;
   rehyat::phi::Params pp{};
