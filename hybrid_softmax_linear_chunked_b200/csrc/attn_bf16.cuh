@@ -143,7 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
 
   // ---- chunk geometry (uniform over the CTA) ----
-  const int c = blockIdx.y, bh = blockIdx.z, h = bh % p.H;
+  // grid (tile pairs, BH, chunks): chunk 0, whose window is shortest, is dispatched last
+  const int bh = blockIdx.y, c = (blockIdx.z + 1) % gridDim.z, h = bh % p.H;
   const int gs = p.frames_before + c * p.Tc;
   const int ge = min(gs + p.Tc, p.frames_before + p.T);
   const int gw = max(0, gs - p.To);

@@ -703,7 +703,7 @@ static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int
     ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
     ap.out = static_cast<__nv_bfloat16*>(out);
     ap.lse = lse;
-    dim3 grid((rows_per_chunk + 255) / 256, pl.C, BH);
+    dim3 grid((rows_per_chunk + 255) / 256, BH, pl.C);
     return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, grid, st);
   }
   rehyat::fp32::AttnParams ap{};
@@ -989,7 +989,7 @@ int rehyat_chunk_forward_sched(rehyat_dims d, rehyat_dtype dt, int L, int frames
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
     ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
     RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
-                                  dim3((pl.nq + 255) / 256, 1, BH), st));
+                                  dim3((pl.nq + 255) / 256, BH, 1), st));
     if (pl.fold_rows > 0) {
       RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
       rehyat::state::FoldParams fp{};
@@ -1156,7 +1156,7 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
-  RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3((pl.nq + 255) / 256, 1, nbh),
+  RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3((pl.nq + 255) / 256, nbh, 1),
                                  st));
   if (pl.fold_rows > 0) {
     RH_TRY(prepare_blockdiag(d, Wk, Wkbd, &mwk, st));
