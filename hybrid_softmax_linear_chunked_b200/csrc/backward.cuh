@@ -82,14 +82,23 @@ __global__ void rpart_kernel(int nq, int F, long long N, long long row0,
   rpart[((long long)bh * nblk + blk) * F + f] = acc;
 }
 
+// r_c = the sum of its rpart blocks ([C][BH][nblk][F], zeros for chunks without a linear
+// region), into r [BH][C][F].  grid (C, BH), block F.
+__global__ void rreduce_kernel(const float* __restrict__ rpart, int nblk, int F,
+                               float* __restrict__ r) {
+  const int c = blockIdx.x, bh = blockIdx.y, BH = gridDim.y, C = gridDim.x, f = threadIdx.x;
+  float acc = 0.f;
+  for (int b = 0; b < nblk; ++b) acc += rpart[(((long long)c * BH + bh) * nblk + b) * F + f];
+  r[((long long)bh * C + c) * F + f] = acc;
+}
+
 // Suffix sums over chunks: Rt_c = sum_{c' >= c} R_c' (bf16 [BH][C][F][D], R fp32, chunks
-// without a linear region hold zeros) and rt_c = sum_{c' >= c} r_c' (fp32 [BH][C][F]) with
-// r_c = sum of its rpart blocks ([C][BH][nblk][F], zeros for chunks without a linear region).
+// without a linear region hold zeros) and rt_c = sum_{c' >= c} r_c' (fp32 [BH][C][F], in place
+// over r).
 //   grid (ceil(F*D / 256), BH), block 256.
-__global__ void suffix_kernel(const float* __restrict__ R, const float* __restrict__ rpart, int C,
-                              int nblk, int F, int D, __nv_bfloat16* __restrict__ Rt,
-                              float* __restrict__ rt) {
-  const int bh = blockIdx.y, BH = gridDim.y;
+__global__ void suffix_kernel(const float* __restrict__ R, int C, int F, int D,
+                              __nv_bfloat16* __restrict__ Rt, float* __restrict__ rt) {
+  const int bh = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const long long FD = (long long)F * D;
   if (e < FD) {
@@ -100,13 +109,11 @@ __global__ void suffix_kernel(const float* __restrict__ R, const float* __restri
       Rt[o] = __float2bfloat16_rn(acc);
     }
   }
-  if (e < F) {
+  if (blockIdx.x == 0 && threadIdx.x < F) {
     float acc = 0.f;
     for (int c = C - 1; c >= 0; --c) {
-      float rc = 0.f;
-      for (int b = 0; b < nblk; ++b) rc += rpart[(((long long)c * BH + bh) * nblk + b) * F + e];
-      acc += rc;
-      rt[((long long)bh * C + c) * F + e] = acc;
+      acc += rt[((long long)bh * C + c) * F + threadIdx.x];
+      rt[((long long)bh * C + c) * F + threadIdx.x] = acc;
     }
   }
 }
@@ -116,32 +123,36 @@ __global__ void suffix_kernel(const float* __restrict__ R, const float* __restri
 // subtracted with chunk index cidx(row) = (frame + To) / Tc + 1 (the first chunk that reads the
 // key linearly).  f' of the polynomial map on part p: p softplus^(p-1) sigmoid; of elu + 1:
 // 1 (u > 0) or e^u (P = 0).  du in bf16 [BH][N][F] for the products that follow.
-//   grid (row1 - row0, BH), block F.
+//   grid (ceil((row1 - row0) / kFeatRows), BH), block F; each block takes kFeatRows rows.
+constexpr int kFeatRows = 16;
 __global__ void feat_grad_kernel(const float* __restrict__ U, const float* __restrict__ bias,
                                  int H, const float* __restrict__ g,
                                  const float* __restrict__ rsub, int C, int L, int Tc, int To,
-                                 int F, int P, long long N, long long row0,
+                                 int F, int P, long long N, long long row0, long long row1,
                                  __nv_bfloat16* __restrict__ du) {
-  const long long row = row0 + blockIdx.x;
   const int bh = blockIdx.y, f = threadIdx.x, h = bh % H;
-  const long long o = ((long long)bh * N + row) * F + f;
-  const float u = U[o] + (bias ? bias[(long long)h * F + f] : 0.f);
-  float gv = g[o];
-  if (rsub) {
-    const int c = (int)((row / L + To) / Tc) + 1;
-    gv -= rsub[((long long)bh * C + c) * F + f];
+  const float b = bias ? bias[(long long)h * F + f] : 0.f;
+  const int p = P == 0 ? 0 : part_power(f, F, P);  // this thread's feature: one power
+  const long long r0 = row0 + (long long)blockIdx.x * kFeatRows;
+  const long long r1 = min(row1, r0 + kFeatRows);
+  for (long long row = r0; row < r1; ++row) {
+    const long long o = ((long long)bh * N + row) * F + f;
+    const float u = U[o] + b;
+    float gv = g[o];
+    if (rsub) {
+      const int c = (int)((row / L + To) / Tc) + 1;
+      gv -= rsub[((long long)bh * C + c) * F + f];
+    }
+    float fp;
+    if (p == 0) {
+      fp = u > 0.f ? 1.f : __expf(u);
+    } else {
+      const float sig = __fdividef(1.f, 1.f + __expf(-u));
+      fp = sig;
+      if (p > 1) fp = (float)p * int_pow(softplus_fast(u), p - 1) * sig;
+    }
+    du[o] = __float2bfloat16_rn(gv * fp);
   }
-  float fp;
-  if (P == 0) {
-    fp = u > 0.f ? 1.f : __expf(u);
-  } else {
-    const int p = part_power(f, F, P);
-    const float sp = softplus_fast(u);
-    const float sig = __fdividef(1.f, 1.f + __expf(-u));
-    fp = (float)p * int_pow(sp, p - 1 > 0 ? p - 1 : 1) * sig;
-    if (p == 1) fp = sig;
-  }
-  du[o] = __float2bfloat16_rn(gv * fp);
 }
 
 // Column sums of du (bf16 [BH][N][F]) over blocks of 256 rows of [row0, row1):

@@ -552,8 +552,9 @@ int feature_backward(const rehyat_dims& d, long long N, long long r0, long long 
                          Operand{Wbd + part * F * D, D, 2 * F * D, false},
                          U + (bo + r0) * F, F, N * F, false, part > 0, 1.f, st));
   }
-  rehyat::bwd::feat_grad_kernel<<<dim3((unsigned)rows, BH), d.F, 0, st>>>(
-      U, bias, H, g, rsub, C, L, Tc, To, d.F, kernel_P(d), N, r0, DU);
+  rehyat::bwd::feat_grad_kernel<<<
+      dim3((unsigned)((rows + rehyat::bwd::kFeatRows - 1) / rehyat::bwd::kFeatRows), BH), d.F, 0,
+      st>>>(U, bias, H, g, rsub, C, L, Tc, To, d.F, kernel_P(d), N, r0, r1, DU);
   RH_TRY(cuda_check(cudaGetLastError(), "feature gradient launch"));
   RH_TRY(cuda_check(cudaMemsetAsync(dWbd, 0, (size_t)H * F * D * 4, st), "memset"));
   for (int b = 0; b < d.B; ++b) {
@@ -880,8 +881,11 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
     }
   }
   if (wl > 0) {
+    rehyat::bwd::rreduce_kernel<<<dim3(C, BH), d.F, 0, st>>>(f32(pl.rpart), pl.nblk_r, d.F,
+                                                             f32(pl.rt));
+    RH_TRY(cuda_check(cudaGetLastError(), "r reduce launch"));
     rehyat::bwd::suffix_kernel<<<dim3((unsigned)((F * D + 255) / 256), BH), 256, 0, st>>>(
-        f32(pl.RB), f32(pl.rpart), C, pl.nblk_r, d.F, d.D, b16(pl.Rt), f32(pl.rt));
+        f32(pl.RB), C, d.F, d.D, b16(pl.Rt), f32(pl.rt));
     RH_TRY(cuda_check(cudaGetLastError(), "suffix launch"));
     // keys folded after chunk c (frames [w_c, w_{c+1})) are read linearly from chunk c + 1 on
     for (int c = 0; c + 1 < C; ++c) {

@@ -331,6 +331,17 @@ __global__ void __launch_bounds__(256) state_scan_kernel(
   }
   if (z_thread) accz = Z0 ? Z0[(size_t)bh * F + f0 + tx] : 0.f;
   for (int c = 0; c < C; ++c) {
+    // this chunk's fold partials are loaded first, so their latency overlaps the stores below
+    float add[4] = {0.f, 0.f, 0.f, 0.f};
+    float addz = 0.f;
+    if (c < n_fold) {
+      for (int s = 0; s < splits; ++s) {
+        const size_t base = (((size_t)bh * n_fold + c) * splits + s);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) add[i] += dS[(base * F + f0 + ty + 8 * i) * D + d0 + tx];
+        if (z_thread) addz += dZ[base * F + f0 + tx];
+      }
+    }
     if (St) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) tile[ty + 8 * i][tx] = acc[i];
@@ -351,14 +362,9 @@ __global__ void __launch_bounds__(256) state_scan_kernel(
       if (Zc) Zc[((size_t)bh * C + c) * F + f0 + tx] = accz;
       if (Z_out) Z_out[((size_t)bh * C + c) * F + f0 + tx] = accz;
     }
-    if (c < n_fold) {
-      for (int s = 0; s < splits; ++s) {
-        const size_t base = (((size_t)bh * n_fold + c) * splits + s);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] += dS[(base * F + f0 + ty + 8 * i) * D + d0 + tx];
-        if (z_thread) accz += dZ[base * F + f0 + tx];
-      }
-    }
+    for (int i = 0; i < 4; ++i) acc[i] += add[i];
+    accz += addz;
   }
 }
 
