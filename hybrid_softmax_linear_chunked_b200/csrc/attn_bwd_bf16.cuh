@@ -9,12 +9,16 @@
 // The derivative is that of the "ReHyAt overview" page's §2.2.1 output formula; the linear
 // terms' gradients are separate (backward.cuh and tensor-core products).
 //
-// Both kernels: 192 threads.  Warps 0-3 compute (one TMEM lane = one row per thread), warp 4
-// loads by TMA (and allocates TMEM), warp 5 issues the MMAs.  Per loop step the MMA warp issues
-// the two score products (S and dP, SS), the compute warps turn them into packed bf16 P / dS
-// written back over the scores in TMEM, and the MMA warp issues the products that use them as
-// the A operand (TS).  Launch once per chunk (keys of the overlap frames belong to two chunks'
-// windows; the launches' += on dK, dV are ordered by the stream).
+// Both kernels: 320 threads.  Warps 0-7 compute: warp w owns TMEM lanes 32 (w % 4) .. + 31 (one
+// row per thread) and the column half w / 4 (64 of the 128 score columns), so two warps share
+// each SM sub-partition's work; warp 8 loads by TMA (and allocates TMEM), warp 9 issues the MMAs.
+// Per loop step the MMA warp issues the two score products (S and dP, SS), the compute warps turn
+// them into packed bf16 P / dS written back over the scores in TMEM (half h's 64 columns pack into
+// TMEM columns [64 h, 64 h + 32), inside its own half, so the two halves never touch each other's
+// scores), and the MMA warp issues the products that use them as the A operand (TS), whose K16
+// step kk reads packed column 64 (kk / 4) + 8 (kk % 4).  Launch once per chunk (keys of the
+// overlap frames belong to two chunks' windows; the launches' += on dK, dV are ordered by the
+// stream).
 #pragma once
 
 #include "attn_bf16.cuh"
@@ -24,10 +28,37 @@ namespace rehyat {
 namespace attn_bwd {
 
 using namespace sm100;
+using attn::f2_add;
+using attn::f2_fma;
+using attn::f2_mul;
+using attn::f2_pack;
+using attn::f2_unpack;
 using attn::kmajor_desc;
 using attn::mnmajor_desc;
 
-constexpr int kThreads = 192;
+// Two probabilities and two dS values from two (score, dP) pairs, on paired fp32 instructions:
+// p = 2^(s scale - lse2), g = (p / sqrt(D)) (dP - D).  neg_l2 and neg_d hold -lse2 and -D.
+__device__ __forceinline__ void grad_pair(uint32_t s0, uint32_t s1, uint32_t d0, uint32_t d1,
+                                          uint64_t sl2x2, uint64_t neg_l2, uint64_t neg_d,
+                                          uint64_t isd2, uint32_t& pp, uint32_t& gg) {
+  const uint64_t x = f2_fma(f2_pack(__uint_as_float(s0), __uint_as_float(s1)), sl2x2, neg_l2);
+  float xa, xb;
+  f2_unpack(x, xa, xb);
+  const uint64_t pr = f2_pack(attn::ex2(xa), attn::ex2(xb));
+  const uint64_t t = f2_add(f2_pack(__uint_as_float(d0), __uint_as_float(d1)), neg_d);
+  const uint64_t g = f2_mul(f2_mul(pr, isd2), t);
+  float pa, pb, ga, gb;
+  f2_unpack(pr, pa, pb);
+  f2_unpack(g, ga, gb);
+  pp = pack_bf16x2(pa, pb);
+  gg = pack_bf16x2(ga, gb);
+}
+
+constexpr int kThreads = 320;
+constexpr int kCompute = 256;  // compute threads (warps 0-7)
+
+// TMEM column of the packed bf16 A operand for the K16 step kk (see above).
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 bf16 tile (two 128 x 64 boxes)
 constexpr uint32_t kStatBytes = 2 * 128 * 4;
 
@@ -105,12 +136,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_sh;
   volatile int* abort_flag = &abort_sh;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < kKBars; ++i) mbar_init(&bars[i], i == kPdFull ? 128 : 1);
+    for (int i = 0; i < kKBars; ++i) mbar_init(&bars[i], i == kPdFull ? kCompute : 1);
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -120,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = tmem_base_sh;
   float* sStat = reinterpret_cast<float*>(sm + kKOffStat);  // [stage][lse 128 | D 128]
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---- producer ----
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -143,8 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qi = i * 128 + lane * 4 + t;
         const bool valid = qi < g.nq;
         const long long idx = (long long)bh * p.N + g.q_row0 + (valid ? qi : 0);
-        st[lane * 4 + t] = valid ? p.lse2[idx] : INFINITY;
-        st[128 + lane * 4 + t] = valid ? p.Drow[idx] : 0.f;
+        st[lane * 4 + t] = valid ? -p.lse2[idx] : -INFINITY;  // negated for the FMA
+        st[128 + lane * 4 + t] = valid ? -p.Drow[idx] : 0.f;
       }
       __syncwarp();
       if (lane == 0) {
@@ -161,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(&bars[kQFull + (i & 1)], (i >> 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---- MMA issuer ----
     const uint32_t id_ss = idesc_bf16(128, 128, false, false);
     const uint32_t id_ts = idesc_bf16(128, 128, false, true);
@@ -189,9 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (lane == 0) {
         for (int kk = 0; kk < 8; ++kk)  // dV += P^T dO
-          mma_ts(tmem + 256, tmem + kk * 8, mnmajor_desc(sO, kk), id_ts, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + 256, tmem + packed_col(kk), mnmajor_desc(sO, kk), id_ts,
+                 (i > 0 || kk > 0) ? 1u : 0u);
         for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
-          mma_ts(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(sQ, kk), id_ts,
+          mma_ts(tmem + 384, tmem + 128 + packed_col(kk), mnmajor_desc(sQ, kk), id_ts,
                  (i > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars[kQEmpty + s]);
       }
@@ -202,37 +234,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait_drain(&bars[kKDone], 0);
     __syncwarp();
   } else {
-    // ---- compute: thread = key row r of the tile ----
-    const int r = tid;  // 0..127, TMEM lane
+    // ---- compute: thread = key row r of the tile, column half hc ----
+    const int r = tid & 127, hc = tid >> 7;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base, tD = tmem + lane_base + 128;
-    const float sl2 = p.scale_log2, isd = p.inv_sqrt_d;
+    const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
+    const uint64_t isd2 = f2_pack(p.inv_sqrt_d, p.inv_sqrt_d);
     bool ok = true;
     for (int i = 0; i < n_q; ++i) {
       const int s = i & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSdFull], i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const float* lse = sStat + s * 256;
-      const float* Dq = lse + 128;
+      // -lse2 and -D of the tile's 128 queries, read four at a time (same address in every lane)
+      const float4* nl4 = reinterpret_cast<const float4*>(sStat + s * 256);
+      const float4* nd4 = nl4 + 32;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = hc * 2 + cc;  // 32-column chunk of the scores
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + c * 32, sv);
         tmem_ld32(tD + c * 32, dv);
         uint32_t pp[16], gg[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int q0 = c * 32 + 2 * e;
-          const float p0 = attn::ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -lse[q0]));
-          const float p1 = attn::ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -lse[q0 + 1]));
-          pp[e] = pack_bf16x2(p0, p1);
-          gg[e] = pack_bf16x2(p0 * (__uint_as_float(dv[2 * e]) - Dq[q0]) * isd,
-                              p1 * (__uint_as_float(dv[2 * e + 1]) - Dq[q0 + 1]) * isd);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 nl = nl4[c * 8 + e4], nd = nd4[c * 8 + e4];
+          grad_pair(sv[4 * e4], sv[4 * e4 + 1], dv[4 * e4], dv[4 * e4 + 1], sl2x2,
+                    f2_pack(nl.x, nl.y), f2_pack(nd.x, nd.y), isd2, pp[2 * e4], gg[2 * e4]);
+          grad_pair(sv[4 * e4 + 2], sv[4 * e4 + 3], dv[4 * e4 + 2], dv[4 * e4 + 3], sl2x2,
+                    f2_pack(nl.z, nl.w), f2_pack(nd.z, nd.w), isd2, pp[2 * e4 + 1],
+                    gg[2 * e4 + 1]);
         }
-        // packed columns [16c, 16c + 16) hold scores already read (chunks c / 2 and c)
-        tmem_st16(tS + c * 16, pp);
-        tmem_st16(tD + c * 16, gg);
+        // packed columns [64 hc + 16 cc, + 16): this half's first chunk, already read
+        tmem_st16(tS + hc * 64 + cc * 16, pp);
+        tmem_st16(tD + hc * 64 + cc * 16, gg);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -244,7 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = key0 + r < g.nw;
       const long long row = (long long)bh * p.N + g.k_row0 + key0 + r;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int cc = hc * 2 + c2;
         uint32_t a[32], b[32];
         tmem_ld32(tmem + lane_base + 256 + cc * 32, a);
         tmem_ld32(tmem + lane_base + 384 + cc * 32, b);
@@ -257,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -290,12 +326,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_sh;
   volatile int* abort_flag = &abort_sh;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < kQBars; ++i) mbar_init(&bars[i], i == kDsFull ? 128 : 1);
+    for (int i = 0; i < kQBars; ++i) mbar_init(&bars[i], i == kDsFull ? kCompute : 1);
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -304,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---- producer ----
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
@@ -334,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(&bars[kKFull + (j & 1)], (j >> 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---- MMA issuer ----
     const uint32_t id_ss = idesc_bf16(128, 128, false, false);
     const uint32_t id_ts = idesc_bf16(128, 128, false, true);
@@ -362,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (lane == 0) {
         for (int kk = 0; kk < 8; ++kk)  // dQ += dS K
-          mma_ts(tmem + 256, tmem + 128 + kk * 8, mnmajor_desc(sK, kk), id_ts,
+          mma_ts(tmem + 256, tmem + 128 + packed_col(kk), mnmajor_desc(sK, kk), id_ts,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars[kKEmpty + s]);
       }
@@ -373,15 +409,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait_drain(&bars[kQDone], 0);
     __syncwarp();
   } else {
-    // ---- compute: thread = query row r of the tile ----
-    const int r = tid;
+    // ---- compute: thread = query row r of the tile, column half hc ----
+    const int r = tid & 127, hc = tid >> 7;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base, tD = tmem + lane_base + 128;
-    const float sl2 = p.scale_log2, isd = p.inv_sqrt_d;
     const bool row_ok = q0 + r < g.nq;
     const long long row = (long long)bh * p.N + g.q_row0 + q0 + r;
     const float l2 = row_ok ? p.lse2[row] : INFINITY;
     const float Di = row_ok ? p.Drow[row] : 0.f;
+    const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
+    const uint64_t isd2 = f2_pack(p.inv_sqrt_d, p.inv_sqrt_d);
+    const uint64_t neg_l2 = f2_pack(-l2, -l2), neg_d = f2_pack(-Di, -Di);
     bool ok = true;
     for (int j = 0; j < n_k; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], j & 1, abort_flag));
@@ -389,22 +427,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int valid = g.nw - j * 128;  // key columns of this tile inside the window
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = hc * 2 + cc;
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + c * 32, sv);
         tmem_ld32(tD + c * 32, dv);
-        uint32_t gg[16];
+        uint32_t gg[16], pp;
+        if (valid < 128) {  // the window's last key tile: keys past the window get dS = 0
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int k0 = c * 32 + 2 * e;
-          float p0 = attn::ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -l2));
-          float p1 = attn::ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -l2));
-          p0 = k0 < valid ? p0 : 0.f;
-          p1 = k0 + 1 < valid ? p1 : 0.f;
-          gg[e] = pack_bf16x2(p0 * (__uint_as_float(dv[2 * e]) - Di) * isd,
-                              p1 * (__uint_as_float(dv[2 * e + 1]) - Di) * isd);
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e >= valid) sv[e] = __float_as_uint(-INFINITY);
         }
-        tmem_st16(tD + c * 16, gg);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          grad_pair(sv[2 * e], sv[2 * e + 1], dv[2 * e], dv[2 * e + 1], sl2x2, neg_l2, neg_d,
+                    isd2, pp, gg[e]);
+        tmem_st16(tD + hc * 64 + cc * 16, gg);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -414,7 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int cc = hc * 2 + c2;
         uint32_t a[32];
         tmem_ld32(tmem + lane_base + 256 + cc * 32, a);
         if (row_ok) add_row32(p.dq + row * 128 + cc * 32, a);
@@ -423,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
