@@ -330,6 +330,34 @@ def test_full_size_streaming_20s(dev):
     check_sampled(out, inp, w, rows, [(0, 0), (1, 7), (1, 11)])
 
 
+def test_full_size_streaming_session_20s(dev):
+    """The same workload through the streaming session (the library assembles each window from
+    the carried frames): sampled rows against the oracle, constant device memory, and the same
+    outputs as the window-slicing loop above up to accumulation order."""
+    from hybrid_softmax_linear_chunked_b200.streaming import ChunkStream
+    w = C.WAN_480P_20S_STREAM
+    inp = make_inputs(w)
+    q, k, v, Wq, bq, Wk, bk = to_dev(inp, dev)
+    L = w.frame_tokens
+    sess = ChunkStream(Wq, bq, Wk, bk, B=w.B, P=w.P, frame_tokens=L, Tc=w.Tc, To=w.To)
+    bounds = w.chunk_bounds()
+    chunks = [[x[:, :, s * L:e * L].contiguous() for x in (q, k, v)] for (_, s, e) in bounds]
+    outs = [torch.full_like(c[0], float("nan")) for c in chunks]
+    torch.cuda.synchronize(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    mem = []
+    for c, (qc, kc, vc) in enumerate(chunks):
+        sess.step(qc, kc, vc, out=outs[c])
+        mem.append(torch.cuda.max_memory_allocated(dev))
+    rb.sync_status(dev)
+    out = torch.cat(outs, dim=2)
+    assert torch.isfinite(out).all()
+    assert len(set(mem)) == 1, f"peak device memory grew across chunks: {mem}"
+    rng = np.random.default_rng(2)
+    rows = sample_rows(w, 2, rng)
+    check_sampled(out, inp, w, rows, [(0, 3), (1, 5)])
+
+
 @pytest.mark.parametrize("Tc,To,P", [(1, 0, 1), (1, 1, 2), (3, 0, 2), (3, 1, 3), (5, 1, 2),
                                      (5, 0, 1), (3, 2, 2)])
 def test_ablation_shapes_sampled(dev, Tc, To, P):
