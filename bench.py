@@ -485,10 +485,11 @@ def backward_runner(w: C.Workload, inp, dev, args) -> _Run:
     C_ = w.n_chunks
     lin = sum(1 for (wf, _, _) in w.chunk_bounds() if wf > 0)
     groups = sum(1 for c in range(C_ - 1) if w.chunk_bounds()[c + 1][0] > w.chunk_bounds()[c][0])
-    # phi_k, row stats, per chunk 2 GEMM + softmax-grad + 3 GEMM (+ linear: GEMM, phi_q grad,
-    # GEMM, r partials), suffix, per fold group 2 GEMM, two feature backwards (per batch 5 GEMM,
-    # feature grad, block-diagonal grad, column sums, bias grad), plus the forward states/phi_q
-    r.launches_per_step = (2 + 6 * C_ + 4 * lin + 1 + 2 * groups + 2 * (5 * w.B + 4) + 6)
+    # per chunk dK/dV + dQ (+ linear: GEMM, phi_q grad, GEMM, r partials), row statistics,
+    # r reduction, suffix, per fold group 2 GEMM, two feature backwards (per batch 5 GEMM,
+    # feature grad, block-diagonal grad, column sums, bias grad), plus the recomputed
+    # states/phi_q/phi_k (2 weight preps, 2 feature maps, fold, scan)
+    r.launches_per_step = (2 * C_ + 4 * lin + 3 + 2 * groups + 2 * (5 * w.B + 4) + 6)
     r.roofline_kernel = "backward pass (all launches; algorithmic FLOPs / time)"
     r.config = {"pass": "backward"}
     return r
