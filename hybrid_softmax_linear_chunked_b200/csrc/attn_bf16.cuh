@@ -76,6 +76,11 @@ struct Params {
   int H, P;
   int n_states;       // states per (b, h) in St / Z (state index = chunk index)
   int nq_rows;        // rows per (b, h) of q and out
+  // Two-source window (streaming with carried frames): the first kv_split rows of the window come
+  // from tmKc/tmVc starting at row carry_row0, the rest from tmK/tmV; each segment is tiled on
+  // its own (its last tile ragged).  kv_split = 0: the whole window is in tmK/tmV.
+  int kv_split;
+  int carry_row0;
   float scale_log2;   // log2(e) / sqrt(D)
   const float* bq;    // [H, F] or null
   const float* Z;     // [BH, n_states, F]
@@ -144,12 +149,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tmV,
                             const __grid_constant__ CUtensorMap tmSt,
                             const __grid_constant__ CUtensorMap tmW,
-                            const __grid_constant__ CUtensorMap tmPhi, const Params p) {
+                            const __grid_constant__ CUtensorMap tmPhi,
+                            const __grid_constant__ CUtensorMap tmKc,
+                            const __grid_constant__ CUtensorMap tmVc, const Params p) {
   static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
 
   // ---- chunk geometry (uniform over the CTA) ----
-  // grid (tile pairs, BH, chunks): chunk 0, whose window is shortest, is dispatched last
-  const int bh = blockIdx.y, c = (blockIdx.z + 1) % gridDim.z, h = bh % p.H;
+  // grid (BH, tile pairs, chunks), dispatched x fastest: within a chunk the lone last tile of an
+  // odd tile count (the shortest CTAs) come last, and chunk 0, whose window is shortest, last
+  // of all
+  const int bh = blockIdx.x, c = (blockIdx.z + 1) % gridDim.z, h = bh % p.H;
   const int gs = p.frames_before + c * p.Tc;
   const int ge = min(gs + p.Tc, p.frames_before + p.T);
   const int gw = max(0, gs - p.To);
@@ -158,10 +167,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int k_row0 = (gw - p.kv_frame0) * p.L;
   const int nk = (ge - gw) * p.L;
   const bool has_linear = gw > 0;
-  const int tile_row0 = blockIdx.x * 2 * kBM;
+  const int tile_row0 = blockIdx.y * 2 * kBM;
   if (tile_row0 >= nq) return;
   const bool has_t1 = tile_row0 + kBM < nq;
-  const int n_kv = (nk + kBN - 1) / kBN;
+  // key tiles: n_kc from the carried segment (rows [0, kv_split) of the window), then the rest
+  const int kv_split = p.kv_split;
+  const int n_kc = (kv_split + kBN - 1) / kBN;
+  const int n_kv = n_kc + (nk - kv_split + kBN - 1) / kBN;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -223,16 +235,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued_k = 0, issued_v = 0;
     bool st_issued = false;
     bool ok = true;
+    if (leader && n_kc > 0) {
+      tma_prefetch_desc(&tmKc);
+      tma_prefetch_desc(&tmVc);
+    }
     for (int j = 0; j < n_kv; ++j) {
       const int s = j & 1;
-      const int row = k_row0 + j * kBN;
+      const bool carried = j < n_kc;
+      const int row = carried ? p.carry_row0 + j * kBN : k_row0 + kv_split + (j - n_kc) * kBN;
+      const CUtensorMap* mK = carried ? &tmKc : &tmK;
+      const CUtensorMap* mV = carried ? &tmVc : &tmV;
       if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty + s], ((j >> 1) - 1) & 1, abort_flag));
       if (!ok) break;
       if (leader) {
         uint8_t* dk = sm + kOffK + s * kTileBytes;
         mbar_arrive_expect_tx(&bars[kKFull + s], kTileBytes);
-        tma_load_3d(dk, &tmK, &bars[kKFull + s], 0, row, bh);
-        tma_load_3d(dk + kBM * 128, &tmK, &bars[kKFull + s], 64, row, bh);
+        tma_load_3d(dk, mK, &bars[kKFull + s], 0, row, bh);
+        tma_load_3d(dk + kBM * 128, mK, &bars[kKFull + s], 64, row, bh);
       }
       __syncwarp();
       ++issued_k;
@@ -241,8 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) {
         uint8_t* dv = sm + kOffV + s * kTileBytes;
         mbar_arrive_expect_tx(&bars[kVFull + s], kTileBytes);
-        tma_load_3d(dv, &tmV, &bars[kVFull + s], 0, row, bh);
-        tma_load_3d(dv + kBM * 128, &tmV, &bars[kVFull + s], 64, row, bh);
+        tma_load_3d(dv, mV, &bars[kVFull + s], 0, row, bh);
+        tma_load_3d(dv + kBM * 128, mV, &bars[kVFull + s], 64, row, bh);
       }
       __syncwarp();
       ++issued_v;
@@ -437,8 +456,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // The S row (128 fp32) is read once into registers; the row max is a tree over eight
         // partial maxima and the row sum uses four accumulators, so neither is one long
-        // dependency chain.  Only the window's last tile can be ragged (uniform branch).
-        const int valid = nk - j * kBN;  // key columns of this tile inside the window
+        // dependency chain.  Only a segment's last tile can be ragged (uniform branch).
+        // key columns of this tile inside its segment of the window
+        const int valid = j < n_kc ? kv_split - j * kBN : nk - kv_split - (j - n_kc) * kBN;
         uint32_t rr[kBN];
         tmem_ld128(tS, rr);
         if (valid < kBN) {

@@ -280,10 +280,11 @@ ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_be
   return p;
 }
 
-// Streaming with carried frames: the chunk step's own workspace, then the assembled K and V
-// windows and the next carry of K and V.
+// Streaming with carried frames: the chunk step's own workspace, then (fp32 only) the assembled K
+// and V windows, then the next carry of K and V (used when the chunk is shorter than the carry).
+// The bf16 kernels read the window straight from the carry and the chunk.
 struct CarryPlan {
-  size_t step, kwin, vwin, kcar, vcar, total;
+  size_t step, step_bytes, kwin, vwin, kcar, vcar, total;
 };
 
 CarryPlan plan_carry(const rehyat_dims& d, rehyat_dtype dt, int L, int chunk_frames, int To,
@@ -292,9 +293,12 @@ CarryPlan plan_carry(const rehyat_dims& d, rehyat_dtype dt, int L, int chunk_fra
   const size_t es = dt == REHYAT_BF16 ? 2 : 4;
   const size_t BH = (size_t)d.B * d.H;
   Carve cv;
-  p.step = cv.take(plan_chunk(d, dt, L, To, chunk_frames, To, To).total);
-  p.kwin = cv.take(BH * (size_t)(To + chunk_frames) * L * d.D * es);
-  p.vwin = cv.take(BH * (size_t)(To + chunk_frames) * L * d.D * es);
+  p.step_bytes = plan_chunk(d, dt, L, To, chunk_frames, To, To).total;
+  p.step = cv.take(p.step_bytes);
+  if (dt != REHYAT_BF16) {
+    p.kwin = cv.take(BH * (size_t)(To + chunk_frames) * L * d.D * es);
+    p.vwin = cv.take(BH * (size_t)(To + chunk_frames) * L * d.D * es);
+  }
   p.kcar = cv.take(BH * (size_t)cap * L * d.D * es);
   p.vcar = cv.take(BH * (size_t)cap * L * d.D * es);
   p.total = cv.off;
@@ -328,12 +332,14 @@ int launch_featmap(const rehyat_dims& d, rehyat_dtype dt, int n, const void* x, 
 template <bool kPhiGlobal>
 int launch_attn_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& ms, const CUtensorMap& mw, const CUtensorMap& mphi,
-                     const rehyat::attn::Params& ap, dim3 grid, cudaStream_t st) {
+                     const rehyat::attn::Params& ap, dim3 grid, cudaStream_t st,
+                     const CUtensorMap* mkc = nullptr, const CUtensorMap* mvc = nullptr) {
   auto k = rehyat::attn::hybrid_attn_bf16_kernel<kPhiGlobal>;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)rehyat::attn::kSmemBytes),
                     "attn attr"));
-  k<<<grid, rehyat::attn::kThreads, rehyat::attn::kSmemBytes, st>>>(mq, mk, mv, ms, mw, mphi, ap);
+  k<<<grid, rehyat::attn::kThreads, rehyat::attn::kSmemBytes, st>>>(
+      mq, mk, mv, ms, mw, mphi, mkc ? *mkc : mk, mvc ? *mvc : mv, ap);
   return cuda_check(cudaGetLastError(), "attention launch");
 }
 
@@ -365,12 +371,14 @@ int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int 
 }
 
 int launch_fold_bf16(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mw,
-                     const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st) {
+                     const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st,
+                     const CUtensorMap* mkc = nullptr, const CUtensorMap* mvc = nullptr) {
   auto k = rehyat::state::fold_partial_bf16_kernel;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)rehyat::state::kSmemBytes),
                     "fold attr"));
-  k<<<grid, rehyat::state::kThreads, rehyat::state::kSmemBytes, st>>>(mk, mv, mw, fp);
+  k<<<grid, rehyat::state::kThreads, rehyat::state::kSmemBytes, st>>>(mk, mv, mw, mkc ? *mkc : mk,
+                                                                       mvc ? *mvc : mv, fp);
   return cuda_check(cudaGetLastError(), "fold launch");
 }
 
@@ -704,7 +712,7 @@ static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int
     ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
     ap.out = static_cast<__nv_bfloat16*>(out);
     ap.lse = lse;
-    dim3 grid((rows_per_chunk + 255) / 256, BH, pl.C);
+    dim3 grid(BH, (rows_per_chunk + 255) / 256, pl.C);
     return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, grid, st);
   }
   rehyat::fp32::AttnParams ap{};
@@ -791,8 +799,6 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
   const int BH = d.B * d.H;
   const long long N = (long long)T * L, F = d.F, D = d.D;
   const int C = pl.C;
-  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
   const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
   auto f32 = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
@@ -839,7 +845,7 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
   for (int c = 0; c < C; ++c) {
     const int s = c * Tc, e = (s + Tc < T ? s + Tc : T), w = (s - To > 0 ? s - To : 0);
     const long long nq = (long long)(e - s) * L, nw = (long long)(e - w) * L;
-    const long long r0 = (long long)s * L, k0 = (long long)w * L;
+    const long long r0 = (long long)s * L;
     // the softmax window's gradients, scores recomputed in TMEM: dK, dV per key tile, dQ per
     // query tile
     {
@@ -936,6 +942,92 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int L, int frames_befor
                                     stream);
 }
 
+// Where a bf16 chunk step's softmax window lives: window rows [0, split) in the carried frames
+// (kc, vc with carry_rows rows per (b, h); window row 0 at row carry_row0), the rest in (k, v)
+// (rows per (b, h); window row `split` at row 0).  split = 0: the whole window is (k, v).
+struct WindowSrc {
+  const void* k;
+  const void* v;
+  long long rows;
+  const void* kc;
+  const void* vc;
+  long long carry_rows;
+  int split, carry_row0;
+};
+
+// One bf16 chunk step ("ReHyAt overview" page §2.2-§2.3 and §5.2): S^T copy, phi_q, the
+// attention with the state readout, then the fold of the frames leaving the window into S, Z.
+static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int chunk_frames,
+                           int To, const ChunkPlan& pl, const void* q, const WindowSrc& w,
+                           const float* Wq, const float* bq, const float* Wk, const float* bk,
+                           float* S, float* Z, void* out, uint8_t* ws, cudaStream_t st) {
+  const int BH = d.B * d.H;
+  __nv_bfloat16* St = reinterpret_cast<__nv_bfloat16*>(ws + pl.St);
+  float* dS = reinterpret_cast<float*>(ws + pl.dS);
+  float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
+  // S^T in bf16 for the readout MMA (C = 1, no folds: a transposed copy of S)
+  RH_TRY(launch_scan_bf16(d, dS, dZ, 0, 1, 1, S, Z, St, nullptr, nullptr, nullptr, st));
+  CUtensorMap mq, mk, mv, mkc, mvc, ms, mwq, mwk;
+  RH_TRY(make_map(&mq, q, d.D, pl.nq, BH));
+  RH_TRY(make_map(&mk, w.k, d.D, w.rows, BH));
+  RH_TRY(make_map(&mv, w.v, d.D, w.rows, BH));
+  if (w.split > 0) {
+    RH_TRY(make_map(&mkc, w.kc, d.D, w.carry_rows, BH));
+    RH_TRY(make_map(&mvc, w.vc, d.D, w.carry_rows, BH));
+  } else {
+    mkc = mk;
+    mvc = mv;
+  }
+  RH_TRY(make_map(&ms, St, d.F, d.D, BH));
+  RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mwq, st));
+  __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
+  if (frames_before - pl.o > 0)  // the chunk reads a linear state
+    RH_TRY(launch_featmap_tc(d, q, pl.nq, 0, pl.nq, mwq, bq, phiq, st));
+  CUtensorMap mphi;
+  RH_TRY(make_map(&mphi, phiq, d.F, pl.nq, BH));
+  rehyat::attn::Params ap{};
+  ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
+  ap.frames_before = frames_before;
+  // the main source's row 0 is window row `split`
+  ap.kv_frame0 = frames_before - pl.o + w.split / L;
+  ap.kv_split = w.split; ap.carry_row0 = w.carry_row0;
+  ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
+  ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
+  RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
+                                dim3(BH, (pl.nq + 255) / 256, 1), st, &mkc, &mvc));
+  if (pl.fold_rows > 0) {
+    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
+    rehyat::state::FoldParams fp{};
+    fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.single_rows = pl.fold_rows; fp.n_fold = 1;
+    fp.seg_rows = pl.fold_rows < w.split ? pl.fold_rows : w.split;
+    fp.seg_row0 = w.carry_row0;
+    fp.splits = pl.splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(pl.splits, 1, BH), st, &mkc, &mvc));
+    rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
+        dS, dZ, pl.splits, d.F, d.D, S, Z);
+    RH_TRY(cuda_check(cudaGetLastError(), "state add launch"));
+  }
+  return REHYAT_OK;
+}
+
+// Argument checks shared by the window-buffer and the carried-frame chunk steps.
+static int check_step(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_before,
+                      int chunk_frames, int To, int To_next) {
+  RH_TRY(check_dims(d, dt));
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(chunk_frames, L, 1, To));
+  if (frames_before < 0) return fail(REHYAT_ERR_ARG, "frames_before must be >= 0");
+  if (To_next < 0) return fail(REHYAT_ERR_ARG, "To_next must be >= 0");
+  const int o = To < frames_before ? To : frames_before;
+  const int seen = frames_before + chunk_frames;
+  if ((To_next < seen ? To_next : seen) > o + chunk_frames)
+    return fail(REHYAT_ERR_ARG,
+                "To_next=%d reaches before this window (%d frames): those frames are already "
+                "folded into S", To_next, o + chunk_frames);
+  return REHYAT_OK;
+}
+
 int rehyat_chunk_forward_sched(rehyat_dims d, rehyat_dtype dt, int L, int frames_before,
                                int chunk_frames, int To, int To_next, const void* q,
                                const void* k_win, const void* v_win, const float* Wq,
@@ -943,19 +1035,7 @@ int rehyat_chunk_forward_sched(rehyat_dims d, rehyat_dtype dt, int L, int frames
                                float* Z, void* out, void* workspace, size_t ws_bytes,
                                void* stream) {
   g_msg[0] = 0;
-  RH_TRY(check_dims(d, dt));
-  RH_TRY(check_path_shape(d, dt));
-  RH_TRY(check_sched(chunk_frames, L, 1, To));
-  if (frames_before < 0) return fail(REHYAT_ERR_ARG, "frames_before must be >= 0");
-  if (To_next < 0) return fail(REHYAT_ERR_ARG, "To_next must be >= 0");
-  {
-    const int o = To < frames_before ? To : frames_before;
-    const int seen = frames_before + chunk_frames;
-    if ((To_next < seen ? To_next : seen) > o + chunk_frames)
-      return fail(REHYAT_ERR_ARG,
-                  "To_next=%d reaches before this window (%d frames): those frames are already "
-                  "folded into S", To_next, o + chunk_frames);
-  }
+  RH_TRY(check_step(d, dt, L, frames_before, chunk_frames, To, To_next));
   if (!q || !k_win || !v_win || !Wq || !Wk || !S || !Z || !out)
     return fail(REHYAT_ERR_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k_win) || !aligned16(v_win) || !aligned16(out))
@@ -970,41 +1050,9 @@ int rehyat_chunk_forward_sched(rehyat_dims d, rehyat_dtype dt, int L, int frames
   const int BH = d.B * d.H;
 
   if (dt == REHYAT_BF16) {
-    __nv_bfloat16* St = reinterpret_cast<__nv_bfloat16*>(ws + pl.St);
-    float* dS = reinterpret_cast<float*>(ws + pl.dS);
-    float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
-    // S^T in bf16 for the readout MMA (C = 1, no folds: a transposed copy of S)
-    RH_TRY(launch_scan_bf16(d, dS, dZ, 0, 1, 1, S, Z, St, nullptr, nullptr, nullptr, st));
-    CUtensorMap mq, mk, mv, ms, mwq, mwk;
-    RH_TRY(make_map(&mq, q, d.D, pl.nq, BH));
-    RH_TRY(make_map(&mk, k_win, d.D, pl.nkv, BH));
-    RH_TRY(make_map(&mv, v_win, d.D, pl.nkv, BH));
-    RH_TRY(make_map(&ms, St, d.F, d.D, BH));
-    RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mwq, st));
-    __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
-    if (frames_before - pl.o > 0)  // the chunk reads a linear state
-      RH_TRY(launch_featmap_tc(d, q, pl.nq, 0, pl.nq, mwq, bq, phiq, st));
-    CUtensorMap mphi;
-    RH_TRY(make_map(&mphi, phiq, d.F, pl.nq, BH));
-    rehyat::attn::Params ap{};
-    ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
-    ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
-    ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
-    ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
-    ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
-    RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
-                                  dim3((pl.nq + 255) / 256, BH, 1), st));
-    if (pl.fold_rows > 0) {
-      RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
-      rehyat::state::FoldParams fp{};
-      fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.single_rows = pl.fold_rows; fp.n_fold = 1;
-      fp.splits = pl.splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
-      RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(pl.splits, 1, BH), st));
-      rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
-          dS, dZ, pl.splits, d.F, d.D, S, Z);
-      RH_TRY(cuda_check(cudaGetLastError(), "state add launch"));
-    }
-    return REHYAT_OK;
+    const WindowSrc w{k_win, v_win, pl.nkv, nullptr, nullptr, 0, 0, 0};
+    return chunk_step_bf16(d, L, frames_before, chunk_frames, To, pl, q, w, Wq, bq, Wk, bk, S, Z,
+                           out, ws, st);
   }
   // fp32
   float* phiq = reinterpret_cast<float*>(ws + pl.phiq);
@@ -1056,17 +1104,16 @@ int rehyat_chunk_forward_carry(rehyat_dims d, rehyat_dtype dt, int L, int frames
                                float* Z, void* k_carry, void* v_carry, void* out,
                                void* workspace, size_t ws_bytes, void* stream) {
   g_msg[0] = 0;
-  RH_TRY(check_dims(d, dt));
-  RH_TRY(check_path_shape(d, dt));
-  RH_TRY(check_sched(chunk_frames, L, 1, To));
-  if (frames_before < 0) return fail(REHYAT_ERR_ARG, "frames_before must be >= 0");
+  RH_TRY(check_step(d, dt, L, frames_before, chunk_frames, To, To_next));
   if (carry_frames < To) return fail(REHYAT_ERR_ARG, "carry_frames %d < To %d", carry_frames, To);
-  if (!k || !v || (carry_frames > 0 && (!k_carry || !v_carry)))
+  if (!q || !k || !v || !Wq || !Wk || !S || !Z || !out ||
+      (carry_frames > 0 && (!k_carry || !v_carry)))
     return fail(REHYAT_ERR_ARG, "null pointer");
-  if (!aligned16(k) || !aligned16(v) || !aligned16(k_carry) || !aligned16(v_carry))
-    return fail(REHYAT_ERR_ALIGN, "k/v/k_carry/v_carry not 16-byte aligned");
-  // the window and the step's workspace are sized for this call's To; the caller's workspace
-  // comes from rehyat_chunk_carry_workspace_size with the largest chunk_frames and To
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_carry) ||
+      !aligned16(v_carry) || !aligned16(out))
+    return fail(REHYAT_ERR_ALIGN, "q/k/v/k_carry/v_carry/out not 16-byte aligned");
+  // the step's workspace is sized for this call's To; the caller's workspace comes from
+  // rehyat_chunk_carry_workspace_size with the largest chunk_frames and To
   const CarryPlan pl = plan_carry(d, dt, L, chunk_frames, To, carry_frames);
   if (!workspace || ws_bytes < pl.total)
     return fail(REHYAT_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", pl.total, ws_bytes);
@@ -1076,32 +1123,73 @@ int rehyat_chunk_forward_carry(rehyat_dims d, rehyat_dtype dt, int L, int frames
   const int BH = d.B * d.H;
   const int ov = To < frames_before ? To : frames_before;
   const size_t es = dt == REHYAT_BF16 ? 2 : 4;
+  const size_t frame_bytes = (size_t)L * d.D * es;  // one frame of one (b, h)
   rehyat::carry::Params cp{};
   cp.L = L; cp.ov = ov; cp.cf = chunk_frames; cp.cap = carry_frames;
   cp.row_vec = (int)(d.D * es / 16);
-  const long long vecs = ((long long)(ov + chunk_frames) + carry_frames) * L * cp.row_vec;
-  long long gx = (vecs + 255) / 256;
-  const long long max_gx = (8LL * 148 + BH - 1) / BH;
-  if (gx > max_gx) gx = max_gx;
-  for (int t = 0; t < 2; ++t) {
-    cp.carry = static_cast<const uint4*>(t ? v_carry : k_carry);
-    cp.chunk = static_cast<const uint4*>(t ? v : k);
-    cp.window = reinterpret_cast<uint4*>(ws + (t ? pl.vwin : pl.kwin));
-    cp.carry_new = reinterpret_cast<uint4*>(ws + (t ? pl.vcar : pl.kcar));
-    rehyat::carry::gather_kernel<<<dim3((unsigned)gx, BH), 256, 0, st>>>(cp);
-    RH_TRY(cuda_check(cudaGetLastError(), "window gather launch"));
-  }
-  RH_TRY(rehyat_chunk_forward_sched(d, dt, L, frames_before, chunk_frames, To, To_next, q,
-                                    ws + pl.kwin, ws + pl.vwin, Wq, bq, Wk, bk, S, Z, out,
-                                    ws + pl.step, pl.kwin - pl.step, stream));
-  const size_t car_bytes = (size_t)BH * carry_frames * L * d.D * es;
-  if (car_bytes) {
+  // gather launch: window (fp32 only) and next carry of K, then of V
+  auto gather = [&](bool window) -> int {
+    cp.window_out = window ? 1 : 0;
+    const long long vecs =
+        ((window ? (long long)(ov + chunk_frames) : 0LL) + carry_frames) * L * cp.row_vec;
+    long long gx = (vecs + 255) / 256;
+    const long long max_gx = (8LL * 148 + BH - 1) / BH;
+    if (gx > max_gx) gx = max_gx;
+    if (gx < 1) gx = 1;
+    for (int t = 0; t < 2; ++t) {
+      cp.carry = static_cast<const uint4*>(t ? v_carry : k_carry);
+      cp.chunk = static_cast<const uint4*>(t ? v : k);
+      cp.window = window ? reinterpret_cast<uint4*>(ws + (t ? pl.vwin : pl.kwin)) : nullptr;
+      cp.carry_new = reinterpret_cast<uint4*>(ws + (t ? pl.vcar : pl.kcar));
+      rehyat::carry::gather_kernel<<<dim3((unsigned)gx, BH), 256, 0, st>>>(cp);
+      RH_TRY(cuda_check(cudaGetLastError(), "window gather launch"));
+    }
+    return REHYAT_OK;
+  };
+  auto copy_back = [&]() -> int {
+    const size_t car_bytes = (size_t)BH * carry_frames * frame_bytes;
+    if (!car_bytes) return REHYAT_OK;
     RH_TRY(cuda_check(cudaMemcpyAsync(k_carry, ws + pl.kcar, car_bytes, cudaMemcpyDeviceToDevice, st),
                       "carry copy"));
     RH_TRY(cuda_check(cudaMemcpyAsync(v_carry, ws + pl.vcar, car_bytes, cudaMemcpyDeviceToDevice, st),
                       "carry copy"));
+    return REHYAT_OK;
+  };
+
+  if (dt == REHYAT_BF16) {
+    // The kernels read the window straight from the carry (its last ov frames) and the chunk.
+    const ChunkPlan cpl = plan_chunk(d, dt, L, frames_before, chunk_frames, To, To_next);
+    if (cpl.total > pl.step_bytes)
+      return fail(REHYAT_ERR_WORKSPACE, "chunk step needs %zu bytes, plan holds %zu", cpl.total,
+                  pl.step_bytes);
+    const WindowSrc w{k, v, (long long)chunk_frames * L, k_carry, v_carry,
+                      (long long)carry_frames * L, ov * L, (carry_frames - ov) * L};
+    RH_TRY(chunk_step_bf16(d, L, frames_before, chunk_frames, To, cpl, q, w, Wq, bq, Wk, bk, S, Z,
+                           out, ws + pl.step, st));
+    // the next carry, after every read of the old one (stream order): the last carry_frames
+    // frames of (carry ++ chunk)
+    if (carry_frames == 0) return REHYAT_OK;
+    if (chunk_frames >= carry_frames) {
+      for (int t = 0; t < 2; ++t) {
+        const uint8_t* src = static_cast<const uint8_t*>(t ? v : k) +
+                             (size_t)(chunk_frames - carry_frames) * frame_bytes;
+        RH_TRY(cuda_check(cudaMemcpy2DAsync(t ? v_carry : k_carry, carry_frames * frame_bytes, src,
+                                            chunk_frames * frame_bytes,
+                                            carry_frames * frame_bytes, BH,
+                                            cudaMemcpyDeviceToDevice, st),
+                          "carry copy"));
+      }
+      return REHYAT_OK;
+    }
+    RH_TRY(gather(false));
+    return copy_back();
   }
-  return REHYAT_OK;
+  // fp32: assemble the window, run the window-buffer step, then replace the carry
+  RH_TRY(gather(true));
+  RH_TRY(rehyat_chunk_forward_sched(d, dt, L, frames_before, chunk_frames, To, To_next, q,
+                                    ws + pl.kwin, ws + pl.vwin, Wq, bq, Wk, bk, S, Z, out,
+                                    ws + pl.step, pl.step_bytes, stream));
+  return copy_back();
 }
 
 int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frames_before,
@@ -1160,7 +1248,7 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
-  RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3((pl.nq + 255) / 256, nbh, 1),
+  RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3(nbh, (pl.nq + 255) / 256, 1),
                                  st));
   if (pl.fold_rows > 0) {
     RH_TRY(prepare_blockdiag(d, Wk, Wkbd, &mwk, st));

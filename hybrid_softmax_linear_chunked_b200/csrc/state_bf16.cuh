@@ -49,6 +49,10 @@ struct FoldParams {
   int L, H, P;
   int T, Tc, To, kv_frame0;  // schedule (mode 0)
   int single_rows;           // mode 1: fold rows [0, single_rows) of the k/v buffer; -1 = mode 0
+  // mode 1 with a carried segment: the first seg_rows of the fold range come from tmKc/tmVc at
+  // row seg_row0, the remaining single_rows - seg_rows from tmK/tmV at row 0; each segment is
+  // tiled on its own.  seg_rows = 0: one segment.
+  int seg_rows, seg_row0;
   int n_fold, splits;
   const float* bk;
   float* dS;  // [BH][n_fold][splits][F][D]
@@ -78,7 +82,9 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_addr, int kk) {
 __global__ void __launch_bounds__(kThreads, 1)
     fold_partial_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
                              const __grid_constant__ CUtensorMap tmV,
-                             const __grid_constant__ CUtensorMap tmW, const FoldParams p) {
+                             const __grid_constant__ CUtensorMap tmW,
+                             const __grid_constant__ CUtensorMap tmKc,
+                             const __grid_constant__ CUtensorMap tmVc, const FoldParams p) {
   static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
   const int split = blockIdx.x, fc = blockIdx.y, bh = blockIdx.z, h = bh % p.H;
   int r0, r1;
@@ -90,7 +96,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     r0 = (w0 - p.kv_frame0) * p.L;
     r1 = (w1 - p.kv_frame0) * p.L;
   }
-  const int n_tiles_all = (r1 - r0 + kTok - 1) / kTok;
+  // tiles [0, n_seg) cover the carried segment, the rest rows [r0 + seg, r1)
+  const int seg = p.single_rows >= 0 ? p.seg_rows : 0;
+  const int n_seg = (seg + kTok - 1) / kTok;
+  const int n_tiles_all = n_seg + (r1 - r0 - seg + kTok - 1) / kTok;
   const int t_begin = (int)((long long)split * n_tiles_all / p.splits);
   const int t_end = (int)((long long)(split + 1) * n_tiles_all / p.splits);
   const int n_tiles = t_end - t_begin;
@@ -159,14 +168,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued_k = 0, issued_v = 0;
     for (int i = 0; i < n_tiles; ++i) {
       const int s = i & 1;
-      const int row = r0 + (t_begin + i) * kTok;
+      const int ti = t_begin + i;
+      const bool carried = ti < n_seg;
+      // the main source holds window row seg at its row r0 (mode 1 with a segment: r0 = 0)
+      const int row = carried ? p.seg_row0 + ti * kTok : r0 + (ti - n_seg) * kTok;
+      const CUtensorMap* mK = carried ? &tmKc : &tmK;
+      const CUtensorMap* mV = carried ? &tmVc : &tmV;
       if (i >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty], (i - 1) & 1, abort_flag));
       if (!ok) break;
       if (leader) {
         uint8_t* dk = sm + kOffK;
         mbar_arrive_expect_tx(&bars[kKFull], kTileBytes);
-        tma_load_3d(dk, &tmK, &bars[kKFull], 0, row, bh);
-        tma_load_3d(dk + kTok * 128, &tmK, &bars[kKFull], 64, row, bh);
+        tma_load_3d(dk, mK, &bars[kKFull], 0, row, bh);
+        tma_load_3d(dk + kTok * 128, mK, &bars[kKFull], 64, row, bh);
       }
       __syncwarp();
       ++issued_k;
@@ -175,8 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) {
         uint8_t* dv = sm + kOffV + s * kTileBytes;
         mbar_arrive_expect_tx(&bars[kVFull + s], kTileBytes);
-        tma_load_3d(dv, &tmV, &bars[kVFull + s], 0, row, bh);
-        tma_load_3d(dv + kTok * 128, &tmV, &bars[kVFull + s], 64, row, bh);
+        tma_load_3d(dv, mV, &bars[kVFull + s], 0, row, bh);
+        tma_load_3d(dv + kTok * 128, mV, &bars[kVFull + s], 64, row, bh);
       }
       __syncwarp();
       ++issued_v;
@@ -262,7 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       uint8_t* prow = sm + kOffPhi + s * kTileBytes;
-      const bool valid = r0 + (t_begin + i) * kTok + r < r1;
+      const int ti = t_begin + i;
+      const bool valid = ti < n_seg ? ti * kTok + r < seg : r0 + seg + (ti - n_seg) * kTok + r < r1;
 #pragma unroll 1
       for (int c16 = 0; c16 < 4; ++c16) {  // 16 features per step keeps the loop body small
         const int f0 = col0 + c16 * 16;

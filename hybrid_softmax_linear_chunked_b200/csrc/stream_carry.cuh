@@ -7,7 +7,8 @@
 //   window rows [ov L, (ov + cf) L) <- chunk rows [0, cf L)
 //   new carry frame f (0 <= f < cap) <- chunk frame f - (cap - cf) if f >= cap - cf,
 //                                       else carry frame f + cf
-// The new carry goes to a separate buffer (the old one is still being read).
+// The new carry goes to a separate buffer (the old one is still being read).  With
+// window_out = 0 only the new carry is written (the kernels read the window in place).
 #pragma once
 
 #include <cstdint>
@@ -20,6 +21,7 @@ struct Params {
   int ov, cf;     // overlap frames taken from the carry, chunk frames
   int cap;        // carried frames
   int row_vec;    // 16-byte vectors per row
+  int window_out; // 1: also write the window
   const uint4* carry;   // [BH][cap L][row]
   const uint4* chunk;   // [BH][cf L][row]
   uint4* window;        // [BH][(ov + cf) L][row]
@@ -30,7 +32,8 @@ struct Params {
 __global__ void __launch_bounds__(256) gather_kernel(const Params p) {
   const long long bh = blockIdx.y;
   const long long L = p.L;
-  const long long win_rows = (long long)(p.ov + p.cf) * L, cap_rows = (long long)p.cap * L;
+  const long long win_rows = p.window_out ? (long long)(p.ov + p.cf) * L : 0LL;
+  const long long cap_rows = (long long)p.cap * L;
   const long long chunk_rows = (long long)p.cf * L;
   const long long total = (win_rows + cap_rows) * p.row_vec;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;

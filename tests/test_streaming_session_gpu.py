@@ -121,15 +121,18 @@ def test_session_rejects_bad_chunks_and_states(dev, data):
         new_session(t).load_state_dict(st)
 
 
-def test_variable_schedule(dev):
+@pytest.mark.parametrize("cfs,ovs", [([5, 3, 3, 2], [0, 1, 2, 1]),
+                                     # a 1-frame chunk under a 2-frame carry: the next carry
+                                     # mixes carried and new frames
+                                     ([3, 1, 2, 3], [0, 2, 2, 1])])
+def test_variable_schedule(dev, cfs, ovs):
     """A longer first chunk and per-chunk overlaps (ReHyAt overview §5.2), bf16, against the
     quadratic form under the schedule's frame mask."""
-    w = C.Workload("sched", B=1, H=2, D=128, T=13, frame_h=6, frame_w=11, Tc=5, To=2, P=2,
-                   F=128, G=8, dtype="bf16", seed=35)
+    w = C.Workload("sched", B=1, H=2, D=128, T=sum(cfs), frame_h=6, frame_w=11, Tc=max(cfs),
+                   To=max(ovs), P=2, F=128, G=8, dtype="bf16", seed=35)
     inp = make_inputs(w)
     t = [x.to(dev) for x in (inp.q, inp.k, inp.v, inp.Wq, inp.bq, inp.Wk, inp.bk)]
     q, k, v = t[:3]
-    cfs, ovs = [5, 3, 3, 2], [0, 1, 2, 1]
     bounds = O.schedule_bounds(cfs, ovs)
     sess = new_session(t, w)
     L = w.frame_tokens
