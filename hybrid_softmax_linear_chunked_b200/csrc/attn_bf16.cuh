@@ -210,6 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  // Z_c is in shared memory: a kernel launched behind this one may start (and update the state)
+  // once every CTA is here, filling the SMs of the last wave.  Window, phi_q and S^T reads follow.
+  grid_dep_signal();
 
   const uint32_t sQ0 = smem_u32(sm + kOffQ0), sQ1 = smem_u32(sm + kOffQ1);
   const uint32_t sK0 = smem_u32(sm + kOffK), sK1 = sK0 + kTileBytes;

@@ -370,16 +370,29 @@ int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int 
   return cuda_check(cudaGetLastError(), "featmap_tc launch");
 }
 
+// behind_attention: launch with programmatic stream serialization right after an attention
+// launch, so the fold starts once every attention CTA is resident (the kernel waits for the
+// attention grid before it exits).
 int launch_fold_bf16(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mw,
                      const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st,
-                     const CUtensorMap* mkc = nullptr, const CUtensorMap* mvc = nullptr) {
+                     const CUtensorMap* mkc = nullptr, const CUtensorMap* mvc = nullptr,
+                     bool behind_attention = false) {
   auto k = rehyat::state::fold_partial_bf16_kernel;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)rehyat::state::kSmemBytes),
                     "fold attr"));
-  k<<<grid, rehyat::state::kThreads, rehyat::state::kSmemBytes, st>>>(mk, mv, mw, mkc ? *mkc : mk,
-                                                                       mvc ? *mvc : mv, fp);
-  return cuda_check(cudaGetLastError(), "fold launch");
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(rehyat::state::kThreads);
+  cfg.dynamicSmemBytes = rehyat::state::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = behind_attention ? 1 : 0;
+  const CUtensorMap kc = mkc ? *mkc : mk, vc = mvc ? *mvc : mv;
+  return cuda_check(cudaLaunchKernelEx(&cfg, k, mk, mv, mw, kc, vc, fp), "fold launch");
 }
 
 // Block-diagonal bf16 hi/lo weights of one feature map into `out` ([H][2][F][D] bf16) and the
@@ -994,16 +1007,19 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
   ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
+  if (pl.fold_rows > 0)
+    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
   RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
                                 dim3(BH, (pl.nq + 255) / 256, 1), st, &mkc, &mvc));
   if (pl.fold_rows > 0) {
-    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
+    // the fold reads only the window and writes its own partials: it runs in the attention's
+    // last wave; the state update after it waits for both
     rehyat::state::FoldParams fp{};
     fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.single_rows = pl.fold_rows; fp.n_fold = 1;
     fp.seg_rows = pl.fold_rows < w.split ? pl.fold_rows : w.split;
     fp.seg_row0 = w.carry_row0;
     fp.splits = pl.splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
-    RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(pl.splits, 1, BH), st, &mkc, &mvc));
+    RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(pl.splits, 1, BH), st, &mkc, &mvc, true));
     rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
         dS, dZ, pl.splits, d.F, d.D, S, Z);
     RH_TRY(cuda_check(cudaGetLastError(), "state add launch"));

@@ -97,6 +97,17 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
 }
 
 // ------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched after this one with programmatic stream
+// serialization may start once every CTA of this grid has signalled (or exited); a kernel so
+// launched waits for the full completion (and memory) of the grid before it with grid_dep_wait.
+// Both are no-ops for ordinary launches.
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dep_signal() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ------------------------------------------------------------------------------------------
 // TMA
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

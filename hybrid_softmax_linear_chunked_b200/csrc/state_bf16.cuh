@@ -106,9 +106,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* dS = p.dS + (((size_t)bh * p.n_fold + fc) * p.splits + split) * kFD * kHD;
   float* dZ = p.dZ + (((size_t)bh * p.n_fold + fc) * p.splits + split) * kFD;
+  // Launched behind the streaming attention with programmatic serialization, the fold reads
+  // only the window (never written there) and overlaps the attention's last wave; every CTA
+  // waits for that grid before it exits, so whatever follows the fold in the stream is ordered
+  // after the attention too.  For an ordinary launch the wait returns at once.
   if (n_tiles <= 0) {
     for (int i = tid; i < kFD * kHD; i += kThreads) dS[i] = 0.f;
     for (int i = tid; i < kFD; i += kThreads) dZ[i] = 0.f;
+    grid_dep_wait();
     return;
   }
 
@@ -321,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  grid_dep_wait();
 }
 
 // Exclusive prefix over fold ranges.  grid (F/32 * D/32, BH), block (32, 8).
