@@ -39,6 +39,8 @@ sys.path.insert(0, ROOT)
 
 from hybrid_softmax_linear_chunked_b200 import binding as rb  # noqa: E402
 from hybrid_softmax_linear_chunked_b200 import configs as C  # noqa: E402
+from hybrid_softmax_linear_chunked_b200.context_parallel import (  # noqa: E402
+    ContextParallel, split_chunks)
 from hybrid_softmax_linear_chunked_b200.inputs import make_inputs  # noqa: E402
 from hybrid_softmax_linear_chunked_b200.replicas import Replicas, job_throughput  # noqa: E402
 from hybrid_softmax_linear_chunked_b200.streaming import ChunkStream  # noqa: E402
@@ -69,6 +71,9 @@ def parse_args():
                          "are computed before the timed region)")
     ap.add_argument("--schedule", default=None,
                     help="streaming only: FRAMES/OVERLAP entries, first once, rest cyclic")
+    ap.add_argument("--parallel", choices=["replicas", "context"], default="replicas",
+                    help="replicas: every rank runs its own batch (weak scaling); context: the "
+                         "ranks split one sequence into chunk ranges (strong scaling)")
     return ap.parse_args()
 
 
@@ -302,8 +307,14 @@ def main():
     torch.cuda.set_device(dev)
     rb.load()
     w = pick_workload(args)
-    inp = make_inputs(w, seed=rep.seed(w.seed))
-    if args.which == "backward":
+    context = args.parallel == "context"
+    if context and (args.which != "forward" or w.mode == "stream"):
+        raise SystemExit("--parallel context times the whole-sequence forward")
+    # context parallelism splits one sequence: every rank draws the same one
+    inp = make_inputs(w, seed=w.seed if context else rep.seed(w.seed))
+    if context:
+        run = context_runner(w, inp, dev, args, rep)
+    elif args.which == "backward":
         run = backward_runner(w, inp, dev, args)
     else:
         run = (stream_runner if w.mode == "stream" else full_runner)(w, inp, dev, args)
@@ -359,21 +370,25 @@ def main():
         achieved = run.attn_flops / (kernel_time * 1e-3) / 1e12
         cfg = workload_config(w, world)
         cfg.update(run.config)
+        # replicas: every rank processed its own batch; context: the ranks shared one
+        units, ranks = (w.B * w.N, 1) if context else (w.B * w.N, world)
+        if context:
+            cfg["global_batch"] = w.B
         line = {
             "metric": METRIC,
-            "value": job_throughput(w.B * w.N, world, ms_per_step),
+            "value": job_throughput(units, ranks, ms_per_step),
             "unit": UNIT,
             "n_gpus": world,
             "steps": K,
             "warmup": args.warmup,
             "ms_per_step": ms_per_step,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong" if context else "weak",
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
             "config": cfg,
-            "tflops": run.step_flops * world / (ms_per_step * 1e-3) / 1e12,
+            "tflops": run.step_flops * ranks / (ms_per_step * 1e-3) / 1e12,
             "frac_of_bf16_peak_step": run.step_flops / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "kernel_ms": ({"attention": attn_ms, "states_and_phiq": pre_ms} if run.attn_isolated
                           else {"step": ms_per_step}),
@@ -385,7 +400,7 @@ def main():
                                                if peaks.get("bf16_tflops_sustained") else None),
                          "traffic": read_traffic() if run.attn_isolated and args.workload == "480p5s"
                                     and w.phi == "poly" else None},
-            "e2e": {"value": job_throughput(w.B * w.N, world, e2e_ms / E), "unit": UNIT,
+            "e2e": {"value": job_throughput(units, ranks, e2e_ms / E), "unit": UNIT,
                     "h2d_bytes_per_step": run.h2d, "d2h_bytes_per_step": run.d2h},
             "gpu_launches": run.launches_per_step * K,
             "clocks": sampler.summary(),
@@ -492,6 +507,58 @@ def backward_runner(w: C.Workload, inp, dev, args) -> _Run:
     r.launches_per_step = (2 * C_ + 4 * lin + 3 + 2 * groups + 2 * (5 * w.B + 4) + 6)
     r.roofline_kernel = "backward pass (all launches; algorithmic FLOPs / time)"
     r.config = {"pass": "backward"}
+    return r
+
+
+def context_runner(w: C.Workload, inp, dev, args, rep) -> _Run:
+    """The whole-sequence forward split into chunk ranges over the ranks (context parallelism):
+    each rank holds its own frames of q, k, v; per step the halo frames go point to point, the
+    segment sums are all-gathered, and each rank computes its chunks' outputs."""
+    r = _Run()
+    r.attn_isolated = False
+    L = w.frame_tokens
+    Wq, bq, Wk, bk = (x.to(dev) for x in (inp.Wq, inp.bq, inp.Wk, inp.bk))
+    cp = ContextParallel(Wq, bq, Wk, bk, T=w.T, frame_tokens=L, Tc=w.Tc, To=w.To, P=w.P,
+                         phi=w.phi_code)
+    own = slice(cp.s0 * L, cp.s1 * L)
+    q_own = inp.q[:, :, own].contiguous().to(dev)
+    k_buf, v_buf = cp.kv_buffer(q_own), cp.kv_buffer(q_own)
+    cp.own(k_buf).copy_(inp.k[:, :, own])
+    cp.own(v_buf).copy_(inp.v[:, :, own])
+    out = torch.empty_like(q_own)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev_mid=None, ev_end=None):
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        cp.forward(q_own, k_buf, v_buf, out=out)
+        if ev_end is not None:
+            ev_end.record(stream)
+
+    host = [inp.q[:, :, own].contiguous().pin_memory(), inp.k[:, :, own].contiguous().pin_memory(),
+            inp.v[:, :, own].contiguous().pin_memory()]
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        q_own.copy_(host[0], non_blocking=True)
+        cp.own(k_buf).copy_(host[1], non_blocking=True)
+        cp.own(v_buf).copy_(host[2], non_blocking=True)
+        cp.forward(q_own, k_buf, v_buf, out=out)
+        host_out.copy_(out, non_blocking=True)
+
+    r.step, r.e2e_step = step, e2e_step
+    r.h2d = sum(x.numel() * x.element_size() for x in host)
+    r.d2h = host_out.numel() * host_out.element_size()
+    r.step_flops = w.flops(streaming=False)
+    r.attn_flops = w.flops(streaming=False)
+    # per rank: [W_k block-diagonal, fold], segment sum; scan, W_q block-diagonal, [phi_q],
+    # attention
+    n_fold = max(0, min(cp.c1, w.n_chunks - 1) - cp.c0)
+    r.launches_per_step = (2 if n_fold else 0) + 1 + 4
+    r.roofline_kernel = "context-parallel forward step (whole-sequence FLOPs / step time)"
+    r.config = {"parallelism": f"cp{rep.world} (chunk ranges [c0, c1) per rank: "
+                               f"{split_chunks(w.n_chunks, rep.world)}; halo point to point, "
+                               "segment sums all-gathered)"}
     return r
 
 

@@ -27,7 +27,8 @@ EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_chunk_forward", "rehyat_chunk_forward_sched", "rehyat_chunk_carry_workspace_size",
             "rehyat_chunk_forward_carry", "rehyat_chunk_forward_static", "rehyat_chunk_states",
             "rehyat_forward_train", "rehyat_backward_workspace_size", "rehyat_backward",
-            "rehyat_gemm_bf16", "rehyat_selftest_wait_timeout", "rehyat_sync_status"]
+            "rehyat_gemm_bf16", "rehyat_segment_workspace_size", "rehyat_segment_states",
+            "rehyat_segment_attend", "rehyat_selftest_wait_timeout", "rehyat_sync_status"]
 
 
 class RehyatError(RuntimeError):
@@ -75,6 +76,12 @@ def load() -> ctypes.CDLL:
                                         c_size_t, P]
     L.rehyat_chunk_workspace_size.argtypes = [Dims, c_int, c_int, c_int, c_int,
                                               ctypes.POINTER(c_size_t)]
+    L.rehyat_segment_workspace_size.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                c_int, ctypes.POINTER(c_size_t)]
+    L.rehyat_segment_states.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                        P, P, P, P, P, P, P, c_size_t, P]
+    L.rehyat_segment_attend.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                        P, P, P, P, P, c_int, P, P, P, P, c_size_t, P]
     L.rehyat_chunk_forward.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, P, P, P, P, P, P,
                                        P, P, P, P, P, c_size_t, P]
     L.rehyat_chunk_forward_sched.argtypes = [Dims, c_int, c_int, c_int, c_int, c_int, c_int, P, P,
@@ -206,6 +213,72 @@ def forward(q, k, v, Wq, bq, Wk, bk, *, P: int, phi: int = 0, frame_tokens: int,
     _check(lib.rehyat_forward(d, code, T, frame_tokens, Tc, To, _ptr(q), _ptr(k), _ptr(v),
                               _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(out), _ptr(ws),
                               ws.numel(), _stream(dev)))
+    return out
+
+
+def segment_bounds(T: int, Tc: int, To: int, c0: int, c1: int) -> tuple[int, int, int]:
+    """(s0, s1, h0) of the segment of chunks [c0, c1): query frames [s0, s1), key/value frames
+    [h0, s1)."""
+    s0, s1 = c0 * Tc, min(c1 * Tc, T)
+    return s0, s1, max(0, s0 - To)
+
+
+def segment_workspace_size(d: Dims, T: int, frame_tokens: int, Tc: int, To: int, c0: int,
+                           c1: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().rehyat_segment_workspace_size(d, REHYAT_BF16, T, frame_tokens, Tc, To, c0, c1,
+                                                ctypes.byref(n)))
+    return n.value
+
+
+def segment_states(k_seg, v_seg, Wk, bk, *, T: int, c0: int, c1: int, P: int, phi: int = 0,
+                   frame_tokens: int, Tc: int, To: int, workspace: torch.Tensor,
+                   S_seg: torch.Tensor | None = None, Z_seg: torch.Tensor | None = None):
+    """First phase of a context-parallel segment (chunks [c0, c1) of a T-frame sequence):
+    k_seg, v_seg [B,H,(s1-h0)*frame_tokens,D] bf16 (halo frames first).  Fills `workspace` with
+    the segment's folds and returns their sum (S_seg [B,H,F,D], Z_seg [B,H,F] fp32)."""
+    lib = load()
+    dev = _dev(k_seg, v_seg, Wk, bk, workspace)
+    d = dims_of(k_seg, Wk, P, phi)
+    B, H = d.B, d.H
+    if S_seg is None:
+        S_seg = torch.empty(B, H, d.F, d.D, dtype=torch.float32, device=dev)
+    if Z_seg is None:
+        Z_seg = torch.empty(B, H, d.F, dtype=torch.float32, device=dev)
+    _dev(S_seg, Z_seg)
+    _check(lib.rehyat_segment_states(d, _dtype_code(k_seg), T, frame_tokens, Tc, To, c0, c1,
+                                     _ptr(k_seg), _ptr(v_seg), _ptr(Wk), _ptr(bk), _ptr(S_seg),
+                                     _ptr(Z_seg), _ptr(workspace), workspace.numel(),
+                                     _stream(dev)))
+    return S_seg, Z_seg
+
+
+def segment_attend(q_seg, k_seg, v_seg, Wq, bq, *, T: int, c0: int, c1: int, P: int,
+                   phi: int = 0, frame_tokens: int, Tc: int, To: int, workspace: torch.Tensor,
+                   S_prefix: torch.Tensor | None = None, Z_prefix: torch.Tensor | None = None,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """Second phase: the segment's outputs.  S_prefix [n,B,H,F,D] / Z_prefix [n,B,H,F] stack
+    the segment sums of every earlier segment (None for the first)."""
+    lib = load()
+    dev = _dev(q_seg, k_seg, v_seg, Wq, bq, workspace)
+    d = dims_of(q_seg, Wq, P, phi)
+    n_prefix = 0
+    if (S_prefix is None) != (Z_prefix is None):
+        raise ValueError("give both S_prefix and Z_prefix or neither")
+    if S_prefix is not None:
+        _dev(S_prefix, Z_prefix)
+        n_prefix = S_prefix.shape[0]
+        if S_prefix.dtype != torch.float32 or Z_prefix.dtype != torch.float32:
+            raise ValueError("S_prefix/Z_prefix must be float32")
+        if Z_prefix.shape[0] != n_prefix:
+            raise ValueError("S_prefix and Z_prefix hold different segment counts")
+    if out is None:
+        out = torch.empty_like(q_seg)
+    _dev(out)
+    _check(lib.rehyat_segment_attend(d, _dtype_code(q_seg), T, frame_tokens, Tc, To, c0, c1,
+                                     _ptr(q_seg), _ptr(k_seg), _ptr(v_seg), _ptr(Wq), _ptr(bq),
+                                     n_prefix, _ptr(S_prefix), _ptr(Z_prefix), _ptr(out),
+                                     _ptr(workspace), workspace.numel(), _stream(dev)))
     return out
 
 

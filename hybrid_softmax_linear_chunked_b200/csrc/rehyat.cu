@@ -280,6 +280,40 @@ ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_be
   return p;
 }
 
+// A segment of chunks [c0, c1) of a T-frame sequence (context parallelism): its query frames
+// [s0, s1), key/value frames [h0, s1) (the overlap halo first), its folds [c0, min(c1, C-1)).
+struct SegPlan {
+  int C, s0, s1, h0, n_local, n_fold, splits;
+  long long nq_rows, nkv_rows;
+  size_t dS, dZ, St, Zc, Wqbd, Wkbd, phiq_bf16, total;
+};
+
+SegPlan plan_segment(const rehyat_dims& d, int T, int L, int Tc, int To, int c0, int c1) {
+  SegPlan p{};
+  const size_t BH = (size_t)d.B * d.H;
+  p.C = (T + Tc - 1) / Tc;
+  p.s0 = c0 * Tc;
+  p.s1 = c1 * Tc < T ? c1 * Tc : T;
+  p.h0 = p.s0 - To > 0 ? p.s0 - To : 0;
+  p.n_local = c1 - c0;
+  const int fold_end = c1 < p.C - 1 ? c1 : p.C - 1;
+  p.n_fold = fold_end > c0 ? fold_end - c0 : 0;
+  p.nq_rows = (long long)(p.s1 - p.s0) * L;
+  p.nkv_rows = (long long)(p.s1 - p.h0) * L;
+  p.splits = fold_splits((int)BH, p.n_fold, (long long)Tc * L);
+  Carve cv;
+  const size_t nf = p.n_fold;
+  p.dS = cv.take(BH * nf * p.splits * d.F * d.D * 4);
+  p.dZ = cv.take(BH * nf * p.splits * d.F * 4);
+  p.St = cv.take(BH * p.n_local * d.D * d.F * 2);
+  p.Zc = cv.take(BH * p.n_local * d.F * 4);
+  p.Wqbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
+  p.Wkbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
+  p.phiq_bf16 = cv.take(BH * (size_t)p.nq_rows * d.F * 2);
+  p.total = cv.off;
+  return p;
+}
+
 // Streaming with carried frames: the chunk step's own workspace, then (fp32 only) the assembled K
 // and V windows, then the next carry of K and V (used when the chunk is shorter than the carry).
 // The bf16 kernels read the window straight from the carry and the chunk.
@@ -405,12 +439,14 @@ int prepare_blockdiag(const rehyat_dims& d, const float* W, __nv_bfloat16* out, 
   return make_map(map, out, d.D, d.F, 2LL * d.H);
 }
 
+// S0/Z0: n_prefix stacked initial states ([n_prefix][BH][F][D], [n_prefix][BH][F]) summed in
+// order, or null for zero.
 int launch_scan_bf16(const rehyat_dims& d, const float* dS, const float* dZ, int n_fold,
                      int splits, int C, const float* S0, const float* Z0, __nv_bfloat16* St,
-                     float* Zc, float* S_out, float* Z_out, cudaStream_t st) {
+                     float* Zc, float* S_out, float* Z_out, cudaStream_t st, int n_prefix = 1) {
   dim3 grid((d.F / 32) * (d.D / 32), d.B * d.H);
-  rehyat::state::state_scan_kernel<<<grid, dim3(32, 8), 0, st>>>(dS, dZ, n_fold, splits, C, d.F,
-                                                                  d.D, S0, Z0, St, Zc, S_out, Z_out);
+  rehyat::state::state_scan_kernel<<<grid, dim3(32, 8), 0, st>>>(
+      dS, dZ, n_fold, splits, C, d.F, d.D, S0, Z0, n_prefix, St, Zc, S_out, Z_out);
   return cuda_check(cudaGetLastError(), "scan launch");
 }
 
@@ -1206,6 +1242,122 @@ int rehyat_chunk_forward_carry(rehyat_dims d, rehyat_dtype dt, int L, int frames
                                     ws + pl.kwin, ws + pl.vwin, Wq, bq, Wk, bk, S, Z, out,
                                     ws + pl.step, pl.step_bytes, stream));
   return copy_back();
+}
+
+static int segment_checks(const rehyat_dims& d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                          int c0, int c1, const void* workspace, size_t ws_bytes, SegPlan* pl) {
+  RH_TRY(check_dims(d, dt));
+  if (dt != REHYAT_BF16) return fail(REHYAT_ERR_DTYPE, "segments are bf16 only");
+  RH_TRY(check_path_shape(d, dt));
+  RH_TRY(check_sched(T, L, Tc, To));
+  const int C = (T + Tc - 1) / Tc;
+  if (c0 < 0 || c1 <= c0 || c1 > C)
+    return fail(REHYAT_ERR_ARG, "segment [%d, %d) is not inside chunks [0, %d)", c0, c1, C);
+  *pl = plan_segment(d, T, L, Tc, To, c0, c1);
+  if (workspace || ws_bytes) {
+    if (!workspace || ws_bytes < pl->total)
+      return fail(REHYAT_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", pl->total, ws_bytes);
+    if (!aligned16(workspace)) return fail(REHYAT_ERR_ALIGN, "workspace not 16-byte aligned");
+  }
+  return REHYAT_OK;
+}
+
+int rehyat_segment_workspace_size(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc,
+                                  int To, int c0, int c1, size_t* bytes) {
+  g_msg[0] = 0;
+  SegPlan pl;
+  RH_TRY(segment_checks(d, dt, T, frame_tokens, Tc, To, c0, c1, nullptr, 0, &pl));
+  if (!bytes) return fail(REHYAT_ERR_ARG, "null bytes pointer");
+  *bytes = pl.total;
+  return REHYAT_OK;
+}
+
+int rehyat_segment_states(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To, int c0,
+                          int c1, const void* k_seg, const void* v_seg, const float* Wk,
+                          const float* bk, float* S_seg, float* Z_seg, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  g_msg[0] = 0;
+  SegPlan pl;
+  if (!workspace) return fail(REHYAT_ERR_WORKSPACE, "null workspace");
+  RH_TRY(segment_checks(d, dt, T, L, Tc, To, c0, c1, workspace, ws_bytes, &pl));
+  if (!k_seg || !v_seg || !Wk || !S_seg || !Z_seg) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (!aligned16(k_seg) || !aligned16(v_seg))
+    return fail(REHYAT_ERR_ALIGN, "k_seg/v_seg not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int BH = d.B * d.H;
+  float* dS = reinterpret_cast<float*>(ws + pl.dS);
+  float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
+  if (pl.n_fold > 0) {
+    CUtensorMap mk, mv, mw;
+    RH_TRY(make_map(&mk, k_seg, d.D, pl.nkv_rows, BH));
+    RH_TRY(make_map(&mv, v_seg, d.D, pl.nkv_rows, BH));
+    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mw, st));
+    rehyat::state::FoldParams fp{};
+    fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.T = T; fp.Tc = Tc; fp.To = To;
+    fp.kv_frame0 = pl.h0; fp.fold_c0 = c0;
+    fp.single_rows = -1; fp.n_fold = pl.n_fold; fp.splits = pl.splits;
+    fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(mk, mv, mw, fp, dim3(pl.splits, pl.n_fold, BH), st));
+  }
+  rehyat::state::state_sum_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
+      dS, dZ, pl.n_fold * pl.splits, d.F, d.D, S_seg, Z_seg);
+  return cuda_check(cudaGetLastError(), "segment sum launch");
+}
+
+int rehyat_segment_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To, int c0,
+                          int c1, const void* q_seg, const void* k_seg, const void* v_seg,
+                          const float* Wq, const float* bq, int n_prefix, const float* S_prefix,
+                          const float* Z_prefix, void* out_seg, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  g_msg[0] = 0;
+  SegPlan pl;
+  if (!workspace) return fail(REHYAT_ERR_WORKSPACE, "null workspace");
+  RH_TRY(segment_checks(d, dt, T, L, Tc, To, c0, c1, workspace, ws_bytes, &pl));
+  if (!q_seg || !k_seg || !v_seg || !Wq || !out_seg) return fail(REHYAT_ERR_ARG, "null pointer");
+  if (n_prefix < 0) return fail(REHYAT_ERR_ARG, "n_prefix must be >= 0");
+  if (n_prefix > 0 && (!S_prefix || !Z_prefix))
+    return fail(REHYAT_ERR_ARG, "null S_prefix/Z_prefix with n_prefix = %d", n_prefix);
+  if (!aligned16(q_seg) || !aligned16(k_seg) || !aligned16(v_seg) || !aligned16(out_seg))
+    return fail(REHYAT_ERR_ALIGN, "q_seg/k_seg/v_seg/out_seg not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int BH = d.B * d.H;
+  // the state each local chunk reads: the earlier segments' sums, then this segment's folds
+  RH_TRY(launch_scan_bf16(d, reinterpret_cast<const float*>(ws + pl.dS),
+                          reinterpret_cast<const float*>(ws + pl.dZ), pl.n_fold, pl.splits,
+                          pl.n_local, n_prefix > 0 ? S_prefix : nullptr,
+                          n_prefix > 0 ? Z_prefix : nullptr,
+                          reinterpret_cast<__nv_bfloat16*>(ws + pl.St),
+                          reinterpret_cast<float*>(ws + pl.Zc), nullptr, nullptr, st,
+                          n_prefix));
+  // phi_q of the rows whose chunk reads a linear state (chunk c with c*Tc > To)
+  CUtensorMap mw;
+  RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mw, st));
+  int c_lin = To / Tc + 1;
+  if (c_lin < c0) c_lin = c0;
+  const long long row_lin = (long long)(c_lin - c0) * Tc * L;
+  __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
+  if (row_lin < pl.nq_rows)
+    RH_TRY(launch_featmap_tc(d, q_seg, (int)pl.nq_rows, (int)row_lin,
+                             (int)(pl.nq_rows - row_lin), mw, bq, phiq, st));
+  CUtensorMap mq, mk, mv, ms, mphi;
+  RH_TRY(make_map(&mq, q_seg, d.D, pl.nq_rows, BH));
+  RH_TRY(make_map(&mk, k_seg, d.D, pl.nkv_rows, BH));
+  RH_TRY(make_map(&mv, v_seg, d.D, pl.nkv_rows, BH));
+  RH_TRY(make_map(&ms, ws + pl.St, d.F, d.D, (long long)BH * pl.n_local));
+  RH_TRY(make_map(&mphi, phiq, d.F, pl.nq_rows, BH));
+  rehyat::attn::Params ap{};
+  ap.L = L; ap.T = pl.s1 - pl.s0; ap.Tc = Tc; ap.To = To;
+  ap.frames_before = pl.s0; ap.kv_frame0 = pl.h0;
+  ap.H = d.H; ap.P = kernel_P(d); ap.n_states = pl.n_local; ap.nq_rows = (int)pl.nq_rows;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
+  ap.bq = nullptr;  // phi_q comes finished from the workspace
+  ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
+  ap.out = static_cast<__nv_bfloat16*>(out_seg);
+  const int rows_per_chunk = (Tc < ap.T ? Tc : ap.T) * L;
+  return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap,
+                                dim3(BH, (rows_per_chunk + 255) / 256, pl.n_local), st);
 }
 
 int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frames_before,

@@ -48,6 +48,7 @@ enum Bar {
 struct FoldParams {
   int L, H, P;
   int T, Tc, To, kv_frame0;  // schedule (mode 0)
+  int fold_c0;               // mode 0: chunk index of fold 0 (a segment of a longer sequence)
   int single_rows;           // mode 1: fold rows [0, single_rows) of the k/v buffer; -1 = mode 0
   // mode 1 with a carried segment: the first seg_rows of the fold range come from tmKc/tmVc at
   // row seg_row0, the remaining single_rows - seg_rows from tmK/tmV at row 0; each segment is
@@ -92,7 +93,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     r0 = 0;
     r1 = p.single_rows;
   } else {
-    const int w0 = max(0, fc * p.Tc - p.To), w1 = max(0, (fc + 1) * p.Tc - p.To);
+    const int c = p.fold_c0 + fc;
+    const int w0 = max(0, c * p.Tc - p.To), w1 = max(0, (c + 1) * p.Tc - p.To);
     r0 = (w0 - p.kv_frame0) * p.L;
     r1 = (w1 - p.kv_frame0) * p.L;
   }
@@ -330,11 +332,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Exclusive prefix over fold ranges.  grid (F/32 * D/32, BH), block (32, 8).
-//   acc starts at S0/Z0 (if given) else 0; for c in 0..C-1: emit state c, then add fold c.
+//   acc starts at the sum of the n_prefix states S0[i]/Z0[i] (i in order; S0 [n_prefix][BH][F][D],
+//   Z0 [n_prefix][BH][F]; none if S0 is null) else 0; for c in 0..C-1: emit state c, then add
+//   fold c.
 //   St  [BH][C][D][F] bf16 (transposed), Zc [BH][C][F] fp32, S_out [BH][C][F][D] fp32 (opt).
 __global__ void __launch_bounds__(256) state_scan_kernel(
     const float* __restrict__ dS, const float* __restrict__ dZ, int n_fold, int splits, int C,
-    int F, int D, const float* __restrict__ S0, const float* __restrict__ Z0,
+    int F, int D, const float* __restrict__ S0, const float* __restrict__ Z0, int n_prefix,
     __nv_bfloat16* __restrict__ St, float* __restrict__ Zc, float* __restrict__ S_out,
     float* __restrict__ Z_out) {
   __shared__ float tile[32][33];
@@ -345,12 +349,18 @@ __global__ void __launch_bounds__(256) state_scan_kernel(
   float acc[4];
   float accz = 0.f;
   const bool z_thread = (d0 == 0 && ty == 0);
+  const int BH = gridDim.y;
+  const int np = S0 ? n_prefix : 0;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int f = f0 + ty + 8 * i;
-    acc[i] = S0 ? S0[((size_t)bh * F + f) * D + d0 + tx] : 0.f;
+  for (int i = 0; i < 4; ++i) acc[i] = 0.f;
+  for (int r = 0; r < np; ++r) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int f = f0 + ty + 8 * i;
+      acc[i] += S0[(((size_t)r * BH + bh) * F + f) * D + d0 + tx];
+    }
+    if (z_thread && Z0) accz += Z0[((size_t)r * BH + bh) * F + f0 + tx];
   }
-  if (z_thread) accz = Z0 ? Z0[(size_t)bh * F + f0 + tx] : 0.f;
   for (int c = 0; c < C; ++c) {
     // this chunk's fold partials are loaded first, so their latency overlaps the stores below
     float add[4] = {0.f, 0.f, 0.f, 0.f};
@@ -386,6 +396,26 @@ __global__ void __launch_bounds__(256) state_scan_kernel(
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i] += add[i];
     accz += addz;
+  }
+}
+
+// S_tot[bh] = sum over the n partial slabs dS[bh][0..n) (n = folds x splits), Z_tot likewise:
+// one segment's fold total.  grid (ceil(F*D/256), BH), block 256.
+__global__ void __launch_bounds__(256) state_sum_kernel(const float* __restrict__ dS,
+                                                        const float* __restrict__ dZ, int n,
+                                                        int F, int D, float* __restrict__ S_tot,
+                                                        float* __restrict__ Z_tot) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * 256 + threadIdx.x;
+  if (e < F * D) {
+    float a = 0.f;
+    for (int s = 0; s < n; ++s) a += dS[((size_t)bh * n + s) * F * D + e];
+    S_tot[(size_t)bh * F * D + e] = a;
+  }
+  if (e < F) {
+    float z = 0.f;
+    for (int s = 0; s < n; ++s) z += dZ[((size_t)bh * n + s) * F + e];
+    Z_tot[(size_t)bh * F + e] = z;
   }
 }
 

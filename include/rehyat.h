@@ -253,6 +253,37 @@ int rehyat_gemm_bf16(int M, int N, int K, int batch, const void* A, long long ld
                      int b_mn, void* C, long long ldc, long long c_batch, int c_bf16,
                      int accumulate, float alpha, void* stream);
 
+/* Context parallelism over chunk ranges ("ReHyAt overview" page §2.3: the state a chunk reads
+ * is a sum over the folds of all chunks before it, so a sequence splits into contiguous chunk
+ * ranges whose only coupling is that sum and the To overlap frames).  A segment is the chunks
+ * [c0, c1) of a bf16 sequence of T frames (0 <= c0 < c1 <= ceil(T/Tc)):
+ *   query frames [s0, s1) with s0 = c0*Tc, s1 = min(c1*Tc, T);
+ *   key/value frames [h0, s1) with h0 = max(0, s0 - To) (the To halo frames before s0 included).
+ *   q_seg [B,H,(s1-s0)*L,D], k_seg, v_seg [B,H,(s1-h0)*L,D], out_seg [B,H,(s1-s0)*L,D] bf16.
+ * Two phases on one workspace (sized by rehyat_segment_workspace_size, unchanged in between):
+ *   _states: the folds of the segment's chunks (every fold c' in [c0, min(c1, C-1)), frames
+ *            [w_c', w_c'+1)) into the workspace, and their sum into S_seg [B,H,F,D] and
+ *            Z_seg [B,H,F] (fp32, caller-owned; zeros when the segment folds nothing);
+ *   _attend: the outputs of the segment's chunks.  S_prefix [n_prefix][B,H,F,D] and Z_prefix
+ *            [n_prefix][B,H,F] hold the S_seg/Z_seg of every segment before this one (n_prefix
+ *            of them, in sequence order; n_prefix = 0 and null pointers for the first segment);
+ *            they are summed in that order into the state of chunk c0.
+ * Between the phases a multi-GPU caller gathers every rank's S_seg/Z_seg; nothing else crosses
+ * ranks except the halo frames of k and v.  With one segment (c0 = 0, c1 = C, n_prefix = 0) the
+ * result equals rehyat_forward up to the order of fp32 additions in the states.  bf16 only
+ * (REHYAT_ERR_DTYPE otherwise).  Enqueued on `stream`; allocates nothing. */
+int rehyat_segment_workspace_size(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc,
+                                  int To, int c0, int c1, size_t* bytes);
+int rehyat_segment_states(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
+                          int c0, int c1, const void* k_seg, const void* v_seg, const float* Wk,
+                          const float* bk, float* S_seg, float* Z_seg, void* workspace,
+                          size_t ws_bytes, void* stream);
+int rehyat_segment_attend(rehyat_dims d, rehyat_dtype dt, int T, int frame_tokens, int Tc, int To,
+                          int c0, int c1, const void* q_seg, const void* k_seg, const void* v_seg,
+                          const float* Wq, const float* bq, int n_prefix, const float* S_prefix,
+                          const float* Z_prefix, void* out_seg, void* workspace, size_t ws_bytes,
+                          void* stream);
+
 /* Failure-path self test (no counterpart on the pages): enqueue on `stream` one small kernel whose
  * warps wait on an mbarrier that nothing arrives on, with the same bounded wait the other
  * kernels use but a limit of `limit_ns` nanoseconds (1e3 .. 2e9).  The wait gives up, the kernel

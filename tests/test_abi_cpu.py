@@ -154,3 +154,25 @@ def test_backward_checks(lib):
     # fp32 training forward refused
     assert lib.rehyat_forward_train(d, rb.REHYAT_F32, 7, 64, 3, 1, FAKE, FAKE, FAKE, FAKE, None,
                                     FAKE, None, FAKE, FAKE, FAKE, 1 << 40, None) == -3
+
+
+def test_segment_checks(lib):
+    """Context-parallel segment calls: range, dtype and workspace checks (no device work)."""
+    d = dims()
+    n = ctypes.c_size_t(0)
+    # 7 chunks of 3 frames (T = 21): [2, 5) is a valid segment
+    assert lib.rehyat_segment_workspace_size(d, rb.REHYAT_BF16, 21, 64, 3, 1, 2, 5,
+                                             ctypes.byref(n)) == 0 and n.value > 0
+    for c0, c1 in [(3, 3), (-1, 2), (5, 8)]:
+        assert lib.rehyat_segment_workspace_size(d, rb.REHYAT_BF16, 21, 64, 3, 1, c0, c1,
+                                                 ctypes.byref(n)) == -1
+    assert lib.rehyat_segment_workspace_size(d, rb.REHYAT_F32, 21, 64, 3, 1, 0, 7,
+                                             ctypes.byref(n)) == -3
+    # the segment sums need a workspace at least the plan's size
+    st = lib.rehyat_segment_states(d, rb.REHYAT_BF16, 21, 64, 3, 1, 2, 5, FAKE, FAKE, FAKE, None,
+                                   FAKE, FAKE, FAKE, 16, None)
+    assert st == -4
+    # prefix states announced but missing
+    st = lib.rehyat_segment_attend(d, rb.REHYAT_BF16, 21, 64, 3, 1, 2, 5, FAKE, FAKE, FAKE, FAKE,
+                                   None, 2, None, None, FAKE, FAKE, 1 << 30, None)
+    assert st == -1 and "S_prefix" in lib.rehyat_last_error().decode()
