@@ -203,15 +203,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = tid; i < kFD; i += 256) {
       sPw[i] = static_cast<uint8_t>(feature_power(i, kFD, p.P));
       sB[i] = p.bq ? p.bq[(size_t)h * kFD + i] : 0.f;
-      sZ[i] = p.Z[((size_t)bh * p.n_states + c) * kFD + i];
+      if (!kPhiGlobal) sZ[i] = p.Z[((size_t)bh * p.n_states + c) * kFD + i];
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  // Z_c is in shared memory: a kernel launched behind this one may start (and update the state)
-  // once every CTA is here, filling the SMs of the last wave.  Window, phi_q and S^T reads follow.
+  // A kernel launched behind this one may start once every CTA is here, filling the SMs of the
+  // last wave; it must not write anything this kernel reads later (window, phi_q, S^T, Z_c).
   grid_dep_signal();
 
   const uint32_t sQ0 = smem_u32(sm + kOffQ0), sQ1 = smem_u32(sm + kOffQ1);
@@ -270,6 +270,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++issued_v;
     }
     if (ok && has_linear) {
+      // S_c^T, Z_c and phi_q come from the kernels enqueued before this one.  Launched behind
+      // the phi_q kernel with programmatic serialization, this kernel ran its key loop while
+      // that grid was still running: wait for it (and so for everything before it) here.
+      grid_dep_wait();
+      if (kPhiGlobal) {  // Z_c for the epilogue; published by the phi_q barrier's arrival below
+        for (int i = lane; i < kFD; i += 32) sZ[i] = p.Z[((size_t)bh * p.n_states + c) * kFD + i];
+        __syncwarp();
+      }
       // S_c^T goes into the K stage that the (absent) tile n_kv would use.
       const int s = n_kv & 1;
       if (n_kv >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty + s], ((n_kv >> 1) - 1) & 1, abort_flag));

@@ -48,6 +48,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     featmap_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                       const __grid_constant__ CUtensorMap tmW, const Params p) {
   static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
+  // the attention launched behind this kernel may start at once: it reads phi_q only after
+  // waiting for this grid
+  grid_dep_signal();
   const int bh = blockIdx.y, h = bh % p.H;
   const int n_tiles_all = (p.n_rows + kRows - 1) / kRows;
   const int t_begin = blockIdx.x * p.tiles_per_cta;

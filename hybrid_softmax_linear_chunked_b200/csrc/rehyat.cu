@@ -367,14 +367,30 @@ template <bool kPhiGlobal>
 int launch_attn_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& ms, const CUtensorMap& mw, const CUtensorMap& mphi,
                      const rehyat::attn::Params& ap, dim3 grid, cudaStream_t st,
-                     const CUtensorMap* mkc = nullptr, const CUtensorMap* mvc = nullptr) {
+                     const CUtensorMap* mkc = nullptr, const CUtensorMap* mvc = nullptr,
+                     bool behind_phiq = false) {
   auto k = rehyat::attn::hybrid_attn_bf16_kernel<kPhiGlobal>;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)rehyat::attn::kSmemBytes),
                     "attn attr"));
-  k<<<grid, rehyat::attn::kThreads, rehyat::attn::kSmemBytes, st>>>(
-      mq, mk, mv, ms, mw, mphi, mkc ? *mkc : mk, mvc ? *mvc : mv, ap);
-  return cuda_check(cudaGetLastError(), "attention launch");
+  // behind_phiq: the launch before this one, in the same call, is the library's phi_q kernel
+  // (everything before that had finished when it started).  The kernel reads what earlier
+  // launches wrote (S^T, Z_c, phi_q) only after waiting for that grid, so it is launched with
+  // programmatic stream serialization and its key loop overlaps the phi_q kernel.  A caller's
+  // own work right before an attention launch is never overlapped.
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(rehyat::attn::kThreads);
+  cfg.dynamicSmemBytes = rehyat::attn::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (kPhiGlobal && behind_phiq) ? 1 : 0;
+  const CUtensorMap kc = mkc ? *mkc : mk, vc = mvc ? *mvc : mv;
+  return cuda_check(cudaLaunchKernelEx(&cfg, k, mq, mk, mv, ms, mw, mphi, kc, vc, ap),
+                    "attention launch");
 }
 
 // phi of rows [row0, row0 + n_rows) of every (b, h) sequence of x (rows_per_bh rows each) into
@@ -722,19 +738,22 @@ int rehyat_forward_phiq(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, in
 
 static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
                                const void* q, const void* k, const void* v, void* out,
-                               float* lse, const void* workspace, size_t ws_bytes, void* stream);
+                               float* lse, const void* workspace, size_t ws_bytes, void* stream,
+                               bool behind_phiq);
 
 int rehyat_forward_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
                           const void* q, const void* k, const void* v, void* out,
                           const void* workspace, size_t ws_bytes, void* stream) {
   return forward_attend_impl(d, dt, T, L, Tc, To, q, k, v, out, nullptr, workspace, ws_bytes,
-                             stream);
+                             stream, false);
 }
 
+// behind_phiq: the caller enqueued rehyat_forward_phiq right before (the attention then overlaps
+// the phi_q kernel).
 static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
                                const void* q, const void* k, const void* v, void* out,
                                float* lse, const void* workspace, size_t ws_bytes,
-                               void* stream) {
+                               void* stream, bool behind_phiq) {
   g_msg[0] = 0;
   ForwardPlan pl;
   RH_TRY(forward_common_checks(d, dt, T, L, Tc, To, workspace, ws_bytes, &pl));
@@ -762,7 +781,8 @@ static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int
     ap.out = static_cast<__nv_bfloat16*>(out);
     ap.lse = lse;
     dim3 grid(BH, (rows_per_chunk + 255) / 256, pl.C);
-    return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, grid, st);
+    return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, grid, st, nullptr, nullptr,
+                                  behind_phiq);
   }
   rehyat::fp32::AttnParams ap{};
   ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
@@ -790,7 +810,8 @@ int rehyat_forward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
     return fail(REHYAT_ERR_ALIGN, "q/k/v/out not 16-byte aligned");
   RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, workspace, ws_bytes, stream));
   RH_TRY(rehyat_forward_phiq(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream));
-  return rehyat_forward_attend(d, dt, T, L, Tc, To, q, k, v, out, workspace, ws_bytes, stream);
+  return forward_attend_impl(d, dt, T, L, Tc, To, q, k, v, out, nullptr, workspace, ws_bytes,
+                             stream, true);
 }
 
 int rehyat_forward_train(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
@@ -806,7 +827,8 @@ int rehyat_forward_train(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, i
     return fail(REHYAT_ERR_ALIGN, "q/k/v/out not 16-byte aligned");
   RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, workspace, ws_bytes, stream));
   RH_TRY(rehyat_forward_phiq(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream));
-  return forward_attend_impl(d, dt, T, L, Tc, To, q, k, v, out, lse, workspace, ws_bytes, stream);
+  return forward_attend_impl(d, dt, T, L, Tc, To, q, k, v, out, lse, workspace, ws_bytes, stream,
+                             true);
 }
 
 int rehyat_backward_workspace_size(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
@@ -1029,7 +1051,10 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
   }
   RH_TRY(make_map(&ms, St, d.F, d.D, BH));
   RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mwq, st));
+  if (pl.fold_rows > 0)
+    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
   __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
+  // phi_q right before the attention, which overlaps it
   if (frames_before - pl.o > 0)  // the chunk reads a linear state
     RH_TRY(launch_featmap_tc(d, q, pl.nq, 0, pl.nq, mwq, bq, phiq, st));
   CUtensorMap mphi;
@@ -1043,10 +1068,8 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
   ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
-  if (pl.fold_rows > 0)
-    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
   RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
-                                dim3(BH, (pl.nq + 255) / 256, 1), st, &mkc, &mvc));
+                                dim3(BH, (pl.nq + 255) / 256, 1), st, &mkc, &mvc, true));
   if (pl.fold_rows > 0) {
     // the fold reads only the window and writes its own partials: it runs in the attention's
     // last wave; the state update after it waits for both
@@ -1357,7 +1380,8 @@ int rehyat_segment_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
   ap.out = static_cast<__nv_bfloat16*>(out_seg);
   const int rows_per_chunk = (Tc < ap.T ? Tc : ap.T) * L;
   return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap,
-                                dim3(BH, (rows_per_chunk + 255) / 256, pl.n_local), st);
+                                dim3(BH, (rows_per_chunk + 255) / 256, pl.n_local), st, nullptr,
+                                nullptr, true);
 }
 
 int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frames_before,
