@@ -501,10 +501,10 @@ def backward_runner(w: C.Workload, inp, dev, args) -> _Run:
     lin = sum(1 for (wf, _, _) in w.chunk_bounds() if wf > 0)
     groups = sum(1 for c in range(C_ - 1) if w.chunk_bounds()[c + 1][0] > w.chunk_bounds()[c][0])
     # per chunk dK/dV + dQ (+ linear: GEMM, phi_q grad, GEMM, r partials), row statistics,
-    # r reduction, suffix, per fold group 2 GEMM, two feature backwards (per batch 5 GEMM,
-    # feature grad, block-diagonal grad, column sums, bias grad), plus the recomputed
+    # r reduction, suffix, per fold group 2 GEMM, two feature backwards (per batch 3 GEMM: U,
+    # dx, dW; feature grad, block-diagonal grad, column sums, bias grad), plus the recomputed
     # states/phi_q/phi_k (2 weight preps, 2 feature maps, fold, scan)
-    r.launches_per_step = (2 * C_ + 4 * lin + 3 + 2 * groups + 2 * (5 * w.B + 4) + 6)
+    r.launches_per_step = (2 * C_ + 4 * lin + 3 + 2 * groups + 2 * (3 * w.B + 4) + 6)
     r.roofline_kernel = "backward pass (all launches; algorithmic FLOPs / time)"
     r.config = {"pass": "backward"}
     return r

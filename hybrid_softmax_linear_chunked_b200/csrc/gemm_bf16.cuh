@@ -6,10 +6,15 @@
 //   B is K x N, stored K-contiguous ([N][K], b_mn = 0) or N-contiguous ([K][N], b_mn = 1).
 // With split > 1 the K range is cut into `split` parts computed by separate CTAs that add their
 // partial tiles into C with fp32 atomics (C must hold the initial value; fp32 output only).
+// With b_parts = 2 the product is A (B + B2) computed as A B + A B2 in one accumulator (B2 a
+// second operand of B's shape and layout): the K loop runs twice over A, first against B, then
+// against B2.
 // One CTA computes one 128 x 128 tile of C: warp 0 streams 64-deep K slices of A and B through a
-// 4-stage TMA ring (128-byte swizzle; rows, columns and K past the matrix read zeros), warp 1
+// kStages-deep TMA ring (128-byte swizzle; rows, columns and K past the matrix read zeros), warp 1
 // issues four M128 N128 K16 MMAs per slice and owns the TMEM accumulator, warps 2-5 read the
-// accumulator back (one row per thread) and store, add to, or round into C.
+// accumulator back (one row per thread) and store, add to, or round into C.  Short K loops use
+// the 2-stage instance, whose 65 KB of shared memory lets three CTAs share an SM, so one CTA's
+// epilogue overlaps the others' loads.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -21,14 +26,14 @@ namespace gemm {
 
 using namespace sm100;
 
-constexpr int kBM = 128, kBN = 128, kBK = 64, kStages = 4;
+constexpr int kBM = 128, kBN = 128, kBK = 64;
 constexpr int kThreads = 192;
 constexpr uint32_t kTileA = kBM * kBK * 2;
 constexpr uint32_t kTileB = kBN * kBK * 2;
 constexpr uint32_t kStageBytes = kTileA + kTileB;
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024;
-
-enum Bar { kFull = 0, kEmpty = kStages, kDone = 2 * kStages, kNumBars };
+__host__ __device__ constexpr uint32_t smem_bytes(int stages) {
+  return stages * kStageBytes + 1024;
+}
 
 struct Params {
   int M, N, K;
@@ -37,7 +42,8 @@ struct Params {
   long long ldc, c_batch;  // elements
   int c_bf16, accumulate;
   float alpha;
-  int split;  // K parts (>= 1); blockIdx.z = batch * split + part
+  int split;    // K parts (>= 1); blockIdx.z = batch * split + part
+  int b_parts;  // 1, or 2: C (+)= alpha A (B + B2) (split must be 1)
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -65,16 +71,20 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
 }
 
 // grid (ceil(N / 128), ceil(M / 128), batch * split), block 192.
+template <int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
-                     const __grid_constant__ CUtensorMap tmB, const Params p) {
-  static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
+                     const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmB2, const Params p) {
+  static_assert(smem_bytes(kStages) + 256 <= 232448, "shared memory over the limit");
+  enum { kFull = 0, kEmpty = kStages, kDone = 2 * kStages, kNumBars };
   const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
   const int b = blockIdx.z / p.split, part = blockIdx.z - b * p.split;
   const int k_slices = (p.K + kBK - 1) / kBK;
   const int per_part = (k_slices + p.split - 1) / p.split;
   const int kb0 = part * per_part;
-  const int num_k = max(0, min(k_slices, kb0 + per_part) - kb0);
+  const int num_k1 = max(0, min(k_slices, kb0 + per_part) - kb0);  // slices against one B
+  const int num_k = num_k1 * p.b_parts;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ __align__(8) uint64_t bars[kNumBars];
@@ -113,9 +123,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (leader) {
         uint8_t* st = sm + s * kStageBytes;
+        const int kk0 = (kb0 + kb % num_k1) * kBK;
         mbar_arrive_expect_tx(&bars[kFull + s], kStageBytes);
-        load_operand(st, &tmA, &bars[kFull + s], p.a_mn, m0, (kb0 + kb) * kBK, b);
-        load_operand(st + kTileA, &tmB, &bars[kFull + s], p.b_mn, n0, (kb0 + kb) * kBK, b);
+        load_operand(st, &tmA, &bars[kFull + s], p.a_mn, m0, kk0, b);
+        load_operand(st + kTileA, kb < num_k1 ? &tmB : &tmB2, &bars[kFull + s], p.b_mn, n0, kk0, b);
       }
       __syncwarp();
       ++issued;

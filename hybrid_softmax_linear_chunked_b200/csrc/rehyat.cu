@@ -151,32 +151,48 @@ struct Operand {
 };
 
 // C[b] (+)= alpha A[b] B[b] with A M x K, B K x N (layouts per Operand::mn), C [M][N] with row
-// stride ldc.  Strides and bases must be 16-byte aligned (multiples of 8 elements).
+// stride ldc.  Strides and bases must be 16-byte aligned (multiples of 8 elements).  With B2
+// (same shape and layout as B, no split) the product is A (B + B2), summed in the accumulator.
 int launch_gemm(int M, int N, int K, int batch, const Operand& A, const Operand& B, void* C,
                 long long ldc, long long c_batch, bool c_bf16, bool accumulate, float alpha,
-                cudaStream_t st, int split = 1) {
+                cudaStream_t st, int split = 1, const Operand* B2 = nullptr) {
   if (split < 1 || (split > 1 && (c_bf16 || !accumulate)))
     return fail(REHYAT_ERR_ARG, "split-K GEMM needs fp32 output accumulated into C");
+  if (B2 && (split > 1 || B2->mn != B.mn))
+    return fail(REHYAT_ERR_ARG, "a two-part B needs split = 1 and one layout");
   if (M < 1 || N < 1 || K < 1 || batch < 1) return fail(REHYAT_ERR_ARG, "empty GEMM");
   if ((A.ld | A.batch_stride | B.ld | B.batch_stride) & 7)
     return fail(REHYAT_ERR_ALIGN, "GEMM operand strides must be multiples of 8 elements");
   if (!aligned16(A.ptr) || !aligned16(B.ptr) || !aligned16(C) || (!c_bf16 && ((ldc | c_batch) & 3)))
     return fail(REHYAT_ERR_ALIGN, "GEMM pointers must be 16-byte aligned");
-  CUtensorMap ma, mb;
+  if (B2 && (!aligned16(B2->ptr) || ((B2->ld | B2->batch_stride) & 7)))
+    return fail(REHYAT_ERR_ALIGN, "GEMM pointers must be 16-byte aligned");
+  CUtensorMap ma, mb, mb2;
   if (A.mn) RH_TRY(make_map_strided(&ma, A.ptr, M, K, batch, A.ld, A.batch_stride, 64, 64));
   else RH_TRY(make_map_strided(&ma, A.ptr, K, M, batch, A.ld, A.batch_stride, 64, 128));
   if (B.mn) RH_TRY(make_map_strided(&mb, B.ptr, N, K, batch, B.ld, B.batch_stride, 64, 64));
   else RH_TRY(make_map_strided(&mb, B.ptr, K, N, batch, B.ld, B.batch_stride, 64, 128));
+  if (B2) {
+    if (B2->mn) RH_TRY(make_map_strided(&mb2, B2->ptr, N, K, batch, B2->ld, B2->batch_stride, 64, 64));
+    else RH_TRY(make_map_strided(&mb2, B2->ptr, K, N, batch, B2->ld, B2->batch_stride, 64, 128));
+  } else {
+    mb2 = mb;
+  }
   rehyat::gemm::Params gp{};
   gp.M = M; gp.N = N; gp.K = K; gp.a_mn = A.mn; gp.b_mn = B.mn;
   gp.C = C; gp.ldc = ldc; gp.c_batch = c_batch; gp.c_bf16 = c_bf16; gp.accumulate = accumulate;
   gp.alpha = alpha;
   gp.split = split;
-  auto k = rehyat::gemm::gemm_bf16_kernel;
+  gp.b_parts = B2 ? 2 : 1;
+  // a K loop of at most four 64-deep slices per CTA runs on the 2-stage ring (three CTAs per SM)
+  const int slices = (int)((((K + 63) / 64) + split - 1) / split) * gp.b_parts;
+  const bool short_k = slices <= 4;
+  auto k = short_k ? rehyat::gemm::gemm_bf16_kernel<2> : rehyat::gemm::gemm_bf16_kernel<4>;
+  const uint32_t smem = rehyat::gemm::smem_bytes(short_k ? 2 : 4);
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)rehyat::gemm::kSmemBytes), "gemm attr"));
+                                         (int)smem), "gemm attr"));
   dim3 grid((N + 127) / 128, (M + 127) / 128, batch * split);
-  k<<<grid, rehyat::gemm::kThreads, rehyat::gemm::kSmemBytes, st>>>(ma, mb, gp);
+  k<<<grid, rehyat::gemm::kThreads, smem, st>>>(ma, mb, mb2, gp);
   return cuda_check(cudaGetLastError(), "gemm launch");
 }
 
@@ -619,11 +635,11 @@ int feature_backward(const rehyat_dims& d, long long N, long long r0, long long 
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   for (int b = 0; b < d.B; ++b) {
     const long long bo = (long long)b * H * N;  // first row of batch b
-    for (int part = 0; part < 2; ++part)       // U = x Wbd_hi^T + x Wbd_lo^T
-      RH_TRY(launch_gemm((int)rows, (int)F, (int)D, H,
-                         Operand{xb + (bo + r0) * D, D, N * D, false},
-                         Operand{Wbd + part * F * D, D, 2 * F * D, false},
-                         U + (bo + r0) * F, F, N * F, false, part > 0, 1.f, st));
+    // U = x (Wbd_hi + Wbd_lo)^T, both parts in one accumulator
+    const Operand lo{Wbd + F * D, D, 2 * F * D, false};
+    RH_TRY(launch_gemm((int)rows, (int)F, (int)D, H, Operand{xb + (bo + r0) * D, D, N * D, false},
+                       Operand{Wbd, D, 2 * F * D, false}, U + (bo + r0) * F, F, N * F, false,
+                       false, 1.f, st, 1, &lo));
   }
   rehyat::bwd::feat_grad_kernel<<<
       dim3((unsigned)((rows + rehyat::bwd::kFeatRows - 1) / rehyat::bwd::kFeatRows), BH), d.F, 0,
@@ -632,11 +648,11 @@ int feature_backward(const rehyat_dims& d, long long N, long long r0, long long 
   RH_TRY(cuda_check(cudaMemsetAsync(dWbd, 0, (size_t)H * F * D * 4, st), "memset"));
   for (int b = 0; b < d.B; ++b) {
     const long long bo = (long long)b * H * N;
-    for (int part = 0; part < 2; ++part)       // dx += du Wbd_hi + du Wbd_lo
-      RH_TRY(launch_gemm((int)rows, (int)D, (int)F, H,
-                         Operand{DU + (bo + r0) * F, F, N * F, false},
-                         Operand{Wbd + part * F * D, D, 2 * F * D, true},
-                         dx + (bo + r0) * D, D, N * D, false, true, 1.f, st));
+    // dx += du (Wbd_hi + Wbd_lo), both parts in one accumulator
+    const Operand lo{Wbd + F * D, D, 2 * F * D, true};
+    RH_TRY(launch_gemm((int)rows, (int)D, (int)F, H, Operand{DU + (bo + r0) * F, F, N * F, false},
+                       Operand{Wbd, D, 2 * F * D, true}, dx + (bo + r0) * D, D, N * D, false,
+                       true, 1.f, st, 1, &lo));
     // dWbd += du^T x over this batch's rows
     RH_TRY(launch_gemm((int)F, (int)D, (int)rows, H, Operand{DU + (bo + r0) * F, F, N * F, true},
                        Operand{xb + (bo + r0) * D, D, N * D, true}, dWbd, D, F * D, false, true,
