@@ -155,10 +155,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
 
   // ---- chunk geometry (uniform over the CTA) ----
-  // grid (BH, tile pairs, chunks), dispatched x fastest: within a chunk the lone last tile of an
-  // odd tile count (the shortest CTAs) come last, and chunk 0, whose window is shortest, last
-  // of all
-  const int bh = blockIdx.x, c = (blockIdx.z + 1) % gridDim.z, h = bh % p.H;
+  // grid (tile-pair slots, BH, chunks).  Within one chunk the linear CTA index walks the full
+  // tile pairs of one (b, h) after another, so the CTAs in flight share few K/V windows in L2;
+  // the lone last tiles of an odd tile count (the shortest CTAs) follow, one per (b, h).  Chunk
+  // 0, whose window is shortest, is dispatched last.
+  const int c = (blockIdx.z + 1) % gridDim.z;
   const int gs = p.frames_before + c * p.Tc;
   const int ge = min(gs + p.Tc, p.frames_before + p.T);
   const int gw = max(0, gs - p.To);
@@ -167,8 +168,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int k_row0 = (gw - p.kv_frame0) * p.L;
   const int nk = (ge - gw) * p.L;
   const bool has_linear = gw > 0;
-  const int tile_row0 = blockIdx.y * 2 * kBM;
-  if (tile_row0 >= nq) return;
+  const int n_full = ((nq + kBM - 1) / kBM) / 2, n_lone = ((nq + kBM - 1) / kBM) & 1;
+  const int n_bh = gridDim.y;
+  const int lin = blockIdx.x + gridDim.x * blockIdx.y;
+  int bh, pair;
+  if (lin < n_full * n_bh) {
+    bh = lin / n_full;
+    pair = lin - bh * n_full;
+  } else if (lin < (n_full + n_lone) * n_bh) {
+    bh = lin - n_full * n_bh;
+    pair = n_full;
+  } else {
+    return;  // a slot past this chunk's tiles (its chunk is shorter than the longest)
+  }
+  const int h = bh % p.H;
+  const int tile_row0 = pair * 2 * kBM;
   const bool has_t1 = tile_row0 + kBM < nq;
   // key tiles: n_kc from the carried segment (rows [0, kv_split) of the window), then the rest
   const int kv_split = p.kv_split;

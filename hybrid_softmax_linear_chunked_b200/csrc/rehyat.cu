@@ -796,7 +796,7 @@ static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int
     ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
     ap.out = static_cast<__nv_bfloat16*>(out);
     ap.lse = lse;
-    dim3 grid(BH, (rows_per_chunk + 255) / 256, pl.C);
+    dim3 grid((rows_per_chunk + 255) / 256, BH, pl.C);
     return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, grid, st, nullptr, nullptr,
                                   behind_phiq);
   }
@@ -1085,7 +1085,7 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
   RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
-                                dim3(BH, (pl.nq + 255) / 256, 1), st, &mkc, &mvc, true));
+                                dim3((pl.nq + 255) / 256, BH, 1), st, &mkc, &mvc, true));
   if (pl.fold_rows > 0) {
     // the fold reads only the window and writes its own partials: it runs in the attention's
     // last wave; the state update after it waits for both
@@ -1396,7 +1396,7 @@ int rehyat_segment_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
   ap.out = static_cast<__nv_bfloat16*>(out_seg);
   const int rows_per_chunk = (Tc < ap.T ? Tc : ap.T) * L;
   return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap,
-                                dim3(BH, (rows_per_chunk + 255) / 256, pl.n_local), st, nullptr,
+                                dim3((rows_per_chunk + 255) / 256, BH, pl.n_local), st, nullptr,
                                 nullptr, true);
 }
 
@@ -1456,7 +1456,7 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
-  RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3(nbh, (pl.nq + 255) / 256, 1),
+  RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3((pl.nq + 255) / 256, nbh, 1),
                                  st));
   if (pl.fold_rows > 0) {
     RH_TRY(prepare_blockdiag(d, Wk, Wkbd, &mwk, st));
