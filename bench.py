@@ -619,14 +619,16 @@ def stream_runner(w: C.Workload, inp, dev, args) -> _Run:
         fold = max(0, max(0, e - nxt) - wf) * L
         step_f += (2.0 * nq * F + (2.0 * nq * D * F / w.G) if wf > 0 else 0.0)
         step_f += fold * (2.0 * F * D + F + 2.0 * D * F / w.G)
-        launches += 5 + (1 if wf > 0 else 0) + (3 if fold > 0 else 0)
+        # S transpose, W_q block-diagonal, attention; [phi_q]; [W_k block-diagonal, fold, state
+        # add]; the carry update is a device copy, or 2 gathers when the chunk is shorter
+        cap = max(ov_ for _, ov_ in sched)
+        launches += (3 + (1 if wf > 0 else 0) + (3 if fold > 0 else 0)
+                     + (2 if 0 < e - s < cap else 0))
     r.attn_flops = attn * w.B * w.H
     r.step_flops = (attn + step_f) * w.B * w.H
     r.step, r.e2e_step = step, e2e_step
     r.h2d = sum(x.numel() * x.element_size() for c in host for x in c)
     r.d2h = sum(o.numel() * o.element_size() for o in host_out)
-    # per call: K and V window gathers, S transpose, W_q block-diagonal, [phi_q], attention,
-    # [W_k block-diagonal, fold, state add]
     r.launches_per_step = launches
     r.roofline_kernel = "whole streaming step (attention FLOPs / step time)"
     r.config = {"mode": "stream", "calls_per_step": len(bounds),

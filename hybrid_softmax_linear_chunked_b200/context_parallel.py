@@ -37,6 +37,22 @@ def split_chunks(C: int, world: int) -> list[tuple[int, int]]:
     return out
 
 
+def plan_ranks(T: int, Tc: int, To: int, world: int):
+    """Chunk ranges and (s0, s1, h0) bounds of every rank.  Raises ValueError when a rank holds
+    fewer frames than the overlap the next rank takes from it (its halo must come from one
+    rank)."""
+    C = (T + Tc - 1) // Tc
+    ranges = split_chunks(C, world)
+    bounds = [rb.segment_bounds(T, Tc, To, c0, c1) for c0, c1 in ranges]
+    for r in range(world - 1):
+        s0, s1, _ = bounds[r]
+        n0, _, nh = bounds[r + 1]
+        if s1 - s0 < n0 - nh:
+            raise ValueError(f"rank {r} holds {s1 - s0} frames, fewer than the {n0 - nh} overlap "
+                             "frames the next rank needs")
+    return ranges, bounds
+
+
 class ContextParallel:
     """The forward of one sequence of T frames over the ranks of `group` (or one process)."""
 
@@ -51,12 +67,7 @@ class ContextParallel:
         self.Wq, self.bq, self.Wk, self.bk = Wq, bq, Wk, bk
         self.T, self.L, self.Tc, self.To, self.P, self.phi = T, frame_tokens, Tc, To, P, phi
         self.C = (T + Tc - 1) // Tc
-        self.ranges = split_chunks(self.C, self.world)
-        self.bounds = [rb.segment_bounds(T, Tc, To, c0, c1) for c0, c1 in self.ranges]
-        for r, (s0, s1, _) in enumerate(self.bounds):
-            if r + 1 < self.world and s1 - s0 < self.halo_frames(r + 1):
-                raise ValueError(f"rank {r} holds {s1 - s0} frames, fewer than the {To} overlap "
-                                 "frames the next rank needs")
+        self.ranges, self.bounds = plan_ranks(T, Tc, To, self.world)
         self.c0, self.c1 = self.ranges[self.rank]
         self.s0, self.s1, self.h0 = self.bounds[self.rank]
         self._ws = None

@@ -146,15 +146,16 @@ int rehyat_chunk_forward(rehyat_dims d, rehyat_dtype dt, int frame_tokens, int f
                          const float* bk, float* S, float* Z, void* out, void* workspace,
                          size_t ws_bytes, void* stream);
 
-/* The streaming step with the overlap frames kept by the library's own copy kernel: the caller
- * passes only the chunk (k, v [B,H,chunk_frames*L,D]) and a carry buffer per tensor
- * (k_carry, v_carry [B,H,carry_frames*L,D], inout, same dtype): the last carry_frames frames of
- * K and V seen so far, right-aligned (after f frames, only the last min(f, carry_frames) are
- * meaningful).  The call builds the window [the last min(To, frames_before) carried frames |
- * the chunk] in the workspace, runs rehyat_chunk_forward_sched on it (To_next as there), and
- * updates the carry to the last carry_frames frames of (carry ++ chunk).  Needs To <=
- * carry_frames; a zero-initialised carry is fine for the first call.  The state between calls
- * is then S, Z and the carry: the method's recurrent state (page §2.3).  Workspace:
+/* The streaming step with the overlap frames kept by the library: the caller passes only the
+ * chunk (k, v [B,H,chunk_frames*L,D]) and a carry buffer per tensor (k_carry, v_carry
+ * [B,H,carry_frames*L,D], inout, same dtype): the last carry_frames frames of K and V seen so
+ * far, right-aligned (after f frames, only the last min(f, carry_frames) are meaningful).  The
+ * result is that of rehyat_chunk_forward_sched (To_next as there) on the window [the last
+ * min(To, frames_before) carried frames | the chunk]; bf16 kernels read that window in place
+ * from the carry and the chunk, fp32 assembles it in the workspace.  Afterwards the carry holds
+ * the last carry_frames frames of (carry ++ chunk).  Needs To <= carry_frames; a
+ * zero-initialised carry is fine for the first call.  The state between calls is then S, Z and
+ * the carry: the method's recurrent state (page §2.3).  Workspace:
  * rehyat_chunk_carry_workspace_size with the largest chunk_frames and To of the stream. */
 int rehyat_chunk_carry_workspace_size(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
                                       int chunk_frames, int To, int carry_frames, size_t* bytes);

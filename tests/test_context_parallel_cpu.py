@@ -13,7 +13,8 @@ import torch
 import torch.multiprocessing as mp
 
 from hybrid_softmax_linear_chunked_b200 import binding as rb
-from hybrid_softmax_linear_chunked_b200.context_parallel import ContextParallel, split_chunks
+from hybrid_softmax_linear_chunked_b200.context_parallel import (ContextParallel, plan_ranks,
+                                                                 split_chunks)
 from oracle import rehyat_oracle as O
 
 L, T, Tc, To, P = 6, 11, 2, 1, 2   # 6 chunks, the last one frame long
@@ -165,3 +166,15 @@ def test_segment_bounds():
     assert rb.segment_bounds(11, 2, 1, 2, 4) == (4, 8, 3)
     assert rb.segment_bounds(11, 2, 1, 0, 2) == (0, 4, 0)
     assert rb.segment_bounds(11, 2, 3, 5, 6) == (10, 11, 7)   # ragged last chunk, wide halo
+
+
+def test_plan_ranks():
+    ranges, bounds = plan_ranks(11, 2, 1, 3)
+    assert ranges == [(0, 2), (2, 4), (4, 6)]
+    assert bounds == [(0, 4, 0), (4, 8, 3), (8, 11, 7)]
+    # one frame per rank cannot supply a two-frame halo
+    with pytest.raises(ValueError):
+        plan_ranks(6, 1, 2, 6)
+    # To wider than a chunk is fine while each rank holds enough frames
+    ranges, bounds = plan_ranks(12, 2, 3, 3)
+    assert bounds[1] == (4, 8, 1) and bounds[2] == (8, 12, 5)
