@@ -490,17 +490,19 @@ def backward_runner(w: C.Workload, inp, dev, args) -> _Run:
 
     host = [x.pin_memory() for x in (inp.q, inp.k, inp.v, inp.Wq, inp.bq, inp.Wk, inp.bk)]
     host += [out.cpu().pin_memory(), lse.cpu().pin_memory(), dout.cpu().pin_memory()]
-    grads_h = {}
+    # end to end: every step uploads q, k, v, the weights, out, the row statistics and dL/dout
+    # and downloads the seven gradients; copies overlap the computation (HostPipeline)
+    shapes = {"dq": q.shape, "dk": q.shape, "dv": q.shape, "dWq": Wq.shape, "dWk": Wk.shape,
+              "dbq": (w.H, w.F), "dbk": (w.H, w.F)}
+    grad_like = [torch.empty(shapes[n], dtype=torch.float32, device=dev) for n in rb.GRAD_NAMES]
+    grads_h = [torch.empty(g.shape, dtype=g.dtype).pin_memory() for g in grad_like]
 
-    def e2e_step():
-        t = [x.to(dev, non_blocking=True) for x in host]
-        g = rb.backward(*t[:7], t[7], t[8], t[9], workspace=ws, **kw)
-        for name, x in g.items():
-            if name not in grads_h:
-                grads_h[name] = torch.empty(x.shape, dtype=x.dtype).pin_memory()
-            grads_h[name].copy_(x, non_blocking=True)
+    def e2e_compute(i, ins, outs):
+        rb.backward(*ins, workspace=ws, grads=dict(zip(rb.GRAD_NAMES, outs)), **kw)
 
-    r.step, r.e2e_step = step, e2e_step
+    pipe = HostPipeline(e2e_compute, host, grad_like, dev)
+    r.step = step
+    r.e2e_run = lambda n: pipe.run([host] * n, [grads_h] * n)
     r.h2d = sum(x.numel() * x.element_size() for x in host)
     r.d2h = 3 * q.numel() * 4 + 2 * Wq.numel() * 4 + 2 * w.H * w.F * 4
     r.attn_flops = w.backward_flops()

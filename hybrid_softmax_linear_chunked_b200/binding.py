@@ -439,10 +439,15 @@ def backward_workspace_size(d: Dims, dtype_code: int, T: int, L_: int, Tc: int, 
     return n.value
 
 
+GRAD_NAMES = ("dq", "dk", "dv", "dWq", "dbq", "dWk", "dbk")
+
+
 def backward(q, k, v, Wq, bq, Wk, bk, out, lse, dout, *, P: int, phi: int = 0,
-             frame_tokens: int, Tc: int, To: int, workspace: torch.Tensor | None = None) -> dict:
+             frame_tokens: int, Tc: int, To: int, workspace: torch.Tensor | None = None,
+             grads: dict | None = None) -> dict:
     """Gradients of sum(dout * out) for every input: dict with dq, dk, dv [B,H,N,D], dWq, dWk
-    [H,G,F/G,D/G], dbq, dbk [H,F] (fp32)."""
+    [H,G,F/G,D/G], dbq, dbk [H,F] (fp32).  `grads` may hold those buffers (written, not added
+    to)."""
     lib = load()
     dev = _dev(q, k, v, Wq, bq, Wk, bk, out, lse, dout)
     d = dims_of(q, Wq, P, phi)
@@ -450,11 +455,17 @@ def backward(q, k, v, Wq, bq, Wk, bk, out, lse, dout, *, P: int, phi: int = 0,
     T = N // frame_tokens
     code = _dtype_code(q)
     ws = _workspace(backward_workspace_size(d, code, T, frame_tokens, Tc, To), dev, workspace)
-    g = {n: torch.empty(q.shape, dtype=torch.float32, device=dev) for n in ("dq", "dk", "dv")}
-    g["dWq"] = torch.empty(Wq.shape, dtype=torch.float32, device=dev)
-    g["dWk"] = torch.empty(Wk.shape, dtype=torch.float32, device=dev)
-    g["dbq"] = torch.empty(d.H, d.F, dtype=torch.float32, device=dev)
-    g["dbk"] = torch.empty(d.H, d.F, dtype=torch.float32, device=dev)
+    shapes = {"dq": q.shape, "dk": q.shape, "dv": q.shape, "dWq": Wq.shape, "dWk": Wk.shape,
+              "dbq": (d.H, d.F), "dbk": (d.H, d.F)}
+    g = {}
+    for n in GRAD_NAMES:
+        t = grads.get(n) if grads is not None else None
+        if t is None:
+            t = torch.empty(shapes[n], dtype=torch.float32, device=dev)
+        elif tuple(t.shape) != tuple(shapes[n]) or t.dtype != torch.float32:
+            raise ValueError(f"grads[{n!r}] must be float32 of shape {tuple(shapes[n])}")
+        g[n] = t
+    _dev(*g.values())
     _check(lib.rehyat_backward(d, code, T, frame_tokens, Tc, To, _ptr(q), _ptr(k), _ptr(v),
                                _ptr(Wq), _ptr(bq), _ptr(Wk), _ptr(bk), _ptr(out), _ptr(lse),
                                _ptr(dout), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),

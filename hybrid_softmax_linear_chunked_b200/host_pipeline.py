@@ -20,15 +20,18 @@ import torch
 class HostPipeline:
     """`compute(i, dev_inputs, dev_out)` enqueues step i on the current stream; `in_like` and
     `out_like` give the shapes and dtypes of one step's device inputs and output (the same for
-    every step)."""
+    every step).  `out_like` may be a list: `dev_out` and each step's host output are then lists
+    in the same order."""
 
-    def __init__(self, compute: Callable[[int, list, torch.Tensor], None],
-                 in_like: Sequence[torch.Tensor], out_like: torch.Tensor, device):
+    def __init__(self, compute: Callable[[int, list, object], None],
+                 in_like: Sequence[torch.Tensor], out_like, device):
         self.compute = compute
         self.device = torch.device(device)
+        self.multi = not isinstance(out_like, torch.Tensor)
+        outs = list(out_like) if self.multi else [out_like]
         self.inputs = [[torch.empty(t.shape, dtype=t.dtype, device=self.device) for t in in_like]
                        for _ in range(2)]
-        self.outputs = [torch.empty(out_like.shape, dtype=out_like.dtype, device=self.device)
+        self.outputs = [[torch.empty(t.shape, dtype=t.dtype, device=self.device) for t in outs]
                         for _ in range(2)]
         self.up = torch.cuda.Stream(self.device)
         self.down = torch.cuda.Stream(self.device)
@@ -45,9 +48,9 @@ class HostPipeline:
                 dst.copy_(src, non_blocking=True)
             self.ev_up[b].record(self.up)
 
-    def run(self, host_inputs: Sequence[Sequence[torch.Tensor]],
-            host_outputs: Sequence[torch.Tensor]) -> None:
-        """Step i reads host_inputs[i] (pinned tensors) and writes host_outputs[i] (pinned)."""
+    def run(self, host_inputs: Sequence[Sequence[torch.Tensor]], host_outputs: Sequence) -> None:
+        """Step i reads host_inputs[i] (pinned tensors) and writes host_outputs[i] (pinned; a list
+        when the outputs are)."""
         n = len(host_inputs)
         if len(host_outputs) != n:
             raise ValueError("one host output per step")
@@ -65,11 +68,14 @@ class HostPipeline:
             main.wait_event(self.ev_up[b])
             if i >= 2:
                 main.wait_event(self.ev_down[b])
-            self.compute(i, self.inputs[b], self.outputs[b])
+            outs = self.outputs[b]
+            self.compute(i, self.inputs[b], outs if self.multi else outs[0])
             self.ev_comp[b].record(main)
             with torch.cuda.stream(self.down):
                 self.down.wait_event(self.ev_comp[b])
-                host_outputs[i].copy_(self.outputs[b], non_blocking=True)
+                dst = host_outputs[i] if self.multi else [host_outputs[i]]
+                for h, d in zip(dst, self.outputs[b]):
+                    h.copy_(d, non_blocking=True)
                 self.ev_down[b].record(self.down)
         main.wait_event(self.ev_down[(n - 1) % 2])
         if n >= 2:

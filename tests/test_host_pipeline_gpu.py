@@ -44,3 +44,36 @@ def test_pipeline_outputs_match_direct_forward(dev, n):
     for i in range(n):
         want = rb.forward(*(x.to(dev) for x in batches[i]), **kw).cpu()
         assert torch.equal(outs[i], want), f"step {i}"
+
+
+def test_pipeline_with_several_outputs(dev):
+    """The backward through the pipeline (ten inputs, seven gradients per step) against direct
+    calls.  dq, dk, dv are deterministic; the weight and bias gradients sum split-K partials with
+    fp32 atomics, so their order of additions may differ."""
+    w = C.Workload("pipe", B=1, H=2, D=128, T=7, frame_h=10, frame_w=20, Tc=3, To=1, P=2, F=128,
+                   G=8, dtype="bf16", seed=3)
+    kw = dict(P=w.P, frame_tokens=w.frame_tokens, Tc=w.Tc, To=w.To)
+    batches = []
+    for i in range(3):
+        inp = make_inputs(w, seed=200 + i)
+        t = [x.to(dev) for x in (inp.q, inp.k, inp.v, inp.Wq, inp.bq, inp.Wk, inp.bk)]
+        out, lse = rb.forward_train(*t, **kw)
+        dout = torch.randn(out.shape, generator=torch.Generator().manual_seed(i)).to(torch.bfloat16)
+        batches.append([x.cpu().pin_memory() for x in t] +
+                       [out.cpu().pin_memory(), lse.cpu().pin_memory(), dout.pin_memory()])
+    ref = [rb.backward(*(x.to(dev) for x in bt), **kw) for bt in batches]
+    like = [ref[0][n] for n in rb.GRAD_NAMES]
+    host_out = [[torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in like] for _ in batches]
+    pipe = HostPipeline(
+        lambda i, ins, outs: rb.backward(*ins, grads=dict(zip(rb.GRAD_NAMES, outs)), **kw),
+        batches[0], like, dev)
+    pipe.run(batches, host_out)
+    torch.cuda.current_stream(dev).synchronize()
+    rb.sync_status(dev)
+    for i in range(3):
+        for n, got in zip(rb.GRAD_NAMES, host_out[i]):
+            want = ref[i][n].cpu()
+            if n in ("dq", "dk", "dv"):
+                assert torch.equal(got, want), f"step {i} {n}"
+            else:
+                torch.testing.assert_close(got, want, rtol=1e-5, atol=1e-6)
