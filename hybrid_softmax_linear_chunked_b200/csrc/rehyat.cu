@@ -1044,10 +1044,12 @@ struct WindowSrc {
 
 // One bf16 chunk step ("ReHyAt overview" page §2.2-§2.3 and §5.2): S^T copy, phi_q, the
 // attention with the state readout, then the fold of the frames leaving the window into S, Z.
+// With `cc`, the next carry of K and V is copied in the same closing launch as the state add.
 static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int chunk_frames,
                            int To, const ChunkPlan& pl, const void* q, const WindowSrc& w,
                            const float* Wq, const float* bq, const float* Wk, const float* bk,
-                           float* S, float* Z, void* out, uint8_t* ws, cudaStream_t st) {
+                           float* S, float* Z, void* out, uint8_t* ws, cudaStream_t st,
+                           const rehyat::state::CarryCopy* cc = nullptr) {
   const int BH = d.B * d.H;
   __nv_bfloat16* St = reinterpret_cast<__nv_bfloat16*>(ws + pl.St);
   float* dS = reinterpret_cast<float*>(ws + pl.dS);
@@ -1095,8 +1097,18 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
     fp.seg_row0 = w.carry_row0;
     fp.splits = pl.splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
     RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(pl.splits, 1, BH), st, &mkc, &mvc, true));
-    rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
-        dS, dZ, pl.splits, d.F, d.D, S, Z);
+  }
+  const int n_add = pl.fold_rows > 0 ? (d.F * d.D + 255) / 256 : 0;
+  if (cc && cc->n_vec > 0) {
+    long long n_copy = (2 * cc->n_vec + 255) / 256;
+    if (n_copy > 16) n_copy = 16;
+    rehyat::state::state_add_carry_kernel<<<dim3((unsigned)(n_add + n_copy), BH), 256, 0, st>>>(
+        dS, dZ, pl.splits, d.F, d.D, S, Z, n_add, *cc);
+    return cuda_check(cudaGetLastError(), "state add and carry launch");
+  }
+  if (n_add > 0) {
+    rehyat::state::state_add_kernel<<<dim3(n_add, BH), 256, 0, st>>>(dS, dZ, pl.splits, d.F, d.D,
+                                                                     S, Z);
     RH_TRY(cuda_check(cudaGetLastError(), "state add launch"));
   }
   return REHYAT_OK;
@@ -1255,23 +1267,20 @@ int rehyat_chunk_forward_carry(rehyat_dims d, rehyat_dtype dt, int L, int frames
                   pl.step_bytes);
     const WindowSrc w{k, v, (long long)chunk_frames * L, k_carry, v_carry,
                       (long long)carry_frames * L, ov * L, (carry_frames - ov) * L};
+    // the next carry, after every read of the old one (stream order): the last carry_frames
+    // frames of (carry ++ chunk); a chunk at least that long supplies all of them, copied in
+    // the step's closing launch
+    if (chunk_frames >= carry_frames) {
+      const long long fv = (long long)(frame_bytes / 16);  // 16-byte vectors per frame
+      const rehyat::state::CarryCopy cc{static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+                                        static_cast<uint4*>(k_carry), static_cast<uint4*>(v_carry),
+                                        chunk_frames * fv, (chunk_frames - carry_frames) * fv,
+                                        carry_frames * fv};
+      return chunk_step_bf16(d, L, frames_before, chunk_frames, To, cpl, q, w, Wq, bq, Wk, bk, S,
+                             Z, out, ws + pl.step, st, &cc);
+    }
     RH_TRY(chunk_step_bf16(d, L, frames_before, chunk_frames, To, cpl, q, w, Wq, bq, Wk, bk, S, Z,
                            out, ws + pl.step, st));
-    // the next carry, after every read of the old one (stream order): the last carry_frames
-    // frames of (carry ++ chunk)
-    if (carry_frames == 0) return REHYAT_OK;
-    if (chunk_frames >= carry_frames) {
-      for (int t = 0; t < 2; ++t) {
-        const uint8_t* src = static_cast<const uint8_t*>(t ? v : k) +
-                             (size_t)(chunk_frames - carry_frames) * frame_bytes;
-        RH_TRY(cuda_check(cudaMemcpy2DAsync(t ? v_carry : k_carry, carry_frames * frame_bytes, src,
-                                            chunk_frames * frame_bytes,
-                                            carry_frames * frame_bytes, BH,
-                                            cudaMemcpyDeviceToDevice, st),
-                          "carry copy"));
-      }
-      return REHYAT_OK;
-    }
     RH_TRY(gather(false));
     return copy_back();
   }

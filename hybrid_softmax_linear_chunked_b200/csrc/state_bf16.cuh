@@ -419,13 +419,11 @@ __global__ void __launch_bounds__(256) state_sum_kernel(const float* __restrict_
   }
 }
 
-// S[bh] += sum_s dS[bh][0][s], Z likewise.  grid (ceil(F*D/256), BH), block 256.
-__global__ void __launch_bounds__(256) state_add_kernel(const float* __restrict__ dS,
-                                                        const float* __restrict__ dZ, int splits,
-                                                        int F, int D, float* __restrict__ S,
-                                                        float* __restrict__ Z) {
-  const int bh = blockIdx.y;
-  const int e = blockIdx.x * 256 + threadIdx.x;
+// Element e of (b, h) bh: S[bh] += sum_s dS[bh][0][s], Z likewise.
+__device__ __forceinline__ void state_add_element(const float* __restrict__ dS,
+                                                  const float* __restrict__ dZ, int splits, int F,
+                                                  int D, float* __restrict__ S,
+                                                  float* __restrict__ Z, int bh, int e) {
   if (e < F * D) {
     float a = S[(size_t)bh * F * D + e];
     for (int s = 0; s < splits; ++s) a += dS[((size_t)bh * splits + s) * F * D + e];
@@ -435,6 +433,49 @@ __global__ void __launch_bounds__(256) state_add_kernel(const float* __restrict_
     float z = Z[(size_t)bh * F + e];
     for (int s = 0; s < splits; ++s) z += dZ[((size_t)bh * splits + s) * F + e];
     Z[(size_t)bh * F + e] = z;
+  }
+}
+
+// S[bh] += sum_s dS[bh][0][s], Z likewise.  grid (ceil(F*D/256), BH), block 256.
+__global__ void __launch_bounds__(256) state_add_kernel(const float* __restrict__ dS,
+                                                        const float* __restrict__ dZ, int splits,
+                                                        int F, int D, float* __restrict__ S,
+                                                        float* __restrict__ Z) {
+  state_add_element(dS, dZ, splits, F, D, S, Z, blockIdx.y, blockIdx.x * 256 + threadIdx.x);
+}
+
+// The streaming step's closing launch: the state add above (blocks [0, n_add)) and the next
+// carry of K and V (the remaining blocks): per (b, h), n_vec 16-byte vectors from
+// src[bh * src_stride + src_off ..] to dst[bh * n_vec ..], K then V.  grid (n_add + n_copy, BH),
+// block 256.  The carry copy reads the chunk, which the attention and the fold read too; it
+// writes the carry, which they read as well, so it must run after both (stream order).
+struct CarryCopy {
+  const uint4* k_src;
+  const uint4* v_src;
+  uint4* k_dst;
+  uint4* v_dst;
+  long long src_stride, src_off, n_vec;  // in 16-byte vectors
+};
+
+__global__ void __launch_bounds__(256) state_add_carry_kernel(const float* __restrict__ dS,
+                                                              const float* __restrict__ dZ,
+                                                              int splits, int F, int D,
+                                                              float* __restrict__ S,
+                                                              float* __restrict__ Z, int n_add,
+                                                              const CarryCopy cc) {
+  const int bh = blockIdx.y;
+  if ((int)blockIdx.x < n_add) {
+    state_add_element(dS, dZ, splits, F, D, S, Z, bh, blockIdx.x * 256 + threadIdx.x);
+    return;
+  }
+  const long long stride = (long long)(gridDim.x - n_add) * 256;
+  for (long long i = (long long)(blockIdx.x - n_add) * 256 + threadIdx.x; i < 2 * cc.n_vec;
+       i += stride) {
+    const bool is_v = i >= cc.n_vec;
+    const long long j = is_v ? i - cc.n_vec : i;
+    const uint4* src = is_v ? cc.v_src : cc.k_src;
+    uint4* dst = is_v ? cc.v_dst : cc.k_dst;
+    dst[bh * cc.n_vec + j] = src[bh * cc.src_stride + cc.src_off + j];
   }
 }
 

