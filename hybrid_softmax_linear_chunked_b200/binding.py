@@ -144,6 +144,49 @@ def _dev(*ts: torch.Tensor) -> torch.device:
     return dev
 
 
+def _shape(t: torch.Tensor | None, shape, what: str) -> None:
+    """The library reads exactly the sizes the other arguments imply; a tensor of another shape
+    is refused here, before anything is enqueued."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _frames(n_rows: int, frame_tokens: int, what: str) -> int:
+    if frame_tokens < 1 or n_rows % frame_tokens:
+        raise ValueError(f"{what}: {n_rows} rows are not a whole number of frames of "
+                         f"{frame_tokens} tokens")
+    return n_rows // frame_tokens
+
+
+def _check_x_w(x: torch.Tensor, W: torch.Tensor, b: torch.Tensor | None, what: str) -> None:
+    """x [B,H,n,D]; W [H,G,F/G,D/G]; b [H,F] or None."""
+    if x.dim() != 4:
+        raise ValueError(f"{what} must be [B,H,rows,D], got {tuple(x.shape)}")
+    if W.dim() != 4 or W.shape[0] != x.shape[1] or W.shape[1] * W.shape[3] != x.shape[3]:
+        raise ValueError(f"feature-map weights must be [H,G,F/G,D/G] for {what} of shape "
+                         f"{tuple(x.shape)}, got {tuple(W.shape)}")
+    _shape(b, (W.shape[0], W.shape[1] * W.shape[2]), "feature-map bias")
+
+
+def _check_step(q, k, v, Wq, bq, Wk, bk, S, Z, out, frame_tokens: int, kv_frames: int | None,
+                what_kv: str) -> int:
+    """Shapes of a streaming step: q [B,H,cf*L,D]; k, v [B,H,kv_frames*L,D] (the chunk's own
+    frames when kv_frames is None); S [B,H,F,D], Z [B,H,F]; out like q.  Returns cf."""
+    _check_x_w(q, Wq, bq, "q")
+    _check_x_w(q, Wk, bk, "q")
+    _shape(Wk, Wq.shape, "Wk")
+    cf = _frames(q.shape[2], frame_tokens, "q")
+    B, H, _, D = q.shape
+    F = Wq.shape[1] * Wq.shape[2]
+    rows = (cf if kv_frames is None else kv_frames) * frame_tokens
+    _shape(k, (B, H, rows, D), what_kv)
+    _shape(v, (B, H, rows, D), what_kv.replace("k", "v", 1))
+    _shape(S, (B, H, F, D), "S")
+    _shape(Z, (B, H, F), "Z")
+    _shape(out, q.shape, "out")
+    return cf
+
+
 def _weights(W: torch.Tensor, b: torch.Tensor | None):
     if W.dtype != torch.float32 or (b is not None and b.dtype != torch.float32):
         raise TypeError("feature-map weights and biases are fp32")
@@ -199,6 +242,11 @@ def forward(q, k, v, Wq, bq, Wk, bk, *, P: int, phi: int = 0, frame_tokens: int,
             out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
     """Hybrid attention over a whole sequence: q, k, v [B,H,T*frame_tokens,D] -> out."""
     lib = load()
+    _check_x_w(q, Wq, bq, "q")
+    _check_x_w(q, Wk, bk, "q")
+    _shape(Wk, Wq.shape, "Wk")
+    for t, n in ((k, "k"), (v, "v"), (out, "out")):
+        _shape(t, q.shape, n)
     dev = _dev(q, k, v, Wq, bq, Wk, bk)
     _weights(Wq, bq), _weights(Wk, bk)
     d = dims_of(q, Wq, P, phi)
@@ -238,6 +286,14 @@ def segment_states(k_seg, v_seg, Wk, bk, *, T: int, c0: int, c1: int, P: int, ph
     k_seg, v_seg [B,H,(s1-h0)*frame_tokens,D] bf16 (halo frames first).  Fills `workspace` with
     the segment's folds and returns their sum (S_seg [B,H,F,D], Z_seg [B,H,F] fp32)."""
     lib = load()
+    _check_x_w(k_seg, Wk, bk, "k_seg")
+    s0, s1, h0 = segment_bounds(T, Tc, To, c0, c1)
+    B, H, _, D = k_seg.shape
+    F = Wk.shape[1] * Wk.shape[2]
+    _shape(k_seg, (B, H, (s1 - h0) * frame_tokens, D), "k_seg")
+    _shape(v_seg, k_seg.shape, "v_seg")
+    _shape(S_seg, (B, H, F, D), "S_seg")
+    _shape(Z_seg, (B, H, F), "Z_seg")
     dev = _dev(k_seg, v_seg, Wk, bk, workspace)
     d = dims_of(k_seg, Wk, P, phi)
     B, H = d.B, d.H
@@ -260,6 +316,18 @@ def segment_attend(q_seg, k_seg, v_seg, Wq, bq, *, T: int, c0: int, c1: int, P: 
     """Second phase: the segment's outputs.  S_prefix [n,B,H,F,D] / Z_prefix [n,B,H,F] stack
     the segment sums of every earlier segment (None for the first)."""
     lib = load()
+    _check_x_w(q_seg, Wq, bq, "q_seg")
+    s0, s1, h0 = segment_bounds(T, Tc, To, c0, c1)
+    B, H, _, D = q_seg.shape
+    F = Wq.shape[1] * Wq.shape[2]
+    _shape(q_seg, (B, H, (s1 - s0) * frame_tokens, D), "q_seg")
+    _shape(k_seg, (B, H, (s1 - h0) * frame_tokens, D), "k_seg")
+    _shape(v_seg, k_seg.shape, "v_seg")
+    _shape(out, q_seg.shape, "out")
+    if S_prefix is not None:
+        _shape(S_prefix, (S_prefix.shape[0], B, H, F, D), "S_prefix")
+    if Z_prefix is not None:
+        _shape(Z_prefix, (Z_prefix.shape[0], B, H, F), "Z_prefix")
     dev = _dev(q_seg, k_seg, v_seg, Wq, bq, workspace)
     d = dims_of(q_seg, Wq, P, phi)
     n_prefix = 0
@@ -286,6 +354,9 @@ def forward_states(k, v, Wk, bk, *, P: int, phi: int = 0, frame_tokens: int, Tc:
                    workspace: torch.Tensor) -> torch.Tensor:
     """First phase of `forward`: fills `workspace` with the state every chunk reads."""
     lib = load()
+    _check_x_w(k, Wk, bk, "k")
+    _shape(v, k.shape, "v")
+    _frames(k.shape[2], frame_tokens, "k")
     dev = _dev(k, v, Wk, bk, workspace)
     d = dims_of(k, Wk, P, phi)
     T = k.shape[2] // frame_tokens
@@ -299,6 +370,8 @@ def forward_phiq(q, Wq, bq, *, P: int, phi: int = 0, frame_tokens: int, Tc: int,
                  workspace: torch.Tensor) -> torch.Tensor:
     """Second phase of `forward`: phi_q of the query rows that read a state, into `workspace`."""
     lib = load()
+    _check_x_w(q, Wq, bq, "q")
+    _frames(q.shape[2], frame_tokens, "q")
     dev = _dev(q, Wq, bq, workspace)
     d = dims_of(q, Wq, P, phi)
     T = q.shape[2] // frame_tokens
@@ -311,6 +384,9 @@ def forward_attend(q, k, v, *, dims: Dims, frame_tokens: int, Tc: int, To: int,
                    workspace: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
     """Third phase of `forward`: the hybrid output from q, k, v and the workspace."""
     lib = load()
+    for t, n in ((k, "k"), (v, "v"), (out, "out")):
+        _shape(t, q.shape, n)
+    _frames(q.shape[2], frame_tokens, "q")
     dev = _dev(q, k, v, workspace, out)
     T = q.shape[2] // frame_tokens
     _check(lib.rehyat_forward_attend(dims, _dtype_code(q), T, frame_tokens, Tc, To, _ptr(q),
@@ -323,6 +399,9 @@ def chunk_states(k, v, Wk, bk, *, P: int, phi: int = 0, frame_tokens: int, Tc: i
                  workspace: torch.Tensor | None = None):
     """States each chunk of `forward` reads: S [B,H,C,F,D], Z [B,H,C,F] (fp32)."""
     lib = load()
+    _check_x_w(k, Wk, bk, "k")
+    _shape(v, k.shape, "v")
+    _frames(k.shape[2], frame_tokens, "k")
     dev = _dev(k, v, Wk, bk)
     d = dims_of(k, Wk, P, phi)
     N = k.shape[2]
@@ -344,6 +423,9 @@ def chunk_forward(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, phi: int = 0
     """One streaming step; S [B,H,F,D] and Z [B,H,F] (fp32) are updated in place.  To_next (the
     overlap of the next call, for a variable schedule) defaults to To."""
     lib = load()
+    cf = _frames(q.shape[2], frame_tokens, "q")
+    _check_step(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, out, frame_tokens,
+                min(To, frames_before) + cf, "k_win")
     dev = _dev(q, k_win, v_win, Wq, bq, Wk, bk, S, Z)
     d = dims_of(q, Wq, P, phi)
     chunk_frames = q.shape[2] // frame_tokens
@@ -377,6 +459,10 @@ def chunk_forward_carry(q, k, v, Wq, bq, Wk, bk, S, Z, k_carry, v_carry, *, P: i
     """Streaming step on the chunk alone; S, Z and the carried frames k_carry, v_carry
     [B,H,carry_frames*L,D] are updated in place."""
     lib = load()
+    _check_step(q, k, v, Wq, bq, Wk, bk, S, Z, out, frame_tokens, None, "k")
+    _frames(k_carry.shape[2], frame_tokens, "k_carry")
+    _shape(k_carry, (q.shape[0], q.shape[1], k_carry.shape[2], q.shape[3]), "k_carry")
+    _shape(v_carry, k_carry.shape, "v_carry")
     dev = _dev(q, k, v, Wq, bq, Wk, bk, S, Z, k_carry, v_carry)
     d = dims_of(q, Wq, P, phi)
     chunk_frames = q.shape[2] // frame_tokens
@@ -400,6 +486,9 @@ def chunk_forward_static(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, *, P: int, phi: 
     """chunk_forward without a workspace: the library's own fixed device scratch is used (for
     callers that cannot allocate); bf16 only."""
     lib = load()
+    cf = _frames(q.shape[2], frame_tokens, "q")
+    _check_step(q, k_win, v_win, Wq, bq, Wk, bk, S, Z, out, frame_tokens,
+                min(To, frames_before) + cf, "k_win")
     dev = _dev(q, k_win, v_win, Wq, bq, Wk, bk, S, Z)
     d = dims_of(q, Wq, P, phi)
     chunk_frames = q.shape[2] // frame_tokens
@@ -417,6 +506,12 @@ def forward_train(q, k, v, Wq, bq, Wk, bk, *, P: int, phi: int = 0, frame_tokens
     """`forward` that also returns lse [B,H,N] fp32 (log2 of every row's denominator), which
     `backward` needs.  bf16 only."""
     lib = load()
+    _check_x_w(q, Wq, bq, "q")
+    _check_x_w(q, Wk, bk, "q")
+    _shape(Wk, Wq.shape, "Wk")
+    for t, n in ((k, "k"), (v, "v"), (out, "out")):
+        _shape(t, q.shape, n)
+    _frames(q.shape[2], frame_tokens, "q")
     dev = _dev(q, k, v, Wq, bq, Wk, bk)
     _weights(Wq, bq), _weights(Wk, bk)
     d = dims_of(q, Wq, P, phi)
@@ -449,6 +544,13 @@ def backward(q, k, v, Wq, bq, Wk, bk, out, lse, dout, *, P: int, phi: int = 0,
     [H,G,F/G,D/G], dbq, dbk [H,F] (fp32).  `grads` may hold those buffers (written, not added
     to)."""
     lib = load()
+    _check_x_w(q, Wq, bq, "q")
+    _check_x_w(q, Wk, bk, "q")
+    _shape(Wk, Wq.shape, "Wk")
+    for t, n in ((k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _shape(t, q.shape, n)
+    _shape(lse, q.shape[:3], "lse")
+    _frames(q.shape[2], frame_tokens, "q")
     dev = _dev(q, k, v, Wq, bq, Wk, bk, out, lse, dout)
     d = dims_of(q, Wq, P, phi)
     N = q.shape[2]
