@@ -33,7 +33,10 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only enqueues work
  *     on it: the library never allocates device memory, never synchronises, and keeps no state
  *     between calls other than the device error word read by rehyat_sync_status().
- *   - The caller owns every buffer.  Buffers may not overlap, except where stated.
+ *   - The caller owns every buffer.  Buffers may not overlap, except where stated.  Sizes come
+ *     from the integer arguments; the library cannot see how large a buffer really is, so a
+ *     buffer smaller than its documented shape is read or written past its end.  (The Python
+ *     binding compares every tensor's shape with the shape its call implies.)
  *   - dtype REHYAT_BF16: q, k, v, out (and phi) are bf16; arithmetic is bf16 tensor-core
  *     products with fp32 accumulation, fp32 softmax and fp32 states.  Requires D = F = 128.
  *     dtype REHYAT_F32: everything fp32 on CUDA cores; requires D % 32 == 0, D <= 256,
