@@ -7,12 +7,13 @@ prefix scan, phi_q, and the fused softmax + linear attention, through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
                     [--workload 480p5s|480p10s|720p5s|480p20s-stream] [--phi poly|elu1]
-                    [--schedule FRAMES/OVERLAP,...]
+                    [--schedule FRAMES/OVERLAP,...] [--tc TC] [--to TO] [--p P]
 
 The other workloads and options measure the remaining configurations: the streaming workload's
 step is the whole chunk-by-chunk pass (27 calls per sequence, both sequences of the batch at
 once) through the streaming session; --schedule gives it a variable chunk schedule (the first
-entry once, the others cyclically, e.g. 5/0,3/1,3/2); --phi elu1 swaps the feature map.
+entry once, the others cyclically, e.g. 5/0,3/1,3/2); --phi elu1 swaps the feature map;
+--tc/--to/--p change the chunk length, overlap or part count (the ablation sweep).
 
 N > 1 runs under torchrun: every rank runs its own replica of the workload (weak scaling, no
 collective on the data path; NCCL only for the timing barrier and the max over ranks).
@@ -72,6 +73,9 @@ def parse_args():
                          "are computed before the timed region)")
     ap.add_argument("--schedule", default=None,
                     help="streaming only: FRAMES/OVERLAP entries, first once, rest cyclic")
+    ap.add_argument("--tc", type=int, default=None, help="chunk length in frames (ablation)")
+    ap.add_argument("--to", type=int, default=None, help="overlap frames (ablation)")
+    ap.add_argument("--p", type=int, default=None, help="polynomial parts of phi (ablation)")
     ap.add_argument("--parallel", choices=["replicas", "context"], default="replicas",
                     help="replicas: every rank runs its own batch (weak scaling); context: the "
                          "ranks split one sequence into chunk ranges (strong scaling)")
@@ -82,6 +86,10 @@ def pick_workload(args) -> C.Workload:
     w = WORKLOADS[args.workload]
     if args.phi != "poly":
         w = dataclasses.replace(w, phi=args.phi, P=1, name=w.name + ", elu+1 feature map")
+    over = {k: v for k, v in (("Tc", args.tc), ("To", args.to), ("P", args.p)) if v is not None}
+    if over:
+        w = dataclasses.replace(w, name=w.name + ", " + " ".join(f"{k}={v}" for k, v in
+                                                                  over.items()), **over)
     return w
 
 
@@ -213,26 +221,52 @@ def f64(t):
     return t.to(torch.float64).numpy()
 
 
-def cpu_baseline(inp, w: C.Workload, budget_s: float = 12.0):
+def cpu_baseline(inp, w: C.Workload, out=None, budget_s: float = 28.0):
     """The oracle's recurrent (linear-cost) form, head by head, until `budget_s` has passed or all
     heads are done; tokens/s scaled to the whole workload (a token = one query position across
-    all heads)."""
+    all heads).  With `out` (the timed run's output, [B, H, N, D] on the device) the oracle's rows
+    are also compared with it: relative L2 and max-abs per head and per chunk.  The row-sampled
+    quadratic form (the check form) is timed on 64 rows as well."""
     import oracle.rehyat_oracle as O
+    kind = O.PHI_ELU1 if w.phi == "elu1" else O.PHI_POLY
     t0 = time.perf_counter()
-    heads = 0
+    heads, per_head, per_chunk, max_abs = 0, [], {}, 0.0
+    L = w.frame_tokens
     for h in range(w.H):
         q, k, v = f64(inp.q[0, h]), f64(inp.k[0, h]), f64(inp.v[0, h])
-        pq = O.feature_map(q, f64(inp.Wq[h]), f64(inp.bq[h]), w.P)
-        pk = O.feature_map(k, f64(inp.Wk[h]), f64(inp.bk[h]), w.P)
-        O.hybrid_attention_recurrent(q, k, v, pq, pk, w.frame_tokens, w.Tc, w.To)
+        pq = O.feature_map(q, f64(inp.Wq[h]), f64(inp.bq[h]), w.P, kind)
+        pk = O.feature_map(k, f64(inp.Wk[h]), f64(inp.bk[h]), w.P, kind)
+        want = O.hybrid_attention_recurrent(q, k, v, pq, pk, L, w.Tc, w.To)
         heads += 1
+        if out is not None:
+            got = f64(out[0, h].cpu())
+            per_head.append(float(np.linalg.norm(got - want) / np.linalg.norm(want)))
+            max_abs = max(max_abs, float(np.abs(got - want).max()))
+            for c, (_, s, e) in enumerate(w.chunk_bounds()):
+                a, b = got[s * L:e * L], want[s * L:e * L]
+                r = float(np.linalg.norm(a - b) / np.linalg.norm(b))
+                per_chunk[c] = max(per_chunk.get(c, 0.0), r)
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
     tokens = w.B * w.N * heads / w.H
-    return {"value": tokens / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"float64 recurrent form, batch 0 heads 0-{heads - 1} of {w.H} (all "
-                      f"{w.N} query rows each), {dt:.1f} s; scaled to query tokens of all heads"}
+    res = {"value": tokens / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+           "sample": f"float64 recurrent form, batch 0 heads 0-{heads - 1} of {w.H} (all "
+                     f"{w.N} query rows each), {dt:.1f} s; scaled to query tokens of all heads"}
+    rows = np.random.default_rng(0).integers(0, w.N, size=64)
+    args_h = [f64(x) for x in (inp.q[0, 0], inp.k[0, 0], inp.v[0, 0], inp.Wq[0], inp.bq[0],
+                               inp.Wk[0], inp.bk[0])]
+    t1 = time.perf_counter()
+    O.hybrid_attention_rows(*args_h, w.P, L, w.Tc, w.To, rows, kind)
+    res["check_form"] = {"value": 64 / w.H / (time.perf_counter() - t1), "unit": UNIT,
+                         "what": "quadratic form (explicit weight of every key), 64 random "
+                                 "rows of head 0; a correctness tool, not a baseline"}
+    if out is not None:
+        res["parity_vs_timed_output"] = {
+            "heads": heads, "rel_l2_per_head": per_head, "max_abs": max_abs,
+            "rel_l2_per_chunk_worst_head": [per_chunk[c] for c in sorted(per_chunk)],
+            "bounds": "rel-L2 <= 5e-3, max-abs <= 2e-2"}
+    return res
 
 
 def run_reference(args, rank: int):
@@ -328,6 +362,7 @@ def main():
     K = args.steps
     mids = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    sts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(device_index_for_smi(dev))
     with sampler:
@@ -335,7 +370,7 @@ def main():
         torch.cuda.synchronize(dev)
         start.record(stream)
         for i in range(K):
-            run.step(mids[i], ends[i])
+            run.step(mids[i], ends[i], sts[i])
         stop.record(stream)
         torch.cuda.synchronize(dev)
         rep.barrier()
@@ -346,6 +381,20 @@ def main():
     attn_ms = statistics.mean(mids[i].elapsed_time(ends[i]) for i in range(K))
     pre_ms = statistics.mean((ends[i - 1].elapsed_time(mids[i]) if i else
                               start.elapsed_time(mids[0])) for i in range(K))
+    phases = None
+    if run.attn_isolated:
+        # states (weight preps, fold, scan) from the end of step i-1 to its states event; phi_q
+        # from there to the attention's start
+        st_ms = statistics.mean((ends[i - 1].elapsed_time(sts[i]) if i else
+                                 start.elapsed_time(sts[0])) for i in range(K))
+        phi_ms = statistics.mean(sts[i].elapsed_time(mids[i]) for i in range(K))
+        phases = {"states_ms": st_ms, "phiq_ms": phi_ms,
+                  "states_gbs": run.states_bytes / (st_ms * 1e-3) / 1e9,
+                  "phiq_gbs": run.phiq_bytes / (phi_ms * 1e-3) / 1e9,
+                  "bytes": "algorithmic: states = K and V of the folded tokens (bf16); phi_q = "
+                           "q rows in and phi_q rows out (bf16) of the chunks with a linear "
+                           "region"}
+    peak_mem = torch.cuda.max_memory_allocated(dev)
     elapsed_ms = rep.max(elapsed_ms, dev)
 
     # ---- end to end through the public API: pinned host inputs in, result out ----
@@ -391,6 +440,8 @@ def main():
             "frac_of_bf16_peak_step": run.step_flops / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "kernel_ms": ({"attention": attn_ms, "states_and_phiq": pre_ms} if run.attn_isolated
                           else {"step": ms_per_step}),
+            "hbm_phases": phases,
+            "peak_device_bytes": peak_mem,
             "roofline": {"kernel": run.roofline_kernel, "bound": "tensor",
                          "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"],
@@ -405,7 +456,8 @@ def main():
             "clocks": sampler.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(inp, w)
+            out_fn = getattr(run, "output", None)
+            line["cpu_baseline"] = cpu_baseline(inp, w, out_fn() if out_fn else None)
         print(json.dumps(line), flush=True)
     rep.close()
 
@@ -435,8 +487,10 @@ def full_runner(w: C.Workload, inp, dev, args) -> _Run:
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev_mid=None, ev_end=None):
+    def step(ev_mid=None, ev_end=None, ev_states=None):
         rb.forward_states(k, v, Wk, bk, workspace=ws, **kw)
+        if ev_states is not None:
+            ev_states.record(stream)
         rb.forward_phiq(q, Wq, bq, workspace=ws, **kw)
         if ev_mid is not None:
             ev_mid.record(stream)
@@ -456,12 +510,18 @@ def full_runner(w: C.Workload, inp, dev, args) -> _Run:
 
     pipe = HostPipeline(e2e_compute, host, out, dev)
     r.step = step
+    r.output = lambda: out
     r.e2e_run = lambda n: pipe.run([host] * n, [out_h] * n)
     r.h2d = sum(x.numel() * x.element_size() for x in host)
     r.d2h = out_h.numel() * out_h.element_size()
     r.attn_flops = w.attn_tensor_flops()
     r.step_flops = w.flops(streaming=False)
     r.launches_per_step = 6  # 2 weight preps, fold, scan, phi_q, attention
+    bnd = w.chunk_bounds()
+    folded = bnd[-1][0] * w.frame_tokens                       # tokens folded (frames < w_{C-1})
+    phiq_rows = sum((e - s) * w.frame_tokens for (wf, s, e) in bnd if wf > 0)
+    r.states_bytes = w.B * w.H * folded * 2 * w.D * 2
+    r.phiq_bytes = w.B * w.H * phiq_rows * (w.D + w.F) * 2
     return r
 
 
@@ -481,7 +541,7 @@ def backward_runner(w: C.Workload, inp, dev, args) -> _Run:
                                                 w.To), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev_mid=None, ev_end=None):
+    def step(ev_mid=None, ev_end=None, ev_states=None):
         if ev_mid is not None:
             ev_mid.record(stream)
         rb.backward(q, k, v, Wq, bq, Wk, bk, out, lse, dout, workspace=ws, **kw)
@@ -538,7 +598,7 @@ def context_runner(w: C.Workload, inp, dev, args, rep) -> _Run:
     out = torch.empty_like(q_own)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev_mid=None, ev_end=None):
+    def step(ev_mid=None, ev_end=None, ev_states=None):
         if ev_mid is not None:
             ev_mid.record(stream)
         cp.forward(q_own, k_buf, v_buf, out=out)
@@ -598,7 +658,7 @@ def stream_runner(w: C.Workload, inp, dev, args) -> _Run:
                        Tc=max(cf for cf, _ in sched), To=max(ov for _, ov in sched))
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev_mid=None, ev_end=None):
+    def step(ev_mid=None, ev_end=None, ev_states=None):
         if ev_mid is not None:
             ev_mid.record(stream)
         sess.reset()
@@ -653,6 +713,8 @@ def stream_runner(w: C.Workload, inp, dev, args) -> _Run:
     r.attn_flops = attn * w.B * w.H
     r.step_flops = (attn + step_f) * w.B * w.H
     r.step, r.e2e_step = step, e2e_step
+    if not args.schedule:
+        r.output = lambda: torch.cat(outs, dim=2)
     r.h2d = sum(x.numel() * x.element_size() for c in host for x in c)
     r.d2h = sum(o.numel() * o.element_size() for o in host_out)
     r.launches_per_step = launches

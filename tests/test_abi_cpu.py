@@ -176,3 +176,15 @@ def test_segment_checks(lib):
     st = lib.rehyat_segment_attend(d, rb.REHYAT_BF16, 21, 64, 3, 1, 2, 5, FAKE, FAKE, FAKE, FAKE,
                                    None, 2, None, None, FAKE, FAKE, 1 << 30, None)
     assert st == -1 and "S_prefix" in lib.rehyat_last_error().decode()
+
+
+def test_static_chunk_refuses_problems_beyond_its_scratch(lib):
+    """The static-scratch streaming call needs B*H*(6FD + 4F) + 8HFD bytes with one fold split;
+    past 16 MiB it refuses before anything is enqueued (no device is touched here)."""
+    def call(B, H):
+        return lib.rehyat_chunk_forward_static(dims(B=B, H=H), rb.REHYAT_BF16, 64, 3, 3, 1, FAKE,
+                                               FAKE, FAKE, FAKE, None, FAKE, None, FAKE, FAKE,
+                                               FAKE, None)
+    for B, H in [(13, 12), (1, 200), (169, 1)]:
+        assert call(B, H) == -4, (B, H)
+        assert "scratch" in lib.rehyat_last_error().decode()

@@ -358,17 +358,6 @@ def test_full_size_streaming_session_20s(dev):
     check_sampled(out, inp, w, rows, [(0, 3), (1, 5)])
 
 
-@pytest.mark.parametrize("Tc,To,P", [(1, 0, 1), (1, 1, 2), (3, 0, 2), (3, 1, 3), (5, 1, 2),
-                                     (5, 0, 1), (3, 2, 2)])
-def test_ablation_shapes_sampled(dev, Tc, To, P):
-    w = C.ablation(Tc, To, P)
-    inp = make_inputs(w, heads=2)
-    out = run_forward(inp, C.ablation(Tc, To, P), dev)
-    rng = np.random.default_rng(2)
-    rows = sample_rows(w, 3, rng)
-    check_sampled(out, inp, w, rows, [(0, 0), (0, 1)])
-
-
 # ------------------------------------------------------------------------------------------
 # argument errors reported through the C ABI on a GPU machine
 # ------------------------------------------------------------------------------------------
