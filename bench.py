@@ -42,6 +42,7 @@ from hybrid_softmax_linear_chunked_b200 import binding as rb  # noqa: E402
 from hybrid_softmax_linear_chunked_b200 import configs as C  # noqa: E402
 from hybrid_softmax_linear_chunked_b200.context_parallel import (  # noqa: E402
     ContextParallel, split_chunks)
+from hybrid_softmax_linear_chunked_b200.head_parallel import HeadSharded  # noqa: E402
 from hybrid_softmax_linear_chunked_b200.host_pipeline import HostPipeline  # noqa: E402
 from hybrid_softmax_linear_chunked_b200.inputs import make_inputs  # noqa: E402
 from hybrid_softmax_linear_chunked_b200.replicas import Replicas, job_throughput  # noqa: E402
@@ -76,9 +77,11 @@ def parse_args():
     ap.add_argument("--tc", type=int, default=None, help="chunk length in frames (ablation)")
     ap.add_argument("--to", type=int, default=None, help="overlap frames (ablation)")
     ap.add_argument("--p", type=int, default=None, help="polynomial parts of phi (ablation)")
-    ap.add_argument("--parallel", choices=["replicas", "context"], default="replicas",
+    ap.add_argument("--parallel", choices=["replicas", "context", "heads"], default="replicas",
                     help="replicas: every rank runs its own batch (weak scaling); context: the "
-                         "ranks split one sequence into chunk ranges (strong scaling)")
+                         "ranks split one sequence into chunk ranges; heads: the ranks split the "
+                         "(batch, head) problems of one batch and all-gather the outputs (both "
+                         "strong scaling)")
     return ap.parse_args()
 
 
@@ -342,12 +345,14 @@ def main():
     torch.cuda.set_device(dev)
     rb.load()
     w = pick_workload(args)
-    context = args.parallel == "context"
+    context = args.parallel in ("context", "heads")
     if context and (args.which != "forward" or w.mode == "stream"):
-        raise SystemExit("--parallel context times the whole-sequence forward")
-    # context parallelism splits one sequence: every rank draws the same one
+        raise SystemExit(f"--parallel {args.parallel} times the whole-sequence forward")
+    # context and head parallelism split one problem: every rank draws the same one
     inp = make_inputs(w, seed=w.seed if context else rep.seed(w.seed))
-    if context:
+    if args.parallel == "heads":
+        run = heads_runner(w, inp, dev, args, rep)
+    elif context:
         run = context_runner(w, inp, dev, args, rep)
     elif args.which == "backward":
         run = backward_runner(w, inp, dev, args)
@@ -629,6 +634,50 @@ def context_runner(w: C.Workload, inp, dev, args, rep) -> _Run:
     r.config = {"parallelism": f"cp{rep.world} (chunk ranges [c0, c1) per rank: "
                                f"{split_chunks(w.n_chunks, rep.world)}; halo point to point, "
                                "segment sums all-gathered)"}
+    return r
+
+
+def heads_runner(w: C.Workload, inp, dev, args, rep) -> _Run:
+    """The whole-sequence forward with the B*H (batch, head) problems split over the ranks: each
+    rank holds its units' q, k, v, runs the library forward on them, and the output slices are
+    all-gathered so that every rank ends with the whole output."""
+    r = _Run()
+    r.attn_isolated = False
+    Wq, bq, Wk, bk = (x.to(dev) for x in (inp.Wq, inp.bq, inp.Wk, inp.bk))
+    hs = HeadSharded(Wq, bq, Wk, bk, B=w.B, H=w.H, frame_tokens=w.frame_tokens, Tc=w.Tc,
+                     To=w.To, P=w.P, phi=w.phi_code)
+    host = [hs.shard(x).contiguous().pin_memory() for x in (inp.q, inp.k, inp.v)]
+    q_s, k_s, v_s = (x.to(dev) for x in host)
+    out_s = torch.empty_like(q_s)
+    stream = torch.cuda.current_stream(dev)
+    full = [None]
+
+    def step(ev_mid=None, ev_end=None, ev_states=None):
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        hs.forward(q_s, k_s, v_s, out=out_s)
+        full[0] = hs.gather(out_s)
+        if ev_end is not None:
+            ev_end.record(stream)
+
+    host_out = torch.empty((w.B, w.H, w.N, w.D), dtype=q_s.dtype).pin_memory()
+
+    def e2e_step():
+        for d_, h_ in zip((q_s, k_s, v_s), host):
+            d_.copy_(h_, non_blocking=True)
+        hs.forward(q_s, k_s, v_s, out=out_s)
+        host_out.copy_(hs.gather(out_s), non_blocking=True)
+
+    r.step, r.e2e_step = step, e2e_step
+    r.output = lambda: full[0]
+    r.h2d = sum(x.numel() * x.element_size() for x in host)
+    r.d2h = host_out.numel() * host_out.element_size()
+    r.step_flops = w.flops(streaming=False)
+    r.attn_flops = w.flops(streaming=False)
+    r.launches_per_step = 6  # 2 weight preps, fold, scan, phi_q, attention (+ the all-gather)
+    r.roofline_kernel = "head-sharded forward step (whole-problem FLOPs / step time)"
+    r.config = {"parallelism": f"heads{rep.world} ((batch, head) units per rank: "
+                               f"{hs.ranges}; output slices all-gathered)"}
     return r
 
 

@@ -220,6 +220,18 @@ int fold_splits(int BH, int n_fold, long long rows_per_fold) {
   return (int)s;
 }
 
+// Token splits of one fold range in the whole-sequence forward (and its segments): a function
+// of the range's length only, about 18 tiles of 128 tokens per split and at most 16, so that
+// every (b, h) is folded in the same order whatever other (b, h) share the call (a head-sharded
+// run reproduces the one-call result bit for bit).
+int fold_splits_shape(long long rows_per_fold) {
+  const long long tiles = (rows_per_fold + 127) / 128;
+  long long s = (tiles + 8) / 18;
+  if (s < 1) s = 1;
+  if (s > 16) s = 16;
+  return (int)s;
+}
+
 struct ForwardPlan {
   int C, n_fold, splits;
   size_t dS, dZ, St, Zc, Wqbd, Wkbd, phiq_bf16, phiq, phik, Sc, total;
@@ -232,7 +244,7 @@ ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, in
   p.n_fold = p.C - 1;
   Carve cv;
   if (dt == REHYAT_BF16) {
-    p.splits = fold_splits((int)BH, p.n_fold, (long long)Tc * L);
+    p.splits = fold_splits_shape((long long)Tc * L);
     const size_t nf = p.n_fold > 0 ? p.n_fold : 0;
     p.dS = cv.take(BH * nf * p.splits * d.F * d.D * 4);
     p.dZ = cv.take(BH * nf * p.splits * d.F * 4);
@@ -316,7 +328,7 @@ SegPlan plan_segment(const rehyat_dims& d, int T, int L, int Tc, int To, int c0,
   p.n_fold = fold_end > c0 ? fold_end - c0 : 0;
   p.nq_rows = (long long)(p.s1 - p.s0) * L;
   p.nkv_rows = (long long)(p.s1 - p.h0) * L;
-  p.splits = fold_splits((int)BH, p.n_fold, (long long)Tc * L);
+  p.splits = fold_splits_shape((long long)Tc * L);
   Carve cv;
   const size_t nf = p.n_fold;
   p.dS = cv.take(BH * nf * p.splits * d.F * d.D * 4);

@@ -19,6 +19,7 @@ pytestmark = pytest.mark.gpu
 
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
+STATE_REL = 1e-5
 
 
 @pytest.fixture(scope="module")
@@ -29,6 +30,18 @@ def dev():
     build.build()
     rb.load()
     return torch.device("cuda", 0)
+
+
+def close_state(a, b, what):
+    """S and Z are fp32 sums over thousands of tokens (Z reaches ~1e4): when the two calls split
+    the fold differently the summation order differs, so they agree to fp32 rounding relative to
+    their size, not to an absolute bound."""
+    a = a.double().cpu().numpy()
+    b = b.double().cpu().numpy()
+    err = np.abs(a - b).max() / max(np.abs(b).max(), 1e-30)
+    rel = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
+    assert np.isfinite(a).all(), what + ": non-finite"
+    assert err <= STATE_REL and rel <= STATE_REL, f"{what}: max-abs/max {err:.3e} rel-L2 {rel:.3e}"
 
 
 def close(a, b, what):
@@ -64,5 +77,5 @@ def test_static_scratch_matches_workspace_call(dev, B, H, fh, fw):
         rb.chunk_forward_static(qc, kw, vw, Wq, bq, Wk, bk, S_st, Z_st, out=got, **kwargs)
         rb.sync_status(dev)
         close(got, ref, f"output of the chunk at frame {s}")
-        close(S_st, S_ref, f"S after the chunk at frame {s}")
-        close(Z_st, Z_ref, f"Z after the chunk at frame {s}")
+        close_state(S_st, S_ref, f"S after the chunk at frame {s}")
+        close_state(Z_st, Z_ref, f"Z after the chunk at frame {s}")
