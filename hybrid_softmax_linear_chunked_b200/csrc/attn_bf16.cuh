@@ -56,7 +56,7 @@ enum Bar {
   kVEmpty = 7,   // 2
   kSFull = 9,    // 2 (per query tile)
   kPFull = 11,   // 2 (per query tile, 128 arrivals)
-  kOFull = 13,   // 2 (per query tile)
+  kOFull = 13,   // 2 (per query tile): its last P.V is complete (one phase per CTA)
   kStFull = 15,
   kPhiFull = 16,  // 2 (per query tile, 128 arrivals)
   kRoDone = 18,   // 2
@@ -86,7 +86,34 @@ struct Params {
   const float* Z;     // [BH, n_states, F]
   __nv_bfloat16* out; // [BH, nq_rows, D]
   float* lse;         // [BH, nq_rows] or null: log2 of each row's denominator (for the backward)
+  // A chunk whose tile count is odd has a lone last tile.  With n_split > 1 that tile's key window
+  // is cut into n_split parts, each run by its own (short) CTA, which writes its rows'
+  // unnormalised O and (m, l) here instead of the output; lone_combine_kernel merges the parts.
+  // Only part 0 adds the linear-state readout.  Slot of (chunk c, bh, part):
+  // (c * BH + bh) * n_split + part.  Not combined with lse.
+  int n_split;
+  float* part_o;      // [chunks * BH * n_split][128][D] fp32
+  float* part_ml;     // [chunks * BH * n_split][128][2] fp32: m (log2 units) and l per row
 };
+
+// Rows and key window of chunk c of a launch (frames relative to the video).
+struct ChunkGeom {
+  int q_row0, nq;    // query rows [q_row0, q_row0 + nq) of the q/out buffers
+  int k_row0, nk;    // window rows of the main K/V source (after the carried segment)
+  bool has_linear;   // the chunk reads a linear state
+};
+__device__ __forceinline__ ChunkGeom chunk_geom(const Params& p, int c) {
+  const int gs = p.frames_before + c * p.Tc;
+  const int ge = min(gs + p.Tc, p.frames_before + p.T);
+  const int gw = max(0, gs - p.To);
+  ChunkGeom g;
+  g.q_row0 = (gs - p.frames_before) * p.L;
+  g.nq = (ge - gs) * p.L;
+  g.k_row0 = (gw - p.kv_frame0) * p.L;
+  g.nk = (ge - gw) * p.L;
+  g.has_linear = gw > 0;
+  return g;
+}
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -155,39 +182,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
 
   // ---- chunk geometry (uniform over the CTA) ----
-  // grid (tile-pair slots, BH, chunks).  Within one chunk the linear CTA index walks the full
-  // tile pairs of one (b, h) after another, so the CTAs in flight share few K/V windows in L2;
-  // the lone last tiles of an odd tile count (the shortest CTAs) follow, one per (b, h).  Chunk
-  // 0, whose window is shortest, is dispatched last.
+  // grid (slots, BH, chunks).  Within one chunk the linear CTA index walks the full tile pairs of
+  // one (b, h) after another, so the CTAs in flight share few K/V windows in L2; the lone last
+  // tiles of an odd tile count follow (one per (b, h), or n_split short parts of its key window
+  // each).  Chunk 0, whose window is shortest, is dispatched last.
   const int c = (blockIdx.z + 1) % gridDim.z;
-  const int gs = p.frames_before + c * p.Tc;
-  const int ge = min(gs + p.Tc, p.frames_before + p.T);
-  const int gw = max(0, gs - p.To);
-  const int q_row0 = (gs - p.frames_before) * p.L;
-  const int nq = (ge - gs) * p.L;
-  const int k_row0 = (gw - p.kv_frame0) * p.L;
-  const int nk = (ge - gw) * p.L;
-  const bool has_linear = gw > 0;
+  const ChunkGeom geo = chunk_geom(p, c);
+  const int q_row0 = geo.q_row0, nq = geo.nq, k_row0 = geo.k_row0, nk = geo.nk;
+  const bool has_linear = geo.has_linear;
   const int n_full = ((nq + kBM - 1) / kBM) / 2, n_lone = ((nq + kBM - 1) / kBM) & 1;
+  const int n_split = p.n_split > 1 ? p.n_split : 1;
   const int n_bh = gridDim.y;
   const int lin = blockIdx.x + gridDim.x * blockIdx.y;
-  int bh, pair;
+  int bh, pair, part = -1;  // part >= 0: one part of the lone tile's key window
   if (lin < n_full * n_bh) {
     bh = lin / n_full;
     pair = lin - bh * n_full;
-  } else if (lin < (n_full + n_lone) * n_bh) {
-    bh = lin - n_full * n_bh;
+  } else if (lin < (n_full + n_lone * n_split) * n_bh) {
+    const int idx = lin - n_full * n_bh;
+    bh = idx / n_split;
     pair = n_full;
+    if (n_split > 1) part = idx - bh * n_split;
   } else {
     return;  // a slot past this chunk's tiles (its chunk is shorter than the longest)
   }
   const int h = bh % p.H;
   const int tile_row0 = pair * 2 * kBM;
   const bool has_t1 = tile_row0 + kBM < nq;
-  // key tiles: n_kc from the carried segment (rows [0, kv_split) of the window), then the rest
+  // key tiles: n_kc from the carried segment (rows [0, kv_split) of the window), then the rest;
+  // a part covers key tiles [j0, j0 + n_kv) of them (the host keeps every part non-empty)
   const int kv_split = p.kv_split;
   const int n_kc = (kv_split + kBN - 1) / kBN;
-  const int n_kv = n_kc + (nk - kv_split + kBN - 1) / kBN;
+  const int n_kv_all = n_kc + (nk - kv_split + kBN - 1) / kBN;
+  const int j0 = part >= 0 ? (int)((long long)part * n_kv_all / n_split) : 0;
+  const int n_kv = (part >= 0 ? (int)((long long)(part + 1) * n_kv_all / n_split) : n_kv_all) - j0;
+  // the linear-state readout (phi_q . S, phi_q . Z) is added once: by the whole-window CTA or by
+  // part 0
+  const bool readout = has_linear && part <= 0;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -213,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     abort_sh = 0;
     fence_mbar_init();
   }
-  if (tid < 256 && has_linear) {
+  if (tid < 256 && readout) {
     for (int i = tid; i < kFD; i += 256) {
       sPw[i] = static_cast<uint8_t>(feature_power(i, kFD, p.P));
       sB[i] = p.bq ? p.bq[(size_t)h * kFD + i] : 0.f;
@@ -258,8 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int j = 0; j < n_kv; ++j) {
       const int s = j & 1;
-      const bool carried = j < n_kc;
-      const int row = carried ? p.carry_row0 + j * kBN : k_row0 + kv_split + (j - n_kc) * kBN;
+      const int jg = j0 + j;  // key tile of the window
+      const bool carried = jg < n_kc;
+      const int row = carried ? p.carry_row0 + jg * kBN : k_row0 + kv_split + (jg - n_kc) * kBN;
       const CUtensorMap* mK = carried ? &tmKc : &tmK;
       const CUtensorMap* mV = carried ? &tmVc : &tmV;
       if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty + s], ((j >> 1) - 1) & 1, abort_flag));
@@ -283,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       ++issued_v;
     }
-    if (ok && has_linear) {
+    if (ok && readout) {
       // S_c^T, Z_c and phi_q come from the kernels enqueued before this one.  Launched behind
       // the phi_q kernel with programmatic serialization, this kernel ran its key loop while
       // that grid was still running: wait for it (and so for everything before it) here.
@@ -307,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     bool wb_issued = false;
-    if (ok && has_linear && kPhiGlobal) {
+    if (ok && readout && kPhiGlobal) {
       // phi_q tiles go over the Q tiles once both tiles' last S MMAs are done.
       const int last = n_kv - 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty + (last & 1)], (last >> 1) & 1, abort_flag));
@@ -324,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         wb_issued = true;
       }
-    } else if (ok && has_linear) {
+    } else if (ok && readout) {
       // Block-diagonal W_q (hi, lo) goes into the two V stages once their last P.V is done.
       for (int s = 0; s < 2 && ok; ++s) {
         const int last = (n_kv - 1) - (((n_kv - 1) & 1) != s ? 1 : 0);  // last use of stage s
@@ -357,77 +389,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 9) {
     // ================================ MMA issuer ================================
-    // The whole warp runs the loop and waits; lane 0 issues the MMAs and commits.
-    const bool leader = lane == 0;
-    const uint32_t id_qk = idesc_bf16(kBM, kBN, false, false);
-    const uint32_t id_pv = idesc_bf16(kBM, kHD, false, true);
-    const int nt = has_t1 ? 2 : 1;
-    auto issue_s = [&](int t, int j) {
-      if (leader) {
+    // Lane 0 runs the loop alone (waits, MMAs, commits); the other lanes wait at the end.  The
+    // two query tiles alternate strictly (P.V and the next S of tile 0, then of tile 1), so one
+    // tile's MMAs run while the other tile's softmax works.  There is no per-step O_FULL commit:
+    // S_FULL(t, j) is committed after P.V(t, j-1) was issued by this thread, so its completion
+    // already tells the softmax that O_t may be rescaled.
+    if (lane == 0) {
+      const uint32_t id_qk = idesc_bf16(kBM, kBN, false, false);
+      const uint32_t id_pv = idesc_bf16(kBM, kHD, false, true);
+      const int nt = has_t1 ? 2 : 1;
+      auto issue_s = [&](int t, int j) {
         const uint32_t d = tmem + t * 128;
         const uint32_t qb = t ? sQ1 : sQ0;
         const uint32_t kb = (j & 1) ? sK1 : sK0;
         for (int kk = 0; kk < kHD / 16; ++kk)
           mma_ss(d, kmajor_desc(qb, kk), kmajor_desc(kb, kk), id_qk, kk > 0 ? 1u : 0u);
         mma_commit(&bars[kSFull + t]);
-      }
-      __syncwarp();
-    };
-    auto issue_pv = [&](int t, int j) {
-      if (leader) {
+      };
+      auto issue_pv = [&](int t, int j) {
         const uint32_t d = tmem + 256 + t * 128;
         const uint32_t a = tmem + t * 128;
         const uint32_t vb = (j & 1) ? sV1 : sV0;
         for (int kk = 0; kk < kBN / 16; ++kk)
           mma_ts(d, a + kk * 8, mnmajor_desc(vb, kk), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars[kOFull + t]);
+      };
+      auto wait = [&](int b, uint32_t parity) { return mbar_wait(&bars[b], parity, abort_flag); };
+      bool ok = wait(kQFull, 0) && wait(kKFull, 0);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < nt; ++t) issue_s(t, 0);
+        mma_commit(&bars[kKEmpty]);
       }
-      __syncwarp();
-    };
-    auto commit = [&](int b) {
-      if (leader) mma_commit(&bars[b]);
-      __syncwarp();
-    };
-    auto wait = [&](int b, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, abort_flag));
-    };
-    bool ok = wait(kQFull, 0) && wait(kKFull, 0);
-    if (ok) {
-      tc_fence_after();
-      for (int t = 0; t < nt; ++t) issue_s(t, 0);
-      commit(kKEmpty);
-    }
-    for (int j = 1; j < n_kv && ok; ++j) {
-      const int s = j & 1, sp = (j - 1) & 1;
-      ok = wait(kKFull + s, (j >> 1) & 1) && wait(kVFull + sp, ((j - 1) >> 1) & 1);
-      for (int t = 0; t < nt && ok; ++t) {
-        ok = wait(kPFull + t, (j - 1) & 1);
+      for (int j = 1; j < n_kv && ok; ++j) {
+        const int s = j & 1, sp = (j - 1) & 1;
+        ok = wait(kKFull + s, (j >> 1) & 1) && wait(kVFull + sp, ((j - 1) >> 1) & 1);
+        for (int t = 0; t < nt && ok; ++t) {
+          ok = wait(kPFull + t, (j - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, j - 1);
+          issue_s(t, j);
+        }
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(t, j - 1);
-        issue_s(t, j);
+        mma_commit(&bars[kVEmpty + sp]);
+        mma_commit(&bars[kKEmpty + s]);
       }
-      if (!ok) break;
-      commit(kVEmpty + sp);
-      commit(kKEmpty + s);
-    }
-    if (ok) {
-      const int j = n_kv - 1;
-      ok = wait(kVFull + (j & 1), (j >> 1) & 1);
-      for (int t = 0; t < nt && ok; ++t) {
-        ok = wait(kPFull + t, j & 1);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(t, j);
+      if (ok) {
+        const int j = n_kv - 1;
+        ok = wait(kVFull + (j & 1), (j >> 1) & 1);
+        for (int t = 0; t < nt && ok; ++t) {
+          ok = wait(kPFull + t, j & 1);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, j);
+          mma_commit(&bars[kOFull + t]);  // the tile's O is final (epilogue without a state)
+        }
+        if (ok) mma_commit(&bars[kVEmpty + (j & 1)]);
       }
-      if (ok) commit(kVEmpty + (j & 1));
-    }
-    if (ok && has_linear) {
-      // U_t = Q_t Wbd_hi^T + Q_t Wbd_lo^T into the S_t columns (free once P_t.V is issued).
-      if (!kPhiGlobal) ok = wait(kWbFull, 0);
-      if (ok && !kPhiGlobal) {
-        tc_fence_after();
-        if (leader) {
+      if (ok && readout) {
+        // U_t = Q_t Wbd_hi^T + Q_t Wbd_lo^T into the S_t columns (free once P_t.V is issued).
+        if (!kPhiGlobal) ok = wait(kWbFull, 0);
+        if (ok && !kPhiGlobal) {
+          tc_fence_after();
           for (int t = 0; t < nt; ++t) {
             const uint32_t d = tmem + t * 128;
             const uint32_t qb = t ? sQ1 : sQ0;
@@ -440,27 +463,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bars[kUFull + t]);
           }
         }
-        __syncwarp();
-      }
-      const uint32_t stb = (n_kv & 1) ? sK1 : sK0;
-      if (ok) ok = wait(kStFull, 0);
-      for (int t = 0; t < nt && ok; ++t) {
-        ok = wait(kPhiFull + t, 0);
-        if (!ok) break;
-        tc_fence_after();
-        if (leader) {
+        const uint32_t stb = (n_kv & 1) ? sK1 : sK0;
+        if (ok) ok = wait(kStFull, 0);
+        for (int t = 0; t < nt && ok; ++t) {
+          ok = wait(kPhiFull + t, 0);
+          if (!ok) break;
+          tc_fence_after();
           const uint32_t d = tmem + 256 + t * 128;
           const uint32_t qb = t ? sQ1 : sQ0;
           for (int kk = 0; kk < kFD / 16; ++kk)
             mma_ss(d, kmajor_desc(qb, kk), kmajor_desc(stb, kk), id_qk, 1u);
           mma_commit(&bars[kRoDone + t]);
         }
-        __syncwarp();
       }
+      // Every tcgen05 op (and the mbarrier arrivals it triggers) must finish before teardown.
+      mma_commit(&bars[kMmaDone]);
+      mbar_wait_drain(&bars[kMmaDone], 0);
     }
-    // Every tcgen05 op (and the mbarrier arrivals it triggers) must finish before teardown.
-    commit(kMmaDone);
-    mbar_wait_drain(&bars[kMmaDone], 0);
     __syncwarp();
   } else {
     // ============================ softmax / epilogue warpgroups ============================
@@ -483,7 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // partial maxima and the row sum uses four accumulators, so neither is one long
         // dependency chain.  Only a segment's last tile can be ragged (uniform branch).
         // key columns of this tile inside its segment of the window
-        const int valid = j < n_kc ? kv_split - j * kBN : nk - kv_split - (j - n_kc) * kBN;
+        const int jg = j0 + j;
+        const int valid = jg < n_kc ? kv_split - jg * kBN : nk - kv_split - (jg - n_kc) * kBN;
         uint32_t rr[kBN];
         tmem_ld128(tS, rr);
         if (valid < kBN) {
@@ -507,11 +527,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_new = (m_tile > m + 8.f) ? m_tile : m;
         const bool rescale = (m_new != m) && (j > 0);
         if (__any_sync(0xffffffffu, rescale)) {
-          // Rare: rescale O and l.  S is reloaded afterwards so it need not stay live here.
+          // Rare: rescale O and l.  S_FULL for this tile was committed after the tile's previous
+          // P.V, so that P.V is complete and O may be rewritten.  S is reloaded afterwards so it
+          // need not stay live here.
           const float fac = rescale ? ex2(m - m_new) : 1.f;
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + t], (j - 1) & 1, abort_flag));
-          if (!ok) break;
-          tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < kHD / 16; ++cc) {
             uint32_t ro[16];
@@ -565,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars[kPFull + t]);
       }
       // ---- epilogue ----
-      if (ok && has_linear && kPhiGlobal) {
+      if (ok && readout && kPhiGlobal) {
         // The precomputed phi_q row sits in this row of the Q tile: scale it by 2^-m in place
         // (bf16) and form phi_q . Z_c with the same rounded values the MMA will use.
         ok = __all_sync(0xffffffffu, mbar_wait(&bars[kPhiqFull], 0, abort_flag));
@@ -596,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           l += lin[0] + lin[1];
           ok = __all_sync(0xffffffffu, mbar_wait(&bars[kRoDone + t], 0, abort_flag));
         }
-      } else if (ok && has_linear) {
+      } else if (ok && readout) {
         // U_FULL also means every earlier MMA of this CTA (the last P.V included) is complete.
         ok = __all_sync(0xffffffffu, mbar_wait(&bars[kUFull + t], 0, abort_flag));
         if (ok) {
@@ -631,9 +650,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(&bars[kRoDone + t], 0, abort_flag));
         }
       } else if (ok) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + t], (n_kv - 1) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + t], 0, abort_flag));
       }
-      if (ok) {
+      if (ok && part >= 0) {
+        // one part of a lone tile's window: its rows' unnormalised O and (m, l), every row
+        tc_fence_after();
+        const size_t slot = ((size_t)c * n_bh + bh) * n_split + part;
+        float* po = p.part_o + (slot * kBM + r) * kHD;
+#pragma unroll
+        for (int cc = 0; cc < kHD / 32; ++cc) {
+          uint32_t rr[32];
+          tmem_ld32(tO + cc * 32, rr);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            *reinterpret_cast<float4*>(po + cc * 32 + q4 * 4) =
+                make_float4(__uint_as_float(rr[q4 * 4]), __uint_as_float(rr[q4 * 4 + 1]),
+                            __uint_as_float(rr[q4 * 4 + 2]), __uint_as_float(rr[q4 * 4 + 3]));
+        }
+        *reinterpret_cast<float2*>(p.part_ml + (slot * kBM + r) * 2) = make_float2(m, l);
+      } else if (ok) {
         tc_fence_after();
         const int row_in_chunk = tile_row0 + t * kBM + r;
         const bool row_valid = row_in_chunk < nq;
@@ -668,6 +703,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// Merges the parts of every chunk's lone last tile (see Params::n_split):
+//   out = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i,  M = max_i m_i.
+// grid (BH, chunks, 128 rows), block D = 128 (one output column per thread).
+__global__ void __launch_bounds__(kHD) lone_combine_kernel(const Params p) {
+  const int bh = blockIdx.x, c = blockIdx.y, r = blockIdx.z, col = threadIdx.x;
+  const ChunkGeom geo = chunk_geom(p, c);
+  const int n_tiles = (geo.nq + kBM - 1) / kBM;
+  if (!(n_tiles & 1)) return;  // no lone tile in this chunk
+  const int row_in_chunk = (n_tiles / 2) * 2 * kBM + r;
+  if (row_in_chunk >= geo.nq) return;
+  const size_t slot0 = ((size_t)c * gridDim.x + bh) * p.n_split;
+  float M = -INFINITY;
+  for (int i = 0; i < p.n_split; ++i) M = fmaxf(M, p.part_ml[((slot0 + i) * kBM + r) * 2]);
+  float num = 0.f, den = 0.f;
+  for (int i = 0; i < p.n_split; ++i) {
+    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + ((slot0 + i) * kBM + r) * 2);
+    const float w = ex2(ml.x - M);
+    den = fmaf(w, ml.y, den);
+    num = fmaf(w, p.part_o[((slot0 + i) * kBM + r) * kHD + col], num);
+  }
+  p.out[((size_t)bh * p.nq_rows + geo.q_row0 + row_in_chunk) * kHD + col] =
+      __float2bfloat16_rn(num / den);
 }
 
 }  // namespace attn

@@ -232,9 +232,52 @@ int fold_splits_shape(long long rows_per_fold) {
   return (int)s;
 }
 
+// Parts a chunk's lone last tile is cut into (its key window spread over that many short CTAs,
+// which fill the attention's last wave instead of forming a wave of their own), at most
+// kMaxLoneSplit; every part keeps at least one key tile.
+constexpr int kMaxLoneSplit = 4;
+int lone_split_count(int min_key_tiles) {
+  int k = kMaxLoneSplit;
+  if (k > min_key_tiles) k = min_key_tiles;
+  return k < 1 ? 1 : k;
+}
+// Scratch for the parts of the lone tiles of `n_chunks` chunks: O [128][D] and (m, l) per row.
+size_t lone_part_bytes(size_t BH, int n_chunks, int D) {
+  return BH * n_chunks * kMaxLoneSplit * 128 * ((size_t)D + 2) * 4;
+}
+
+// Lone-tile split of an attention launch over chunks [0, n_chunks) whose chunk c owns frames
+// [frames_before + c*Tc, min(frames_before + (c+1)*Tc, frames_before + T)) and reads a window
+// reaching To frames back: parts per lone tile (1 when no chunk has one, or when not allowed) and
+// the grid's slot count per (b, h).
+struct LoneSplit {
+  int n_split, slots;
+};
+LoneSplit lone_split_plan(int T, int L, int Tc, int To, int frames_before, int n_chunks,
+                          bool allow) {
+  int max_tiles = 0, min_key = 1 << 30;
+  bool any_lone = false;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int gs = frames_before + c * Tc;
+    const int ge = gs + Tc < frames_before + T ? gs + Tc : frames_before + T;
+    const int gw = gs - To > 0 ? gs - To : 0;
+    const int tiles = ((ge - gs) * L + 127) / 128;
+    if (tiles > max_tiles) max_tiles = tiles;
+    if (tiles & 1) {
+      any_lone = true;
+      const int key_tiles = ((ge - gw) * L + 127) / 128;
+      if (key_tiles < min_key) min_key = key_tiles;
+    }
+  }
+  LoneSplit r;
+  r.n_split = (allow && any_lone) ? lone_split_count(min_key) : 1;
+  r.slots = max_tiles / 2 + (any_lone ? r.n_split : 0);
+  return r;
+}
+
 struct ForwardPlan {
   int C, n_fold, splits;
-  size_t dS, dZ, St, Zc, Wqbd, Wkbd, phiq_bf16, phiq, phik, Sc, total;
+  size_t dS, dZ, St, Zc, Wqbd, Wkbd, phiq_bf16, phiq, phik, Sc, part, total;
 };
 
 ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, int Tc, int To) {
@@ -253,6 +296,7 @@ ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, in
     p.Wqbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
     p.Wkbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
     p.phiq_bf16 = cv.take(BH * (size_t)T * L * d.F * 2);
+    p.part = cv.take(lone_part_bytes(BH, p.C, d.D));
   } else {
     p.splits = 1;
     const size_t N = (size_t)T * L;
@@ -270,7 +314,7 @@ ForwardPlan plan_forward(const rehyat_dims& d, rehyat_dtype dt, int T, int L, in
 
 struct ChunkPlan {
   int o, nq, nkv, fold_rows, splits;
-  size_t St, dS, dZ, Wqbd, Wkbd, phiq_bf16, phiq, phik, total;
+  size_t St, dS, dZ, Wqbd, Wkbd, phiq_bf16, phiq, phik, part, total;
 };
 
 ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_before,
@@ -296,6 +340,7 @@ ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_be
     p.Wqbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
     p.Wkbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
     p.phiq_bf16 = cv.take(BH * (size_t)p.nq * d.F * 2);
+    p.part = cv.take(lone_part_bytes(BH, 1, d.D));
   } else {
     p.splits = 1;
     const size_t max_kv = (size_t)(To + chunk_frames) * L;
@@ -313,7 +358,7 @@ ChunkPlan plan_chunk(const rehyat_dims& d, rehyat_dtype dt, int L, int frames_be
 struct SegPlan {
   int C, s0, s1, h0, n_local, n_fold, splits;
   long long nq_rows, nkv_rows;
-  size_t dS, dZ, St, Zc, Wqbd, Wkbd, phiq_bf16, total;
+  size_t dS, dZ, St, Zc, Wqbd, Wkbd, phiq_bf16, part, total;
 };
 
 SegPlan plan_segment(const rehyat_dims& d, int T, int L, int Tc, int To, int c0, int c1) {
@@ -338,6 +383,7 @@ SegPlan plan_segment(const rehyat_dims& d, int T, int L, int Tc, int To, int c0,
   p.Wqbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
   p.Wkbd = cv.take((size_t)d.H * 2 * d.F * d.D * 2);
   p.phiq_bf16 = cv.take(BH * (size_t)p.nq_rows * d.F * 2);
+  p.part = cv.take(lone_part_bytes(BH, p.n_local, d.D));
   p.total = cv.off;
   return p;
 }
@@ -419,6 +465,12 @@ int launch_attn_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   const CUtensorMap kc = mkc ? *mkc : mk, vc = mvc ? *mvc : mv;
   return cuda_check(cudaLaunchKernelEx(&cfg, k, mq, mk, mv, ms, mw, mphi, kc, vc, ap),
                     "attention launch");
+}
+
+// Merges the parts of the lone last tiles of a split attention launch into its output.
+int launch_lone_combine(const rehyat::attn::Params& ap, int BH, int n_chunks, cudaStream_t st) {
+  rehyat::attn::lone_combine_kernel<<<dim3(BH, n_chunks, 128), rehyat::attn::kHD, 0, st>>>(ap);
+  return cuda_check(cudaGetLastError(), "lone-tile combine launch");
 }
 
 // phi of rows [row0, row0 + n_rows) of every (b, h) sequence of x (rows_per_bh rows each) into
@@ -808,9 +860,15 @@ static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int
     ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
     ap.out = static_cast<__nv_bfloat16*>(out);
     ap.lse = lse;
-    dim3 grid((rows_per_chunk + 255) / 256, BH, pl.C);
-    return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, grid, st, nullptr, nullptr,
-                                  behind_phiq);
+    // lone last tiles run as parts of their key window (not when row statistics are kept)
+    const LoneSplit ls = lone_split_plan(T, L, Tc, To, 0, pl.C, lse == nullptr);
+    ap.n_split = ls.n_split;
+    ap.part_o = reinterpret_cast<float*>(ws + pl.part);
+    ap.part_ml = ap.part_o + (size_t)BH * pl.C * kMaxLoneSplit * 128 * d.D;
+    RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, dim3(ls.slots, BH, pl.C), st,
+                                  nullptr, nullptr, behind_phiq));
+    if (ap.n_split > 1) RH_TRY(launch_lone_combine(ap, BH, pl.C, st));
+    return REHYAT_OK;
   }
   rehyat::fp32::AttnParams ap{};
   ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
@@ -1098,8 +1156,15 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
   ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
+  // the lone last tile (odd tile count) runs as parts of its key window
+  const int q_tiles = (pl.nq + 127) / 128;
+  const int key_tiles = (int)((w.split + 127) / 128 + (pl.nkv - w.split + 127) / 128);
+  ap.n_split = (q_tiles & 1) ? lone_split_count(key_tiles) : 1;
+  ap.part_o = reinterpret_cast<float*>(ws + pl.part);
+  ap.part_ml = ap.part_o + (size_t)BH * kMaxLoneSplit * 128 * d.D;
   RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
-                                dim3((pl.nq + 255) / 256, BH, 1), st, &mkc, &mvc, true));
+                                dim3(q_tiles / 2 + ((q_tiles & 1) ? ap.n_split : 0), BH, 1), st,
+                                &mkc, &mvc, true));
   if (pl.fold_rows > 0) {
     // the fold reads only the window and writes its own partials: it runs in the attention's
     // last wave; the state update after it waits for both
@@ -1110,6 +1175,7 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
     fp.splits = pl.splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
     RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(pl.splits, 1, BH), st, &mkc, &mvc, true));
   }
+  if (ap.n_split > 1) RH_TRY(launch_lone_combine(ap, BH, 1, st));
   const int n_add = pl.fold_rows > 0 ? (d.F * d.D + 255) / 256 : 0;
   if (cc && cc->n_vec > 0) {
     long long n_copy = (2 * cc->n_vec + 255) / 256;
@@ -1415,10 +1481,14 @@ int rehyat_segment_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
   ap.bq = nullptr;  // phi_q comes finished from the workspace
   ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
   ap.out = static_cast<__nv_bfloat16*>(out_seg);
-  const int rows_per_chunk = (Tc < ap.T ? Tc : ap.T) * L;
-  return launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap,
-                                dim3((rows_per_chunk + 255) / 256, BH, pl.n_local), st, nullptr,
-                                nullptr, true);
+  const LoneSplit ls = lone_split_plan(ap.T, L, Tc, To, pl.s0, pl.n_local, true);
+  ap.n_split = ls.n_split;
+  ap.part_o = reinterpret_cast<float*>(ws + pl.part);
+  ap.part_ml = ap.part_o + (size_t)BH * pl.n_local * kMaxLoneSplit * 128 * d.D;
+  RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap, dim3(ls.slots, BH, pl.n_local), st,
+                                nullptr, nullptr, true));
+  if (ap.n_split > 1) RH_TRY(launch_lone_combine(ap, BH, pl.n_local, st));
+  return REHYAT_OK;
 }
 
 int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frames_before,
