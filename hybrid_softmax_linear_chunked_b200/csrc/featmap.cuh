@@ -167,6 +167,47 @@ __global__ void __launch_bounds__(128) featmap_kernel(const Tin* __restrict__ x,
   }
 }
 
+// Compact tensor-core form of the grouped linear u = x Wbd^T, built in shared memory by the CTA
+// that uses it.  The block-diagonal F x D matrix Wbd is covered by TG = min(G, F/16) diagonal
+// tiles of NT = F/TG rows (features) by KT = D/TG columns (input dims): tile t is rows
+// [t NT, (t+1) NT) x columns [t KT, (t+1) KT) of Wbd, and every group's block lies inside one
+// tile (a 16 x 16 tile holds two 8 x 8 blocks when G = 16).  The tiles are stored side by side
+// as one [NT][D] bf16 matrix in the 128-byte-swizzled K-major layout of an MMA B operand (row n,
+// column d = tile t's column d - t KT), twice: hi = bf16(w) and lo = bf16(w - hi).  u's columns
+// [t NT, (t+1) NT) are then the MMAs of tile t's KT / 16 K steps with N = NT: D / 16 MMAs per
+// part whatever G is, against 8 full-width ones for the dense matrix.
+struct CompactW {
+  int TG, NT, KT;
+};
+__host__ __device__ __forceinline__ CompactW compact_w(int F, int D, int G) {
+  const int tg = G < F / 16 ? G : F / 16;
+  return {tg, F / tg, D / tg};
+}
+// Bytes of one part (hi or lo) of the compact matrix.
+__host__ __device__ __forceinline__ int compact_w_bytes(int F, int D, int G) {
+  return compact_w(F, D, G).NT * D * 2;
+}
+
+// Writes both parts of head h's compact matrix (W of that head: [G][F/G][D/G] fp32) into shared
+// memory at hi and lo (1024-byte aligned); threads tid = 0 .. nthreads-1 share the work.  The
+// caller makes the stores visible to the tensor cores (fence.proxy.async + a CTA barrier).
+__device__ __forceinline__ void build_compact_w(const float* __restrict__ W, int F, int D, int G,
+                                                uint8_t* hi, uint8_t* lo, int tid, int nthreads) {
+  const CompactW cw = compact_w(F, D, G);
+  const int Fg = F / G, Dg = D / G;
+  for (int e = tid; e < cw.NT * D; e += nthreads) {
+    const int n = e / D, d = e - n * D;
+    const int f = (d / cw.KT) * cw.NT + n;  // feature of row n in the tile that column d is in
+    const int g = f / Fg;
+    const float w = (d / Dg == g) ? W[f * Dg + (d - g * Dg)] : 0.f;
+    const __nv_bfloat16 wh = __float2bfloat16_rn(w);
+    const __nv_bfloat16 wl = __float2bfloat16_rn(w - __bfloat162float(wh));
+    const uint32_t off = sm100::sw128_offset(n, d, cw.NT);
+    *reinterpret_cast<__nv_bfloat16*>(hi + off) = wh;
+    *reinterpret_cast<__nv_bfloat16*>(lo + off) = wl;
+  }
+}
+
 // Block-diagonal form of the grouped linear for the tensor cores: for head h, the dense
 // F x D matrix Wbd[f][d] = W[g][f - g F/G][d - g D/G] when d lies in f's group g, else 0, split
 // into bf16 hi = bf16(Wbd) and lo = bf16(Wbd - hi) so that x.Wbd^T from two bf16 MMAs with fp32

@@ -1,8 +1,9 @@
 // Feature map phi of the "ReHyAt overview" page §2.2.2 for many bf16 rows, on the tensor cores:
-// u = x Wbd^T (block-diagonal grouped 1x1 linear, bf16 hi + lo weight parts, fp32 in TMEM) by
-// tcgen05, then bias, softplus and the part powers on the CUDA cores, written as bf16 rows.
-// Used for phi_q of the query rows that read a linear state, so that the attention kernel's
-// epilogue only has to load a finished phi_q tile.
+// u = x Wbd^T (the grouped 1x1 linear as the compact block-diagonal matrix of featmap.cuh, bf16 hi
+// + lo parts built in shared memory from the fp32 weights, fp32 in TMEM) by tcgen05, then bias,
+// softplus and the part powers on the CUDA cores, written as bf16 rows.  Used for phi_q of the
+// query rows that read a linear state, so that the attention kernel's epilogue only has to load
+// a finished phi_q tile.
 #pragma once
 
 #include "featmap.cuh"
@@ -20,20 +21,28 @@ constexpr int kThreads = 320;  // warps 0-7 feature map, 8 producer, 9 MMA
 constexpr int kPhiThreads = 256;
 constexpr int kTileBytes = kRows * kHD * 2;
 
-constexpr uint32_t kOffX = 0;                          // 2 stages
-constexpr uint32_t kOffW = kOffX + 2 * kTileBytes;      // block-diagonal W, hi and lo
-constexpr uint32_t kOffB = kOffW + 2 * kTileBytes;      // bias, F fp32
-constexpr uint32_t kOffPw = kOffB + kFD * 4;            // part power of each feature, uint8
-constexpr uint32_t kSmemBytes = kOffPw + kFD + 1024;    // + alignment slack
+// Shared memory of the instance for G >= 2 (compact weights of at most 64 rows: 16 KB per part;
+// two CTAs per SM) or for G = 1 (the full 128 x 128 matrix: 32 KB per part; one CTA per SM).
+template <bool kDense>
+struct Layout {
+  static constexpr uint32_t kWPart = kDense ? 32768 : 16384;
+  static constexpr uint32_t kOffX = 0;                          // 2 stages
+  static constexpr uint32_t kOffW = kOffX + 2 * kTileBytes;      // compact W: hi, then lo
+  static constexpr uint32_t kOffB = kOffW + 2 * kWPart;          // bias, F fp32
+  static constexpr uint32_t kOffPw = kOffB + kFD * 4;            // part power of each feature
+  static constexpr uint32_t kSmemBytes = kOffPw + kFD + 1024;    // + alignment slack
+  static constexpr int kCtasPerSm = kDense ? 1 : 2;
+};
 
-enum Bar { kXFull = 0, kXEmpty = 2, kUFull = 4, kUEmpty = 6, kWbFull = 8, kDone = 9, kNumBars = 10 };
+enum Bar { kXFull = 0, kXEmpty = 2, kUFull = 4, kUEmpty = 6, kDone = 8, kNumBars = 9 };
 
 struct Params {
   int row0;           // first row (of each (b, h) sequence) to map
   int n_rows;         // rows to map, starting at row0
   int rows_per_bh;    // rows of each (b, h) in x and phi
   int tiles_per_cta;  // 128-row tiles per CTA (blockIdx.x picks a run of them)
-  int H, P;
+  int H, P, G;
+  const float* W;     // [H, G, F/G, D/G] fp32
   const float* bias;  // [H, F] or null
   __nv_bfloat16* phi; // [BH, rows_per_bh, F]
 };
@@ -44,10 +53,12 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 // grid (ceil(n_tiles / tiles_per_cta), BH), block 320.  Feature-map thread tid owns row
 // (tid & 127) = TMEM lane and features [64 (tid >> 7), +64).
-__global__ void __launch_bounds__(kThreads, 1)
-    featmap_tc_kernel(const __grid_constant__ CUtensorMap tmX,
-                      const __grid_constant__ CUtensorMap tmW, const Params p) {
-  static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
+template <bool kDense>
+__global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
+    featmap_tc_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
+  using Lay = Layout<kDense>;
+  static_assert(Lay::kSmemBytes + 256 <= 232448 / Lay::kCtasPerSm,
+                "shared memory (dynamic + static) over the limit");
   // the attention launched behind this kernel may start at once: it reads phi_q only after
   // waiting for this grid
   grid_dep_signal();
@@ -63,8 +74,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   volatile int* abort_flag = &abort_sh;
-  float* sB = reinterpret_cast<float*>(sm + kOffB);
-  uint8_t* sPw = sm + kOffPw;
+  float* sB = reinterpret_cast<float*>(sm + Lay::kOffB);
+  uint8_t* sPw = sm + Lay::kOffPw;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (warp == 8) {
@@ -81,6 +92,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     sB[i] = p.bias ? p.bias[(size_t)h * kFD + i] : 0.f;
     sPw[i] = static_cast<uint8_t>(feature_power(i, kFD, p.P));
   }
+  build_compact_w(p.W + (size_t)h * kFD * kHD / p.G, kFD, kHD, p.G, sm + Lay::kOffW,
+                  sm + Lay::kOffW + Lay::kWPart, tid, kThreads);
+  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -89,15 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 8) {
     // ---- producer ----
-    if (leader) {
-      tma_prefetch_desc(&tmX);
-      mbar_arrive_expect_tx(&bars[kWbFull], 2 * kTileBytes);
-      for (int part = 0; part < 2; ++part) {
-        uint8_t* dst = sm + kOffW + part * kTileBytes;
-        tma_load_3d(dst, &tmW, &bars[kWbFull], 0, 0, h * 2 + part);
-        tma_load_3d(dst + kRows * 128, &tmW, &bars[kWbFull], 64, 0, h * 2 + part);
-      }
-    }
+    if (leader) tma_prefetch_desc(&tmX);
     __syncwarp();
     bool ok = true;
     int issued = 0;
@@ -107,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kXEmpty + s], ((i >> 1) - 1) & 1, abort_flag));
       if (!ok) break;
       if (leader) {
-        uint8_t* dx = sm + kOffX + s * kTileBytes;
+        uint8_t* dx = sm + Lay::kOffX + s * kTileBytes;
         mbar_arrive_expect_tx(&bars[kXFull + s], kTileBytes);
         tma_load_3d(dx, &tmX, &bars[kXFull + s], 0, row, bh);
         tma_load_3d(dx + kRows * 128, &tmX, &bars[kXFull + s], 64, row, bh);
@@ -116,21 +122,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++issued;
     }
     if (!ok) {
-      mbar_wait_drain(&bars[kWbFull], 0);
       for (int i = max(0, issued - 2); i < issued; ++i)
         mbar_wait_drain(&bars[kXFull + (i & 1)], (i >> 1) & 1);
     }
     __syncwarp();
   } else if (warp == 9) {
-    // ---- MMA issuer: U[s] = X_i Wbd_hi^T + X_i Wbd_lo^T ----
-    const uint32_t id_u = idesc_bf16(kRows, kFD, false, false);
-    const uint64_t dX0 = sdesc_sw128(smem_u32(sm + kOffX), 16, 1024);
-    const uint64_t dW0 = sdesc_sw128(smem_u32(sm + kOffW), 16, 1024);
-    auto koff = [](int kk) { return (uint64_t)((kk >> 2) * (kRows * 128 / 16) + (kk & 3) * 2); };
+    // ---- MMA issuer: U[s] = X_i Wbd_hi^T + X_i Wbd_lo^T, tile by tile of the compact W ----
+    const CompactW cw = compact_w(kFD, kHD, p.G);
+    const uint32_t id_u = idesc_bf16(kRows, cw.NT, false, false);
+    const uint64_t dX0 = sdesc_sw128(smem_u32(sm + Lay::kOffX), 16, 1024);
+    const uint64_t dW0 = sdesc_sw128(smem_u32(sm + Lay::kOffW), 16, 1024);
+    auto koff = [](int kk, int rows) {
+      return (uint64_t)((kk >> 2) * (rows * 128 / 16) + (kk & 3) * 2);
+    };
     auto wait = [&](int b, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(&bars[b], parity, abort_flag));
     };
-    bool ok = wait(kWbFull, 0);
+    bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
       const int s = i & 1;
       ok = wait(kXFull + s, (i >> 1) & 1);
@@ -139,12 +147,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (leader) {
         const uint64_t dx = dX0 + (uint64_t)(s * kTileBytes / 16);
-#pragma unroll
-        for (int part = 0; part < 2; ++part)
-#pragma unroll
-          for (int kk = 0; kk < kHD / 16; ++kk)
-            mma_ss(tmem + s * 128, dx + koff(kk), dW0 + (uint64_t)(part * kTileBytes / 16) + koff(kk),
-                   id_u, (part > 0 || kk > 0) ? 1u : 0u);
+        const int ks_per_tile = cw.KT / 16;
+        for (int part = 0; part < 2; ++part) {
+          const uint64_t dw = dW0 + (uint64_t)(part * Lay::kWPart / 16);
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            const int t = kk / ks_per_tile, ks = kk - t * ks_per_tile;
+            mma_ss(tmem + s * 128 + t * cw.NT, dx + koff(kk, kRows), dw + koff(kk, cw.NT), id_u,
+                   (part > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
         mma_commit(&bars[kUFull + s]);
         mma_commit(&bars[kXEmpty + s]);
       }

@@ -474,47 +474,60 @@ int launch_lone_combine(const rehyat::attn::Params& ap, int BH, int n_chunks, cu
 }
 
 // phi of rows [row0, row0 + n_rows) of every (b, h) sequence of x (rows_per_bh rows each) into
-// phi ([BH][rows_per_bh][F] bf16) on the tensor cores; `mw` maps the block-diagonal weights.
-int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int row0, int n_rows,
-                      const CUtensorMap& mw, const float* bias, __nv_bfloat16* phi,
-                      cudaStream_t st) {
-  if (n_rows <= 0) return REHYAT_OK;
+// phi ([BH][rows_per_bh][F] bf16) on the tensor cores; W are the fp32 weights [H][G][F/G][D/G]
+// (each CTA builds its head's compact block-diagonal matrix in shared memory).
+template <bool kDense>
+int launch_featmap_tc_inst(const rehyat_dims& d, const CUtensorMap& mx, int n_rows,
+                           rehyat::phi::Params pp, cudaStream_t st) {
+  using Lay = rehyat::phi::Layout<kDense>;
   const int BH = d.B * d.H;
-  CUtensorMap mx;
-  RH_TRY(make_map(&mx, x, d.D, rows_per_bh, BH));
   const int n_tiles = (n_rows + 127) / 128;
-  // one wave (one CTA per SM): as many CTAs per (b, h) as fit in 148
-  const int ctas_per_bh = BH < 148 ? 148 / BH : 1;
+  // one wave: as many CTAs per (b, h) as fit on the 148 SMs
+  const int slots = 148 * Lay::kCtasPerSm;
+  const int ctas_per_bh = BH < slots ? slots / BH : 1;
   int per_cta = (n_tiles + ctas_per_bh - 1) / ctas_per_bh;
   if (per_cta < 1) per_cta = 1;
   if (per_cta > n_tiles) per_cta = n_tiles;
-  rehyat::phi::Params pp{};
-  pp.row0 = row0; pp.n_rows = n_rows; pp.rows_per_bh = rows_per_bh; pp.tiles_per_cta = per_cta;
-  pp.H = d.H; pp.P = kernel_P(d); pp.bias = bias; pp.phi = phi;
-  auto k = rehyat::phi::featmap_tc_kernel;
+  pp.tiles_per_cta = per_cta;
+  auto k = rehyat::phi::featmap_tc_kernel<kDense>;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)rehyat::phi::kSmemBytes),
+                                         (int)Lay::kSmemBytes),
                     "featmap_tc attr"));
-  k<<<dim3((n_tiles + per_cta - 1) / per_cta, BH), rehyat::phi::kThreads, rehyat::phi::kSmemBytes,
-      st>>>(mx, mw, pp);
+  k<<<dim3((n_tiles + per_cta - 1) / per_cta, BH), rehyat::phi::kThreads, Lay::kSmemBytes, st>>>(
+      mx, pp);
   return cuda_check(cudaGetLastError(), "featmap_tc launch");
+}
+
+int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int row0, int n_rows,
+                      const float* W, const float* bias, __nv_bfloat16* phi, cudaStream_t st) {
+  if (n_rows <= 0) return REHYAT_OK;
+  CUtensorMap mx;
+  RH_TRY(make_map(&mx, x, d.D, rows_per_bh, (long long)d.B * d.H));
+  rehyat::phi::Params pp{};
+  pp.row0 = row0; pp.n_rows = n_rows; pp.rows_per_bh = rows_per_bh;
+  pp.H = d.H; pp.P = kernel_P(d); pp.G = d.G; pp.W = W; pp.bias = bias; pp.phi = phi;
+  // the G = 1 matrix is dense (32 KB per part): its instance runs one CTA per SM
+  if (rehyat::compact_w(d.F, d.D, d.G).NT > 64)
+    return launch_featmap_tc_inst<true>(d, mx, n_rows, pp, st);
+  return launch_featmap_tc_inst<false>(d, mx, n_rows, pp, st);
 }
 
 // behind_attention: launch with programmatic stream serialization right after an attention
 // launch, so the fold starts once every attention CTA is resident (the kernel waits for the
 // attention grid before it exits).
-int launch_fold_bf16(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mw,
+template <int kKSt>
+int launch_fold_inst(const CUtensorMap& mk, const CUtensorMap& mv,
                      const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st,
-                     const CUtensorMap* mkc = nullptr, const CUtensorMap* mvc = nullptr,
-                     bool behind_attention = false) {
-  auto k = rehyat::state::fold_partial_bf16_kernel;
+                     const CUtensorMap* mkc, const CUtensorMap* mvc, bool behind_attention) {
+  using Lay = rehyat::state::FoldLayout<kKSt>;
+  auto k = rehyat::state::fold_partial_bf16_kernel<kKSt>;
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)rehyat::state::kSmemBytes),
+                                         (int)Lay::kSmemBytes),
                     "fold attr"));
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(rehyat::state::kThreads);
-  cfg.dynamicSmemBytes = rehyat::state::kSmemBytes;
+  cfg.dynamicSmemBytes = Lay::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -522,7 +535,18 @@ int launch_fold_bf16(const CUtensorMap& mk, const CUtensorMap& mv, const CUtenso
   cfg.attrs = attr;
   cfg.numAttrs = behind_attention ? 1 : 0;
   const CUtensorMap kc = mkc ? *mkc : mk, vc = mvc ? *mvc : mv;
-  return cuda_check(cudaLaunchKernelEx(&cfg, k, mk, mv, mw, kc, vc, fp), "fold launch");
+  return cuda_check(cudaLaunchKernelEx(&cfg, k, mk, mv, kc, vc, fp), "fold launch");
+}
+
+// The fold kernel over `grid` (splits, folds, BH); fp.W / fp.G are the fp32 weights of phi_k.
+int launch_fold_bf16(const CUtensorMap& mk, const CUtensorMap& mv,
+                     const rehyat::state::FoldParams& fp, dim3 grid, cudaStream_t st,
+                     const CUtensorMap* mkc = nullptr, const CUtensorMap* mvc = nullptr,
+                     bool behind_attention = false) {
+  // two K stages unless the weights are the dense G = 1 matrix
+  if (rehyat::compact_w(rehyat::state::kFD, rehyat::state::kHD, fp.G).NT > 64)
+    return launch_fold_inst<1>(mk, mv, fp, grid, st, mkc, mvc, behind_attention);
+  return launch_fold_inst<2>(mk, mv, fp, grid, st, mkc, mvc, behind_attention);
 }
 
 // Block-diagonal bf16 hi/lo weights of one feature map into `out` ([H][2][F][D] bf16) and the
@@ -556,15 +580,14 @@ int forward_states_bf16(const rehyat_dims& d, int T, int L, int Tc, int To, cons
   float* dS = reinterpret_cast<float*>(ws + pl.dS);
   float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
   if (pl.n_fold > 0) {
-    CUtensorMap mk, mv, mw;
+    CUtensorMap mk, mv;
     RH_TRY(make_map(&mk, k, d.D, N, BH));
     RH_TRY(make_map(&mv, v, d.D, N, BH));
-    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mw, st));
     rehyat::state::FoldParams fp{};
     fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.T = T; fp.Tc = Tc; fp.To = To; fp.kv_frame0 = 0;
     fp.single_rows = -1; fp.n_fold = pl.n_fold; fp.splits = pl.splits;
-    fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
-    RH_TRY(launch_fold_bf16(mk, mv, mw, fp, dim3(pl.splits, pl.n_fold, BH), st));
+    fp.G = d.G; fp.W = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(mk, mv, fp, dim3(pl.splits, pl.n_fold, BH), st));
   }
   return launch_scan_bf16(d, dS, dZ, pl.n_fold, pl.splits, pl.C, nullptr, nullptr, St, Zc, S_out,
                           Z_out, st);
@@ -804,12 +827,10 @@ int rehyat_forward_phiq(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, in
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const long long N = (long long)T * L;
   if (dt == REHYAT_BF16) {
-    CUtensorMap mw;
-    RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mw, st));
     // phi_q of every query row whose chunk has a linear region: chunks c >= To / Tc + 1
     const long long row_lin = (long long)(To / Tc + 1) * Tc * L;
     if (row_lin < N)
-      RH_TRY(launch_featmap_tc(d, q, (int)N, (int)row_lin, (int)(N - row_lin), mw, bq,
+      RH_TRY(launch_featmap_tc(d, q, (int)N, (int)row_lin, (int)(N - row_lin), Wq, bq,
                                reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16), st));
     return REHYAT_OK;
   }
@@ -976,6 +997,14 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
   // states S_c (transposed, bf16), Z_c and phi_q of the rows that read a state, as the forward
   RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, fw, pl.fwd_bytes, stream));
   RH_TRY(rehyat_forward_phiq(d, dt, T, L, Tc, To, q, Wq, bq, fw, pl.fwd_bytes, stream));
+  // the block-diagonal weights (bf16 hi, lo) of both feature maps for the gradient GEMMs
+  {
+    CUtensorMap unused;
+    RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(fw + pl.fwd.Wqbd), &unused,
+                             st));
+    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(fw + pl.fwd.Wkbd), &unused,
+                             st));
+  }
   const __nv_bfloat16* St = reinterpret_cast<const __nv_bfloat16*>(fw + pl.fwd.St);
   const float* Zc = reinterpret_cast<const float*>(fw + pl.fwd.Zc);
   const __nv_bfloat16* phiq = reinterpret_cast<const __nv_bfloat16*>(fw + pl.fwd.phiq_bf16);
@@ -983,11 +1012,7 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
   const __nv_bfloat16* Wkbd = reinterpret_cast<const __nv_bfloat16*>(fw + pl.fwd.Wkbd);
   // the key rows that some later chunk reads linearly: [0, w_{C-1} L)
   const long long wl = (long long)((C - 1) * Tc - To > 0 ? (C - 1) * Tc - To : 0) * L;
-  if (wl > 0) {
-    CUtensorMap mwk;
-    RH_TRY(make_map(&mwk, Wkbd, d.D, d.F, 2LL * d.H));
-    RH_TRY(launch_featmap_tc(d, k, (int)N, 0, (int)wl, mwk, bk, b16(pl.phik), st));
-  }
+  if (wl > 0) RH_TRY(launch_featmap_tc(d, k, (int)N, 0, (int)wl, Wk, bk, b16(pl.phik), st));
   rehyat::bwd::rowstats_kernel<<<(unsigned)((BH * N + 7) / 8), 256, 0, st>>>(
       dob, static_cast<const __nv_bfloat16*>(out), lse, BH * N, d.D, f32(pl.Drow), f32(pl.lam));
   RH_TRY(cuda_check(cudaGetLastError(), "row statistics launch"));
@@ -1126,7 +1151,7 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
   float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
   // S^T in bf16 for the readout MMA (C = 1, no folds: a transposed copy of S)
   RH_TRY(launch_scan_bf16(d, dS, dZ, 0, 1, 1, S, Z, St, nullptr, nullptr, nullptr, st));
-  CUtensorMap mq, mk, mv, mkc, mvc, ms, mwq, mwk;
+  CUtensorMap mq, mk, mv, mkc, mvc, ms;
   RH_TRY(make_map(&mq, q, d.D, pl.nq, BH));
   RH_TRY(make_map(&mk, w.k, d.D, w.rows, BH));
   RH_TRY(make_map(&mv, w.v, d.D, w.rows, BH));
@@ -1138,13 +1163,10 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
     mvc = mv;
   }
   RH_TRY(make_map(&ms, St, d.F, d.D, BH));
-  RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mwq, st));
-  if (pl.fold_rows > 0)
-    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mwk, st));
   __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
   // phi_q right before the attention, which overlaps it
   if (frames_before - pl.o > 0)  // the chunk reads a linear state
-    RH_TRY(launch_featmap_tc(d, q, pl.nq, 0, pl.nq, mwq, bq, phiq, st));
+    RH_TRY(launch_featmap_tc(d, q, pl.nq, 0, pl.nq, Wq, bq, phiq, st));
   CUtensorMap mphi;
   RH_TRY(make_map(&mphi, phiq, d.F, pl.nq, BH));
   rehyat::attn::Params ap{};
@@ -1162,7 +1184,8 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
   ap.n_split = (q_tiles & 1) ? lone_split_count(key_tiles) : 1;
   ap.part_o = reinterpret_cast<float*>(ws + pl.part);
   ap.part_ml = ap.part_o + (size_t)BH * kMaxLoneSplit * 128 * d.D;
-  RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mwq, mphi, ap,
+  // (the weight map is unused: phi_q comes finished from the workspace)
+  RH_TRY(launch_attn_bf16<true>(mq, mk, mv, ms, mq, mphi, ap,
                                 dim3(q_tiles / 2 + ((q_tiles & 1) ? ap.n_split : 0), BH, 1), st,
                                 &mkc, &mvc, true));
   if (pl.fold_rows > 0) {
@@ -1172,8 +1195,8 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
     fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.single_rows = pl.fold_rows; fp.n_fold = 1;
     fp.seg_rows = pl.fold_rows < w.split ? pl.fold_rows : w.split;
     fp.seg_row0 = w.carry_row0;
-    fp.splits = pl.splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
-    RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(pl.splits, 1, BH), st, &mkc, &mvc, true));
+    fp.splits = pl.splits; fp.G = d.G; fp.W = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(mk, mv, fp, dim3(pl.splits, 1, BH), st, &mkc, &mvc, true));
   }
   if (ap.n_split > 1) RH_TRY(launch_lone_combine(ap, BH, 1, st));
   const int n_add = pl.fold_rows > 0 ? (d.F * d.D + 255) / 256 : 0;
@@ -1415,16 +1438,15 @@ int rehyat_segment_states(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
   float* dS = reinterpret_cast<float*>(ws + pl.dS);
   float* dZ = reinterpret_cast<float*>(ws + pl.dZ);
   if (pl.n_fold > 0) {
-    CUtensorMap mk, mv, mw;
+    CUtensorMap mk, mv;
     RH_TRY(make_map(&mk, k_seg, d.D, pl.nkv_rows, BH));
     RH_TRY(make_map(&mv, v_seg, d.D, pl.nkv_rows, BH));
-    RH_TRY(prepare_blockdiag(d, Wk, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wkbd), &mw, st));
     rehyat::state::FoldParams fp{};
     fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.T = T; fp.Tc = Tc; fp.To = To;
     fp.kv_frame0 = pl.h0; fp.fold_c0 = c0;
     fp.single_rows = -1; fp.n_fold = pl.n_fold; fp.splits = pl.splits;
-    fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
-    RH_TRY(launch_fold_bf16(mk, mv, mw, fp, dim3(pl.splits, pl.n_fold, BH), st));
+    fp.G = d.G; fp.W = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(mk, mv, fp, dim3(pl.splits, pl.n_fold, BH), st));
   }
   rehyat::state::state_sum_kernel<<<dim3((d.F * d.D + 255) / 256, BH), 256, 0, st>>>(
       dS, dZ, pl.n_fold * pl.splits, d.F, d.D, S_seg, Z_seg);
@@ -1458,15 +1480,13 @@ int rehyat_segment_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
                           reinterpret_cast<float*>(ws + pl.Zc), nullptr, nullptr, st,
                           n_prefix));
   // phi_q of the rows whose chunk reads a linear state (chunk c with c*Tc > To)
-  CUtensorMap mw;
-  RH_TRY(prepare_blockdiag(d, Wq, reinterpret_cast<__nv_bfloat16*>(ws + pl.Wqbd), &mw, st));
   int c_lin = To / Tc + 1;
   if (c_lin < c0) c_lin = c0;
   const long long row_lin = (long long)(c_lin - c0) * Tc * L;
   __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
   if (row_lin < pl.nq_rows)
     RH_TRY(launch_featmap_tc(d, q_seg, (int)pl.nq_rows, (int)row_lin,
-                             (int)(pl.nq_rows - row_lin), mw, bq, phiq, st));
+                             (int)(pl.nq_rows - row_lin), Wq, bq, phiq, st));
   CUtensorMap mq, mk, mv, ms, mphi;
   RH_TRY(make_map(&mq, q_seg, d.D, pl.nq_rows, BH));
   RH_TRY(make_map(&mk, k_seg, d.D, pl.nkv_rows, BH));
@@ -1511,8 +1531,10 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   const size_t BH = (size_t)d.B * d.H;
   const size_t st_bytes = round_up(BH * d.D * d.F * 2, 256);
   const size_t wbd_bytes = round_up((size_t)d.H * 2 * d.F * d.D * 2, 256);
+  // S^T, the block-diagonal W_q the attention's epilogue reads (the fold builds its compact
+  // W_k itself), the fold partials
   auto total_for = [&](int splits) {
-    return st_bytes + 2 * wbd_bytes + round_up(BH * splits * d.F * d.D * 4, 256) +
+    return st_bytes + wbd_bytes + round_up(BH * splits * d.F * d.D * 4, 256) +
            round_up(BH * splits * d.F * 4, 256);
   };
   int splits = pl.splits;
@@ -1526,16 +1548,15 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   __nv_bfloat16* St = reinterpret_cast<__nv_bfloat16*>(ws);
   __nv_bfloat16* Wqbd = reinterpret_cast<__nv_bfloat16*>(ws + st_bytes);
-  __nv_bfloat16* Wkbd = reinterpret_cast<__nv_bfloat16*>(ws + st_bytes + wbd_bytes);
-  float* dS = reinterpret_cast<float*>(ws + st_bytes + 2 * wbd_bytes);
-  float* dZ = reinterpret_cast<float*>(ws + st_bytes + 2 * wbd_bytes +
+  float* dS = reinterpret_cast<float*>(ws + st_bytes + wbd_bytes);
+  float* dZ = reinterpret_cast<float*>(ws + st_bytes + wbd_bytes +
                                        round_up(BH * splits * d.F * d.D * 4, 256));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int nbh = d.B * d.H;
   // Nothing in the scratch has to start at zero: every byte a kernel reads was written earlier
   // in this call (S^T by the scan, every split's partial by the fold kernel).
   RH_TRY(launch_scan_bf16(d, dS, dZ, 0, 1, 1, S, Z, St, nullptr, nullptr, nullptr, st));
-  CUtensorMap mq, mk, mv, ms, mwq, mwk;
+  CUtensorMap mq, mk, mv, ms, mwq;
   RH_TRY(make_map(&mq, q, d.D, pl.nq, nbh));
   RH_TRY(make_map(&mk, k_win, d.D, pl.nkv, nbh));
   RH_TRY(make_map(&mv, v_win, d.D, pl.nkv, nbh));
@@ -1550,11 +1571,10 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3((pl.nq + 255) / 256, nbh, 1),
                                  st));
   if (pl.fold_rows > 0) {
-    RH_TRY(prepare_blockdiag(d, Wk, Wkbd, &mwk, st));
     rehyat::state::FoldParams fp{};
     fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.single_rows = pl.fold_rows; fp.n_fold = 1;
-    fp.splits = splits; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
-    RH_TRY(launch_fold_bf16(mk, mv, mwk, fp, dim3(splits, 1, nbh), st));
+    fp.splits = splits; fp.G = d.G; fp.W = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
+    RH_TRY(launch_fold_bf16(mk, mv, fp, dim3(splits, 1, nbh), st));
     rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, nbh), 256, 0, st>>>(
         dS, dZ, splits, d.F, d.D, S, Z);
     RH_TRY(cuda_check(cudaGetLastError(), "state add launch"));

@@ -3,10 +3,12 @@
 //
 //  * fold_partial_bf16_kernel: for one fold range of key rows (the frames leaving a chunk's
 //    softmax window) and one split of it, dS = phi_k(K)^T V (F x D) and dZ = phi_k(K)^T 1 on the
-//    tensor cores.  The grouped linear of phi_k is a tensor-core product too (block-diagonal
-//    weights); the CUDA cores apply bias, softplus and powers and write phi_k straight into the
-//    shared-memory layout of an MN-major MMA operand; both sums accumulate in TMEM in fp32 over
-//    the split's 128-token tiles.
+//    tensor cores.  The grouped linear of phi_k is a tensor-core product too (the compact
+//    block-diagonal weights of featmap.cuh, built by the CTA in shared memory); the CUDA cores
+//    apply bias, softplus and powers and write phi_k straight into the shared-memory layout of an
+//    MN-major MMA operand; both sums accumulate in TMEM in fp32 over the split's 128-token
+//    tiles.  The compact weights leave room for two K stages, so the next K tile loads while the
+//    current one is still being multiplied (the dense G = 1 matrix keeps one).
 //  * state_scan_kernel: exclusive prefix over fold ranges (the state chunk c reads), written as
 //    a transposed bf16 copy S_c^T [D][F] for the attention kernel's readout MMA, plus fp32 Z_c
 //    (and fp32 S_c on request).
@@ -24,25 +26,35 @@ using namespace sm100;
 constexpr int kTok = 128;  // tokens per tile (MMA K)
 constexpr int kHD = 128;
 constexpr int kFD = 128;
-constexpr int kThreads = 320;   // warps 0-7 feature map, 8 producer, 9 MMA
-constexpr int kPhiThreads = 256;
+// warps 0-15 feature map (four per 32-lane TMEM group, 32 features each), 16 producer, 17 MMA:
+// sixteen feature-map warps keep enough independent softplus chains in flight per SM
+constexpr int kPhiWarps = 16;
+constexpr int kPhiThreads = kPhiWarps * 32;
+constexpr int kWarpProducer = kPhiWarps, kWarpMma = kPhiWarps + 1;
+constexpr int kThreads = kPhiThreads + 64;
 constexpr int kTileBytes = kTok * kHD * 2;
 
-constexpr uint32_t kOffK = 0;                           // 1 stage (consumed early by the U MMA)
-constexpr uint32_t kOffV = kOffK + kTileBytes;           // 2 stages
-constexpr uint32_t kOffPhi = kOffV + 2 * kTileBytes;     // 2 stages
-constexpr uint32_t kOffW = kOffPhi + 2 * kTileBytes;     // block-diagonal W_k, hi and lo
-constexpr uint32_t kOffOnes = kOffW + 2 * kTileBytes;    // 8 rows x 128 B of bf16 1.0
-constexpr uint32_t kOffB = kOffOnes + 1024;              // bias of phi_k, F fp32
-constexpr uint32_t kOffPw = kOffB + kFD * 4;             // part power of each feature, uint8
-constexpr uint32_t kSmemBytes = kOffPw + kFD + 1024;      // + alignment slack
+// Shared memory with kKSt K stages: 2 with the compact weights of G >= 2 (at most 64 rows,
+// 16 KB per part), 1 with the dense G = 1 matrix (32 KB per part).
+template <int kKSt>
+struct FoldLayout {
+  static constexpr uint32_t kWPart = kKSt == 2 ? 16384 : 32768;
+  static constexpr uint32_t kOffK = 0;                           // kKSt stages
+  static constexpr uint32_t kOffV = kOffK + kKSt * kTileBytes;    // 2 stages
+  static constexpr uint32_t kOffPhi = kOffV + 2 * kTileBytes;     // 2 stages
+  static constexpr uint32_t kOffW = kOffPhi + 2 * kTileBytes;     // compact W_k: hi, then lo
+  static constexpr uint32_t kOffOnes = kOffW + 2 * kWPart;        // 8 rows x 128 B of bf16 1.0
+  static constexpr uint32_t kOffB = kOffOnes + 1024;              // bias of phi_k, F fp32
+  static constexpr uint32_t kOffPw = kOffB + kFD * 4;             // part power of each feature
+  static constexpr uint32_t kSmemBytes = kOffPw + kFD + 1024;     // + alignment slack
+};
 
 // TMEM columns: U buffers [0,128) and [128,256), dS [256,384), dZ [384,400).
 constexpr uint32_t kColDS = 256, kColDZ = 384;
 
 enum Bar {
-  kKFull = 0, kKEmpty = 1, kVFull = 2, kVEmpty = 4, kUFull = 6, kUEmpty = 8, kPhiFull = 10,
-  kPhiEmpty = 12, kWbFull = 14, kDone = 15, kNumBars = 16
+  kKFull = 0, kKEmpty = 2, kVFull = 4, kVEmpty = 6, kUFull = 8, kUEmpty = 10, kPhiFull = 12,
+  kPhiEmpty = 14, kDone = 16, kNumBars = 17
 };
 
 struct FoldParams {
@@ -55,6 +67,8 @@ struct FoldParams {
   // tiled on its own.  seg_rows = 0: one segment.
   int seg_rows, seg_row0;
   int n_fold, splits;
+  int G;
+  const float* W;   // [H, G, F/G, D/G] fp32 weights of phi_k
   const float* bk;
   float* dS;  // [BH][n_fold][splits][F][D]
   float* dZ;  // [BH][n_fold][splits][F]
@@ -80,13 +94,14 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_addr, int kk) {
 // cores, fp32 in TMEM); the feature-map warps add the bias, apply softplus and the part powers,
 // and write phi_k as bf16 into the MN-major A operand of dS += phi_k^T V_i and
 // dZ += phi_k^T 1 (a ones matrix as B: N = 16, every row group read from the same 1 KiB).
+template <int kKSt>
 __global__ void __launch_bounds__(kThreads, 1)
     fold_partial_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
                              const __grid_constant__ CUtensorMap tmV,
-                             const __grid_constant__ CUtensorMap tmW,
                              const __grid_constant__ CUtensorMap tmKc,
                              const __grid_constant__ CUtensorMap tmVc, const FoldParams p) {
-  static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
+  using Lay = FoldLayout<kKSt>;
+  static_assert(Lay::kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
   const int split = blockIdx.x, fc = blockIdx.y, bh = blockIdx.z, h = bh % p.H;
   int r0, r1;
   if (p.single_rows >= 0) {
@@ -125,10 +140,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   volatile int* abort_flag = &abort_sh;
-  float* sB = reinterpret_cast<float*>(sm + kOffB);
-  uint8_t* sPw = sm + kOffPw;
+  float* sB = reinterpret_cast<float*>(sm + Lay::kOffB);
+  uint8_t* sPw = sm + Lay::kOffPw;
 
-  if (warp == 8) {
+  if (warp == kWarpProducer) {
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
@@ -145,30 +160,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     sPw[i] = static_cast<uint8_t>(feature_power(i, kFD, p.P));
   }
   {
-    uint32_t* ones = reinterpret_cast<uint32_t*>(sm + kOffOnes);
+    uint32_t* ones = reinterpret_cast<uint32_t*>(sm + Lay::kOffOnes);
     for (int i = tid; i < 256; i += kThreads) ones[i] = 0x3F803F80u;  // bf16 pair (1.0, 1.0)
   }
+  build_compact_w(p.W + (size_t)h * kFD * kHD / p.G, kFD, kHD, p.G, sm + Lay::kOffW,
+                  sm + Lay::kOffW + Lay::kWPart, tid, kThreads);
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t sK0 = smem_u32(sm + kOffK), sV0 = smem_u32(sm + kOffV);  // one K stage
-  const uint32_t sPhi = smem_u32(sm + kOffPhi), sW0 = smem_u32(sm + kOffW);
-  const uint32_t sOnes = smem_u32(sm + kOffOnes);
+  const uint32_t sK0 = smem_u32(sm + Lay::kOffK), sV0 = smem_u32(sm + Lay::kOffV);
+  const uint32_t sPhi = smem_u32(sm + Lay::kOffPhi), sW0 = smem_u32(sm + Lay::kOffW);
+  const uint32_t sOnes = smem_u32(sm + Lay::kOffOnes);
 
   const bool leader = lane == 0;
-  if (warp == 8) {
+  if (warp == kWarpProducer) {
     // ---- producer ----
     if (leader) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bars[kWbFull], 2 * kTileBytes);
-      for (int part = 0; part < 2; ++part) {
-        uint8_t* dst = sm + kOffW + part * kTileBytes;
-        tma_load_3d(dst, &tmW, &bars[kWbFull], 0, 0, h * 2 + part);
-        tma_load_3d(dst + kTok * 128, &tmW, &bars[kWbFull], 64, 0, h * 2 + part);
-      }
     }
     __syncwarp();
     bool ok = true;
@@ -181,20 +192,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = carried ? p.seg_row0 + ti * kTok : r0 + (ti - n_seg) * kTok;
       const CUtensorMap* mK = carried ? &tmKc : &tmK;
       const CUtensorMap* mV = carried ? &tmVc : &tmV;
-      if (i >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKEmpty], (i - 1) & 1, abort_flag));
+      const int sk = i % kKSt;
+      if (i >= kKSt)
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&bars[kKEmpty + sk], ((i / kKSt) - 1) & 1, abort_flag));
       if (!ok) break;
       if (leader) {
-        uint8_t* dk = sm + kOffK;
-        mbar_arrive_expect_tx(&bars[kKFull], kTileBytes);
-        tma_load_3d(dk, mK, &bars[kKFull], 0, row, bh);
-        tma_load_3d(dk + kTok * 128, mK, &bars[kKFull], 64, row, bh);
+        uint8_t* dk = sm + Lay::kOffK + sk * kTileBytes;
+        mbar_arrive_expect_tx(&bars[kKFull + sk], kTileBytes);
+        tma_load_3d(dk, mK, &bars[kKFull + sk], 0, row, bh);
+        tma_load_3d(dk + kTok * 128, mK, &bars[kKFull + sk], 64, row, bh);
       }
       __syncwarp();
       ++issued_k;
       if (i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kVEmpty + s], ((i >> 1) - 1) & 1, abort_flag));
       if (!ok) break;
       if (leader) {
-        uint8_t* dv = sm + kOffV + s * kTileBytes;
+        uint8_t* dv = sm + Lay::kOffV + s * kTileBytes;
         mbar_arrive_expect_tx(&bars[kVFull + s], kTileBytes);
         tma_load_3d(dv, mV, &bars[kVFull + s], 0, row, bh);
         tma_load_3d(dv + kTok * 128, mV, &bars[kVFull + s], 64, row, bh);
@@ -203,15 +217,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++issued_v;
     }
     if (!ok) {
-      mbar_wait_drain(&bars[kWbFull], 0);
-      if (issued_k > 0) mbar_wait_drain(&bars[kKFull], (issued_k - 1) & 1);
+      for (int i = max(0, issued_k - kKSt); i < issued_k; ++i)
+        mbar_wait_drain(&bars[kKFull + i % kKSt], (i / kKSt) & 1);
       for (int i = max(0, issued_v - 2); i < issued_v; ++i)
         mbar_wait_drain(&bars[kVFull + (i & 1)], (i >> 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == kWarpMma) {
     // ---- MMA issuer ----
-    const uint32_t id_u = idesc_bf16(kTok, kFD, false, false);  // K (K-major) x Wbd (K-major)
+    const CompactW cw = compact_w(kFD, kHD, p.G);
+    const uint32_t id_u = idesc_bf16(kTok, cw.NT, false, false);  // K (K-major) x compact Wbd
     const uint32_t id_s = idesc_bf16(kFD, kHD, true, true);     // phi^T (MN) x V (MN)
     const uint32_t id_z = idesc_bf16(kFD, 16, true, false);     // phi^T (MN) x ones (K)
     auto wait = [&](int b, uint32_t parity) {
@@ -233,20 +248,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    bool ok = wait(kWbFull, 0);
+    bool ok = true;
+    const int ks_per_tile = cw.KT / 16;
     for (int i = 0; i < n_tiles && ok; ++i) {
-      const int s = i & 1;
-      ok = wait(kKFull, i & 1);
+      const int s = i & 1, sk = i % kKSt;
+      ok = wait(kKFull + sk, (i / kKSt) & 1);
       if (ok && i >= 2) ok = wait(kUEmpty + s, ((i >> 1) - 1) & 1);
       if (!ok) break;
       tc_fence_after();
       if (leader) {
-        for (int part = 0; part < 2; ++part)
-          for (int kk = 0; kk < kHD / 16; ++kk)
-            mma_ss(tmem + s * 128, kmajor_desc(sK0, kk), kmajor_desc(sW0 + part * kTileBytes, kk),
-                   id_u, (part > 0 || kk > 0) ? 1u : 0u);
+        const uint32_t kb = sK0 + sk * kTileBytes;
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t wb = sW0 + part * Lay::kWPart;
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            // tile t of the compact W fills U's columns [t NT, (t+1) NT)
+            const int t = kk / ks_per_tile, ks = kk - t * ks_per_tile;
+            mma_ss(tmem + s * 128 + t * cw.NT, kmajor_desc(kb, kk),
+                   sdesc_sw128(wb + (kk >> 2) * (cw.NT * 128) + (kk & 3) * 32, 16, 1024), id_u,
+                   (part > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
         mma_commit(&bars[kUFull + s]);
-        mma_commit(&bars[kKEmpty]);
+        mma_commit(&bars[kKEmpty + sk]);
       }
       __syncwarp();
       if (i >= 1) {
@@ -270,10 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait_drain(&bars[kDone], 0);
     __syncwarp();
   } else {
-    // ---- feature-map warps: token row r = TMEM lane, feature half hf ----
+    // ---- feature-map warps: token row r = TMEM lane, feature quarter hf ----
     const int r = tid & 127, hf = tid >> 7;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t col0 = hf * 64;
+    const uint32_t col0 = hf * 32;
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
       const int s = i & 1;
@@ -282,11 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&bars[kPhiEmpty + s], ((i >> 1) - 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint8_t* prow = sm + kOffPhi + s * kTileBytes;
+      uint8_t* prow = sm + Lay::kOffPhi + s * kTileBytes;
       const int ti = t_begin + i;
       const bool valid = ti < n_seg ? ti * kTok + r < seg : r0 + seg + (ti - n_seg) * kTok + r < r1;
 #pragma unroll 1
-      for (int c16 = 0; c16 < 4; ++c16) {  // 16 features per step keeps the loop body small
+      for (int c16 = 0; c16 < 2; ++c16) {  // 16 features per step keeps the loop body small
         const int f0 = col0 + c16 * 16;
         uint32_t uu[16];
         tmem_ld16(tmem + lane_base + s * 128 + f0, uu);
@@ -305,13 +328,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0, abort_flag));
     if (ok) {
       tc_fence_after();
-      // lane r of TMEM is feature f = r: dS row f (this thread writes columns col0 .. col0+63),
+      // lane r of TMEM is feature f = r: dS row f (this thread writes columns col0 .. col0+31),
       // dZ in column kColDZ.
       float* srow = dS + (size_t)r * kHD + col0;
-      uint32_t rr[64];
-      tmem_ld64(tmem + lane_base + kColDS + col0, rr);
+      uint32_t rr[32];
+      tmem_ld32(tmem + lane_base + kColDS + col0, rr);
 #pragma unroll
-      for (int q4 = 0; q4 < 16; ++q4)
+      for (int q4 = 0; q4 < 8; ++q4)
         *reinterpret_cast<float4*>(srow + q4 * 4) =
             make_float4(__uint_as_float(rr[q4 * 4]), __uint_as_float(rr[q4 * 4 + 1]),
                         __uint_as_float(rr[q4 * 4 + 2]), __uint_as_float(rr[q4 * 4 + 3]));
@@ -324,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kWarpProducer) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -197,10 +197,10 @@ int rehyat_chunk_forward_sched(rehyat_dims d, rehyat_dtype dt, int frame_tokens,
  *   - The first call on a device looks up that array's device address (once per device, with
  *     the device current); make that first call before any stream capture.
  *   - Returns REHYAT_ERR_WORKSPACE, before anything is enqueued, when the scratch does not fit
- *     the array.  With one fold split it needs B*H*(6*F*D + 4*F) + 8*H*F*D bytes (S^T, the
- *     fold partials and two block-diagonal weight copies, each part rounded up to 256 B): at
- *     D = F = 128 that is 98,816 bytes per (b, h) plus 131,072 per head, so B*H <= 144 at
- *     H = 12 and B <= 168 at H = 1.  When the token splits rehyat_chunk_forward would use for
+ *     the array.  With one fold split it needs B*H*(6*F*D + 4*F) + 4*H*F*D bytes (S^T, the
+ *     fold partials and one block-diagonal weight copy, each part rounded up to 256 B): at
+ *     D = F = 128 that is 98,816 bytes per (b, h) plus 65,536 per head, so B*H <= 156 at
+ *     H = 12 and B <= 169 at H = 1.  When the token splits rehyat_chunk_forward would use for
  *     the fold do not fit, fewer are used (down to one).
  *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - Every call shares the one array, whatever the stream: calls whose work overlaps on the

@@ -179,12 +179,12 @@ def test_segment_checks(lib):
 
 
 def test_static_chunk_refuses_problems_beyond_its_scratch(lib):
-    """The static-scratch streaming call needs B*H*(6FD + 4F) + 8HFD bytes with one fold split;
+    """The static-scratch streaming call needs B*H*(6FD + 4F) + 4HFD bytes with one fold split;
     past 16 MiB it refuses before anything is enqueued (no device is touched here)."""
     def call(B, H):
         return lib.rehyat_chunk_forward_static(dims(B=B, H=H), rb.REHYAT_BF16, 64, 3, 3, 1, FAKE,
                                                FAKE, FAKE, FAKE, None, FAKE, None, FAKE, FAKE,
                                                FAKE, None)
-    for B, H in [(13, 12), (1, 200), (169, 1)]:
+    for B, H in [(14, 12), (1, 200), (170, 1)]:
         assert call(B, H) == -4, (B, H)
         assert "scratch" in lib.rehyat_last_error().decode()
