@@ -19,7 +19,7 @@ PHI_POLY = 0   # softplus parts raised to powers 1..P
 PHI_ELU1 = 1   # elu(u) + 1
 
 STATUS = {0: "OK", -1: "ERR_ARG", -2: "ERR_SHAPE", -3: "ERR_DTYPE", -4: "ERR_WORKSPACE",
-          -5: "ERR_CUDA", -6: "ERR_TIMEOUT", -7: "ERR_ALIGN"}
+          -5: "ERR_CUDA", -6: "ERR_TIMEOUT", -7: "ERR_ALIGN", -8: "ERR_BOUNDS"}
 
 EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_forward_workspace_size", "rehyat_forward", "rehyat_forward_states",
@@ -28,7 +28,8 @@ EXPORTED = ["rehyat_last_error", "rehyat_version", "rehyat_featmap",
             "rehyat_chunk_forward_carry", "rehyat_chunk_forward_static", "rehyat_chunk_states",
             "rehyat_forward_train", "rehyat_backward_workspace_size", "rehyat_backward",
             "rehyat_gemm_bf16", "rehyat_segment_workspace_size", "rehyat_segment_states",
-            "rehyat_segment_attend", "rehyat_selftest_wait_timeout", "rehyat_sync_status"]
+            "rehyat_segment_attend", "rehyat_selftest_wait_timeout", "rehyat_selftest_bounds",
+            "rehyat_sync_status", "rehyat_debug_bounds"]
 
 
 class RehyatError(RuntimeError):
@@ -47,6 +48,14 @@ _lib = None
 
 def lib_path() -> str:
     return _LIB_PATH
+
+
+def use_library(path: str) -> ctypes.CDLL:
+    """Make every later call go through the library at `path` (for example the debug-bounds
+    build, build.build(debug_bounds=True)); returns it loaded."""
+    global _lib, _LIB_PATH
+    _lib, _LIB_PATH = None, path
+    return load()
 
 
 def load() -> ctypes.CDLL:
@@ -103,6 +112,8 @@ def load() -> ctypes.CDLL:
     L.rehyat_gemm_bf16.argtypes = [c_int, c_int, c_int, c_int, P, LL, LL, c_int, P, LL, LL, c_int,
                                    P, LL, LL, c_int, c_int, ctypes.c_float, P]
     L.rehyat_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
+    L.rehyat_selftest_bounds.argtypes = [P, ctypes.c_longlong, ctypes.c_longlong, P]
+    L.rehyat_debug_bounds.argtypes = []
     L.rehyat_sync_status.argtypes = [P]
     for name in EXPORTED:
         if name not in ("rehyat_last_error",):
@@ -594,6 +605,15 @@ def gemm(A: torch.Tensor, B: torch.Tensor, *, a_mn: bool = False, b_mn: bool = F
                                    int(out.dtype == torch.bfloat16), int(accumulate),
                                    ctypes.c_float(alpha), _stream(dev)))
     return out
+
+
+def selftest_bounds(buf: torch.Tensor, n: int, bad_index: int) -> None:
+    """Enqueue the debug-bounds self test on buf (fp32, at least n + 1 elements past which
+    bad_index must stay)."""
+    if buf.dtype != torch.float32 or buf.numel() <= max(n, bad_index):
+        raise ValueError("buf must be fp32 with room for index max(n, bad_index)")
+    dev = _dev(buf)
+    _check(load().rehyat_selftest_bounds(_ptr(buf), n, bad_index, _stream(dev)))
 
 
 def selftest_wait_timeout(limit_ns: int = 20_000_000, device: torch.device | None = None) -> None:

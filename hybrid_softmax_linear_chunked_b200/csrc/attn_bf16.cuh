@@ -81,6 +81,7 @@ struct Params {
   // its own (its last tile ragged).  kv_split = 0: the whole window is in tmK/tmV.
   int kv_split;
   int carry_row0;
+  int kv_rows, carry_rows;  // rows per (b, h) of the main and of the carried K/V tensor maps
   float scale_log2;   // log2(e) / sqrt(D)
   const float* bq;    // [H, F] or null
   const float* Z;     // [BH, n_states, F]
@@ -275,8 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < (has_t1 ? 2 : 1); ++t) {
         uint8_t* dst = sm + (t ? kOffQ1 : kOffQ0);
         const int row = q_row0 + tile_row0 + t * kBM;
-        tma_load_3d(dst, &tmQ, &bars[kQFull], 0, row, bh);
-        tma_load_3d(dst + kBM * 128, &tmQ, &bars[kQFull], 64, row, bh);
+        tma_load_3d_chk(1, dst, &tmQ, &bars[kQFull], 0, row, bh, kHD, p.nq_rows, n_bh);
+        tma_load_3d_chk(1, dst + kBM * 128, &tmQ, &bars[kQFull], 64, row, bh, kHD, p.nq_rows,
+                        n_bh);
       }
     }
     __syncwarp();
@@ -299,8 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) {
         uint8_t* dk = sm + kOffK + s * kTileBytes;
         mbar_arrive_expect_tx(&bars[kKFull + s], kTileBytes);
-        tma_load_3d(dk, mK, &bars[kKFull + s], 0, row, bh);
-        tma_load_3d(dk + kBM * 128, mK, &bars[kKFull + s], 64, row, bh);
+        const int kv_ext = carried ? p.carry_rows : p.kv_rows;
+        tma_load_3d_chk(2, dk, mK, &bars[kKFull + s], 0, row, bh, kHD, kv_ext, n_bh);
+        tma_load_3d_chk(2, dk + kBM * 128, mK, &bars[kKFull + s], 64, row, bh, kHD, kv_ext, n_bh);
       }
       __syncwarp();
       ++issued_k;
@@ -309,8 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) {
         uint8_t* dv = sm + kOffV + s * kTileBytes;
         mbar_arrive_expect_tx(&bars[kVFull + s], kTileBytes);
-        tma_load_3d(dv, mV, &bars[kVFull + s], 0, row, bh);
-        tma_load_3d(dv + kBM * 128, mV, &bars[kVFull + s], 64, row, bh);
+        const int kv_ext = carried ? p.carry_rows : p.kv_rows;
+        tma_load_3d_chk(3, dv, mV, &bars[kVFull + s], 0, row, bh, kHD, kv_ext, n_bh);
+        tma_load_3d_chk(3, dv + kBM * 128, mV, &bars[kVFull + s], 64, row, bh, kHD, kv_ext, n_bh);
       }
       __syncwarp();
       ++issued_v;
@@ -331,8 +335,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
           uint8_t* dst = sm + kOffK + s * kTileBytes;
           mbar_arrive_expect_tx(&bars[kStFull], kTileBytes);
-          tma_load_3d(dst, &tmSt, &bars[kStFull], 0, 0, bh * p.n_states + c);
-          tma_load_3d(dst + kBM * 128, &tmSt, &bars[kStFull], 64, 0, bh * p.n_states + c);
+          const long long st_depth = (long long)n_bh * p.n_states;
+          tma_load_3d_chk(4, dst, &tmSt, &bars[kStFull], 0, 0, bh * p.n_states + c, kFD, kHD,
+                          st_depth);
+          tma_load_3d_chk(4, dst + kBM * 128, &tmSt, &bars[kStFull], 64, 0, bh * p.n_states + c,
+                          kFD, kHD, st_depth);
         }
         __syncwarp();
         st_issued = true;
@@ -349,8 +356,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < (has_t1 ? 2 : 1); ++t) {
             uint8_t* dst = sm + (t ? kOffQ1 : kOffQ0);
             const int row = q_row0 + tile_row0 + t * kBM;
-            tma_load_3d(dst, &tmPhi, &bars[kPhiqFull], 0, row, bh);
-            tma_load_3d(dst + kBM * 128, &tmPhi, &bars[kPhiqFull], 64, row, bh);
+            tma_load_3d_chk(5, dst, &tmPhi, &bars[kPhiqFull], 0, row, bh, kFD, p.nq_rows, n_bh);
+            tma_load_3d_chk(5, dst + kBM * 128, &tmPhi, &bars[kPhiqFull], 64, row, bh, kFD,
+                            p.nq_rows, n_bh);
           }
         }
         __syncwarp();
@@ -368,8 +376,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&bars[kWbFull], 2 * kTileBytes);
           for (int s = 0; s < 2; ++s) {
             uint8_t* dst = sm + kOffV + s * kTileBytes;
-            tma_load_3d(dst, &tmW, &bars[kWbFull], 0, 0, h * 2 + s);
-            tma_load_3d(dst + kBM * 128, &tmW, &bars[kWbFull], 64, 0, h * 2 + s);
+            tma_load_3d_chk(6, dst, &tmW, &bars[kWbFull], 0, 0, h * 2 + s, kHD, kFD, 2 * p.H);
+            tma_load_3d_chk(6, dst + kBM * 128, &tmW, &bars[kWbFull], 64, 0, h * 2 + s, kHD, kFD,
+                            2 * p.H);
           }
         }
         __syncwarp();
@@ -656,22 +665,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         // one part of a lone tile's window: its rows' unnormalised O and (m, l), every row
         tc_fence_after();
         const size_t slot = ((size_t)c * n_bh + bh) * n_split + part;
+        const bool store_ok = bounds_ok(8, (long long)slot, 0, (long long)gridDim.z * n_bh * n_split);
         float* po = p.part_o + (slot * kBM + r) * kHD;
 #pragma unroll
         for (int cc = 0; cc < kHD / 32; ++cc) {
           uint32_t rr[32];
           tmem_ld32(tO + cc * 32, rr);
+          if (store_ok) {
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
-            *reinterpret_cast<float4*>(po + cc * 32 + q4 * 4) =
-                make_float4(__uint_as_float(rr[q4 * 4]), __uint_as_float(rr[q4 * 4 + 1]),
-                            __uint_as_float(rr[q4 * 4 + 2]), __uint_as_float(rr[q4 * 4 + 3]));
+            for (int q4 = 0; q4 < 8; ++q4)
+              *reinterpret_cast<float4*>(po + cc * 32 + q4 * 4) =
+                  make_float4(__uint_as_float(rr[q4 * 4]), __uint_as_float(rr[q4 * 4 + 1]),
+                              __uint_as_float(rr[q4 * 4 + 2]), __uint_as_float(rr[q4 * 4 + 3]));
+          }
         }
-        *reinterpret_cast<float2*>(p.part_ml + (slot * kBM + r) * 2) = make_float2(m, l);
+        if (store_ok)
+          *reinterpret_cast<float2*>(p.part_ml + (slot * kBM + r) * 2) = make_float2(m, l);
       } else if (ok) {
         tc_fence_after();
         const int row_in_chunk = tile_row0 + t * kBM + r;
-        const bool row_valid = row_in_chunk < nq;
+        const bool row_valid =
+            row_in_chunk < nq && bounds_ok(7, q_row0 + row_in_chunk, 0, p.nq_rows);
         const float inv = 1.f / l;
         if (p.lse && row_valid)
           p.lse[(size_t)bh * p.nq_rows + q_row0 + row_in_chunk] = m + log2f(l);
@@ -716,6 +730,7 @@ __global__ void __launch_bounds__(kHD) lone_combine_kernel(const Params p) {
   const int row_in_chunk = (n_tiles / 2) * 2 * kBM + r;
   if (row_in_chunk >= geo.nq) return;
   const size_t slot0 = ((size_t)c * gridDim.x + bh) * p.n_split;
+  if (!bounds_ok(31, geo.q_row0 + row_in_chunk, 0, p.nq_rows)) return;
   float M = -INFINITY;
   for (int i = 0; i < p.n_split; ++i) M = fmaxf(M, p.part_ml[((slot0 + i) * kBM + r) * 2]);
   float num = 0.f, den = 0.f;

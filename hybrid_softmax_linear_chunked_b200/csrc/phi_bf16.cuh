@@ -115,8 +115,10 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
       if (leader) {
         uint8_t* dx = sm + Lay::kOffX + s * kTileBytes;
         mbar_arrive_expect_tx(&bars[kXFull + s], kTileBytes);
-        tma_load_3d(dx, &tmX, &bars[kXFull + s], 0, row, bh);
-        tma_load_3d(dx + kRows * 128, &tmX, &bars[kXFull + s], 64, row, bh);
+        tma_load_3d_chk(21, dx, &tmX, &bars[kXFull + s], 0, row, bh, kHD, p.rows_per_bh,
+                        gridDim.y);
+        tma_load_3d_chk(21, dx + kRows * 128, &tmX, &bars[kXFull + s], 64, row, bh, kHD,
+                        p.rows_per_bh, gridDim.y);
       }
       __syncwarp();
       ++issued;
@@ -177,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
       if (!ok) break;
       tc_fence_after();
       const int row_in = (t_begin + i) * kRows + r;  // row index inside [row0, row0 + n_rows)
-      const bool valid = row_in < p.n_rows;
+      const bool valid =
+          row_in < p.n_rows && bounds_ok(22, p.row0 + row_in, 0, p.rows_per_bh);
       __nv_bfloat16* dst = p.phi + ((size_t)bh * p.rows_per_bh + p.row0 + row_in) * kFD + col0;
 #pragma unroll 1
       for (int c16 = 0; c16 < 4; ++c16) {

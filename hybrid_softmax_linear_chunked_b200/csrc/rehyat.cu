@@ -586,6 +586,7 @@ int forward_states_bf16(const rehyat_dims& d, int T, int L, int Tc, int To, cons
     rehyat::state::FoldParams fp{};
     fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.T = T; fp.Tc = Tc; fp.To = To; fp.kv_frame0 = 0;
     fp.single_rows = -1; fp.n_fold = pl.n_fold; fp.splits = pl.splits;
+    fp.kv_rows = fp.carry_rows = (int)N;
     fp.G = d.G; fp.W = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
     RH_TRY(launch_fold_bf16(mk, mv, fp, dim3(pl.splits, pl.n_fold, BH), st));
   }
@@ -641,6 +642,16 @@ int static_scratch_for_current_device(void** out) {
   }
   *out = g_static_scratch_ptr[dev];
   return REHYAT_OK;
+}
+
+// Debug-bounds self test: writes 1 to buf[0, n) and then tries buf[bad_index] through the store
+// check (index inside [0, n)), which a debug-bounds build records and skips.  The caller's buffer
+// has room past n, so the write would stay inside it even if the check were missing.
+__global__ void __launch_bounds__(256) bounds_selftest_kernel(float* buf, long long n,
+                                                              long long bad_index) {
+  const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
+  if (i < n) buf[i] = 1.f;
+  if (i == 0 && rehyat::sm100::bounds_ok(99, bad_index, 0, n)) buf[bad_index] = 2.f;
 }
 
 // Exercises the error path of the bounded mbarrier wait: every warp waits on a barrier that
@@ -760,7 +771,15 @@ extern "C" {
 
 const char* rehyat_last_error(void) { return g_msg; }
 
-int rehyat_version(void) { return 101; }
+int rehyat_debug_bounds(void) {
+#ifdef REHYAT_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int rehyat_version(void) { return 102; }
 
 int rehyat_featmap(rehyat_dims d, rehyat_dtype dt, int n_tokens, const void* x, const float* W,
                    const float* bias, void* phi, void* stream) {
@@ -876,6 +895,7 @@ static int forward_attend_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int
     rehyat::attn::Params ap{};
     ap.L = L; ap.T = T; ap.Tc = Tc; ap.To = To; ap.frames_before = 0; ap.kv_frame0 = 0;
     ap.H = d.H; ap.P = kernel_P(d); ap.n_states = pl.C; ap.nq_rows = (int)N;
+    ap.kv_rows = ap.carry_rows = (int)N;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
     ap.bq = nullptr;  // phi_q comes finished from the workspace
     ap.Z = reinterpret_cast<const float*>(ws + pl.Zc);
@@ -1175,6 +1195,8 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
   // the main source's row 0 is window row `split`
   ap.kv_frame0 = frames_before - pl.o + w.split / L;
   ap.kv_split = w.split; ap.carry_row0 = w.carry_row0;
+  ap.kv_rows = (int)w.rows;
+  ap.carry_rows = (int)(w.split > 0 ? w.carry_rows : w.rows);
   ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
@@ -1193,6 +1215,8 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
     // last wave; the state update after it waits for both
     rehyat::state::FoldParams fp{};
     fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.single_rows = pl.fold_rows; fp.n_fold = 1;
+    fp.kv_rows = (int)w.rows;
+    fp.carry_rows = (int)(w.split > 0 ? w.carry_rows : w.rows);
     fp.seg_rows = pl.fold_rows < w.split ? pl.fold_rows : w.split;
     fp.seg_row0 = w.carry_row0;
     fp.splits = pl.splits; fp.G = d.G; fp.W = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
@@ -1445,6 +1469,7 @@ int rehyat_segment_states(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
     fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.T = T; fp.Tc = Tc; fp.To = To;
     fp.kv_frame0 = pl.h0; fp.fold_c0 = c0;
     fp.single_rows = -1; fp.n_fold = pl.n_fold; fp.splits = pl.splits;
+    fp.kv_rows = fp.carry_rows = (int)pl.nkv_rows;
     fp.G = d.G; fp.W = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
     RH_TRY(launch_fold_bf16(mk, mv, fp, dim3(pl.splits, pl.n_fold, BH), st));
   }
@@ -1496,6 +1521,7 @@ int rehyat_segment_attend(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
   rehyat::attn::Params ap{};
   ap.L = L; ap.T = pl.s1 - pl.s0; ap.Tc = Tc; ap.To = To;
   ap.frames_before = pl.s0; ap.kv_frame0 = pl.h0;
+  ap.kv_rows = ap.carry_rows = (int)pl.nkv_rows;
   ap.H = d.H; ap.P = kernel_P(d); ap.n_states = pl.n_local; ap.nq_rows = (int)pl.nq_rows;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = nullptr;  // phi_q comes finished from the workspace
@@ -1566,6 +1592,7 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   ap.L = L; ap.T = chunk_frames; ap.Tc = chunk_frames; ap.To = To;
   ap.frames_before = frames_before; ap.kv_frame0 = frames_before - pl.o;
   ap.H = d.H; ap.P = kernel_P(d); ap.n_states = 1; ap.nq_rows = pl.nq;
+  ap.kv_rows = ap.carry_rows = pl.nkv;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   ap.bq = bq; ap.Z = Z; ap.out = static_cast<__nv_bfloat16*>(out);
   RH_TRY(launch_attn_bf16<false>(mq, mk, mv, ms, mwq, mq, ap, dim3((pl.nq + 255) / 256, nbh, 1),
@@ -1573,6 +1600,7 @@ int rehyat_chunk_forward_static(rehyat_dims d, rehyat_dtype dt, int L, int frame
   if (pl.fold_rows > 0) {
     rehyat::state::FoldParams fp{};
     fp.L = L; fp.H = d.H; fp.P = kernel_P(d); fp.single_rows = pl.fold_rows; fp.n_fold = 1;
+    fp.kv_rows = fp.carry_rows = pl.nkv;
     fp.splits = splits; fp.G = d.G; fp.W = Wk; fp.bk = bk; fp.dS = dS; fp.dZ = dZ;
     RH_TRY(launch_fold_bf16(mk, mv, fp, dim3(splits, 1, nbh), st));
     rehyat::state::state_add_kernel<<<dim3((d.F * d.D + 255) / 256, nbh), 256, 0, st>>>(
@@ -1623,6 +1651,20 @@ int rehyat_selftest_wait_timeout(long long limit_ns, void* stream) {
   return cuda_check(cudaGetLastError(), "wait_timeout_selftest_kernel launch");
 }
 
+int rehyat_selftest_bounds(float* buf, long long n, long long bad_index, void* stream) {
+  g_msg[0] = 0;
+#ifndef REHYAT_DEBUG_BOUNDS
+  (void)buf, (void)n, (void)bad_index, (void)stream;
+  return fail(REHYAT_ERR_ARG, "not a debug-bounds build (compile with REHYAT_DEBUG_BOUNDS)");
+#else
+  if (!buf || n < 1 || n > (1LL << 30)) return fail(REHYAT_ERR_ARG, "need buf and 1 <= n <= 2^30");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned blocks = (unsigned)((n + 256) / 256);
+  bounds_selftest_kernel<<<blocks, 256, 0, st>>>(buf, n, bad_index);
+  return cuda_check(cudaGetLastError(), "bounds self-test launch");
+#endif
+}
+
 int rehyat_sync_status(void* stream) {
   g_msg[0] = 0;
   RH_TRY(cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "stream sync"));
@@ -1632,6 +1674,13 @@ int rehyat_sync_status(void* stream) {
   if (err) {
     const int zero = 0;
     cudaMemcpyToSymbol(rehyat::sm100::g_device_error, &zero, sizeof(int));
+    if (err == 2) {
+      long long info[3] = {0, 0, 0};
+      cudaMemcpyFromSymbol(info, rehyat::sm100::g_bounds_info, sizeof(info));
+      return fail(REHYAT_ERR_BOUNDS,
+                  "bounds check %lld failed: value %lld, limit %lld (access redirected or skipped)",
+                  info[0], info[1], info[2]);
+    }
     return fail(REHYAT_ERR_TIMEOUT, "a kernel wait timed out (device error %d)", err);
   }
   return REHYAT_OK;

@@ -26,8 +26,29 @@ namespace rehyat {
 namespace sm100 {
 
 // Device error word (one per library load; the library is built as one translation unit);
-// non-zero after a wait gave up.  Values: 1 = mbarrier wait timed out.
+// non-zero after a wait gave up or a bounds check failed.  Values: 1 = an mbarrier wait timed
+// out; 2 = a TMA coordinate or a global store index failed a bounds check of a debug-bounds
+// build (compiled with REHYAT_DEBUG_BOUNDS), and the access was redirected or skipped.
+// g_bounds_info holds the first failed check: {site, value, limit}.
 __device__ int g_device_error = 0;
+__device__ long long g_bounds_info[3];
+
+// In debug-bounds builds: true when lo <= value < hi, else the failure is recorded (the first
+// one's site, value and upper limit) and false is returned.  In other builds: true, no code.
+__device__ __forceinline__ bool bounds_ok(int site, long long value, long long lo, long long hi) {
+#ifdef REHYAT_DEBUG_BOUNDS
+  if (value >= lo && value < hi) return true;
+  if (atomicCAS(&g_device_error, 0, 2) == 0) {
+    g_bounds_info[0] = site;
+    g_bounds_info[1] = value;
+    g_bounds_info[2] = hi;
+  }
+  return false;
+#else
+  (void)site, (void)value, (void)lo, (void)hi;
+  return true;
+#endif
+}
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
@@ -128,6 +149,26 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// tma_load_3d of a bf16 tensor map with extents (ext0 inner elements, ext1 rows, ext2 depth) and
+// boxes of box1 rows; in debug-bounds builds its coordinates are checked first: the inner
+// coordinate a multiple of 8 elements (16 bytes) inside the row, the first row no more than one
+// box before the tensor and inside it (rows past either end read zeros, a start further out is
+// a wrong index), the depth inside the tensor.  A failed check is recorded and the copy goes to
+// (0, 0, 0) instead, so that its barrier still completes.
+__device__ __forceinline__ void tma_load_3d_chk(int site, void* dst, const CUtensorMap* map,
+                                                uint64_t* bar, int c0, int c1, int c2,
+                                                long long ext0, long long ext1, long long ext2,
+                                                int box1 = 128) {
+#ifdef REHYAT_DEBUG_BOUNDS
+  const bool ok = bounds_ok(site, c0 & 7, 0, 1) & bounds_ok(site, c0, 0, ext0) &
+                  bounds_ok(site, c1, -box1, ext1) & bounds_ok(site, c2, 0, ext2);
+  if (!ok) c0 = c1 = c2 = 0;
+#else
+  (void)site, (void)ext0, (void)ext1, (void)ext2, (void)box1;
+#endif
+  tma_load_3d(dst, map, bar, c0, c1, c2);
 }
 
 // Make generic-proxy shared-memory writes visible to the async proxy (tensor core reads).

@@ -66,6 +66,7 @@ struct FoldParams {
   // row seg_row0, the remaining single_rows - seg_rows from tmK/tmV at row 0; each segment is
   // tiled on its own.  seg_rows = 0: one segment.
   int seg_rows, seg_row0;
+  int kv_rows, carry_rows;  // rows per (b, h) of the main and of the carried K/V tensor maps
   int n_fold, splits;
   int G;
   const float* W;   // [H, G, F/G, D/G] fp32 weights of phi_k
@@ -200,8 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) {
         uint8_t* dk = sm + Lay::kOffK + sk * kTileBytes;
         mbar_arrive_expect_tx(&bars[kKFull + sk], kTileBytes);
-        tma_load_3d(dk, mK, &bars[kKFull + sk], 0, row, bh);
-        tma_load_3d(dk + kTok * 128, mK, &bars[kKFull + sk], 64, row, bh);
+        const int kv_ext = carried ? p.carry_rows : p.kv_rows;
+        tma_load_3d_chk(11, dk, mK, &bars[kKFull + sk], 0, row, bh, kHD, kv_ext, gridDim.z);
+        tma_load_3d_chk(11, dk + kTok * 128, mK, &bars[kKFull + sk], 64, row, bh, kHD, kv_ext,
+                        gridDim.z);
       }
       __syncwarp();
       ++issued_k;
@@ -210,8 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) {
         uint8_t* dv = sm + Lay::kOffV + s * kTileBytes;
         mbar_arrive_expect_tx(&bars[kVFull + s], kTileBytes);
-        tma_load_3d(dv, mV, &bars[kVFull + s], 0, row, bh);
-        tma_load_3d(dv + kTok * 128, mV, &bars[kVFull + s], 64, row, bh);
+        const int kv_ext = carried ? p.carry_rows : p.kv_rows;
+        tma_load_3d_chk(12, dv, mV, &bars[kVFull + s], 0, row, bh, kHD, kv_ext, gridDim.z);
+        tma_load_3d_chk(12, dv + kTok * 128, mV, &bars[kVFull + s], 64, row, bh, kHD, kv_ext,
+                        gridDim.z);
       }
       __syncwarp();
       ++issued_v;
@@ -326,6 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars[kPhiFull + s]);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0, abort_flag));
+    // the partial slot (grid (splits, n_fold, BH)) lies inside dS / dZ
+    if (ok && !bounds_ok(13, ((long long)bh * p.n_fold + fc) * p.splits + split, 0,
+                         (long long)gridDim.z * p.n_fold * p.splits))
+      ok = false;
     if (ok) {
       tc_fence_after();
       // lane r of TMEM is feature f = r: dS row f (this thread writes columns col0 .. col0+31),

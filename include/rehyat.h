@@ -61,7 +61,10 @@ typedef enum {
   REHYAT_ERR_WORKSPACE = -4, /* workspace NULL or smaller than the *_workspace_size query */
   REHYAT_ERR_CUDA = -5,      /* a CUDA runtime call or a launch failed */
   REHYAT_ERR_TIMEOUT = -6,   /* a kernel's bounded wait gave up (from rehyat_sync_status) */
-  REHYAT_ERR_ALIGN = -7      /* a pointer is not 16-byte aligned */
+  REHYAT_ERR_ALIGN = -7,     /* a pointer is not 16-byte aligned */
+  REHYAT_ERR_BOUNDS = -8     /* debug-bounds builds: a TMA coordinate or store index was out of
+                                range (from rehyat_sync_status); the access was redirected to a
+                                legal coordinate or skipped, so results are not to be trusted */
 } rehyat_status;
 
 typedef enum { REHYAT_F32 = 0, REHYAT_BF16 = 1 } rehyat_dtype;
@@ -87,6 +90,16 @@ const char* rehyat_last_error(void);
 
 /* ABI version of this library (major*100 + minor). */
 int rehyat_version(void);
+
+/* 1 if this library was built with REHYAT_DEBUG_BOUNDS (the package build's debug-bounds
+ * variant, librehyat_debug.so), else 0.  Such a build checks, before every TMA tile load of the
+ * forward kernels (attention, fold, phi_q), that the coordinates lie in the tensor (inner
+ * coordinate a multiple of 16 bytes inside the row, first row no more than one box outside,
+ * depth inside), and before every global store of those kernels (outputs, partial sums, lone-tile
+ * parts) that the index lies in its buffer.  A failed check does not trap: it records the first
+ * failure (site, value, limit) in the device error word, redirects the copy to coordinate
+ * (0, 0, 0) or skips the store, and rehyat_sync_status() returns REHYAT_ERR_BOUNDS. */
+int rehyat_debug_bounds(void);
 
 /* Feature map phi of the "ReHyAt overview" page §2.2.2, standalone.
  *   x    [B,H,n_tokens,D] (dtype), W [H,G,F/G,D/G] fp32, bias [H,F] fp32 or NULL,
@@ -300,9 +313,18 @@ int rehyat_segment_attend(rehyat_dims d, rehyat_dtype dt, int T, int frame_token
  * REHYAT_ERR_ARG for a limit out of range, REHYAT_ERR_CUDA if the launch fails. */
 int rehyat_selftest_wait_timeout(long long limit_ns, void* stream);
 
+/* Exercises the bounds checks of a debug-bounds build: a kernel writes 1.0 to buf[0, n) and then
+ * attempts buf[bad_index] through a store check against [0, n).  With bad_index outside [0, n)
+ * the check records the failure and skips the store, and the next rehyat_sync_status() returns
+ * REHYAT_ERR_BOUNDS.  buf [n + slack] fp32 device memory: give room past n for bad_index, so the
+ * write stays inside the buffer even if the check were absent.  Returns REHYAT_ERR_ARG in a
+ * build without the checks (rehyat_debug_bounds() == 0) or for n outside [1, 2^30]. */
+int rehyat_selftest_bounds(float* buf, long long n, long long bad_index, void* stream);
+
 /* Synchronise `stream` and report device-side failures of earlier calls: REHYAT_ERR_TIMEOUT if
- * a kernel's bounded wait gave up (the error word is then cleared), REHYAT_ERR_CUDA if the
- * stream reports a CUDA error, else REHYAT_OK. */
+ * a kernel's bounded wait gave up, REHYAT_ERR_BOUNDS if a bounds check of a debug-bounds build
+ * failed (the error word is then cleared), REHYAT_ERR_CUDA if the stream reports a CUDA error,
+ * else REHYAT_OK. */
 int rehyat_sync_status(void* stream);
 
 #ifdef __cplusplus

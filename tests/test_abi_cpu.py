@@ -32,7 +32,7 @@ def test_header_declares_the_binding_surface():
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.rehyat_version() == 101
+    assert lib.rehyat_version() == 102
 
 
 FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced: checks come first
@@ -104,7 +104,7 @@ def test_selftest_rejects_limits_out_of_range(lib):
 
 
 def test_abi_version_and_dims_layout(lib):
-    assert lib.rehyat_version() == 101
+    assert lib.rehyat_version() == 102
     assert ctypes.sizeof(rb.Dims) == 7 * 4
     # the elu + 1 kind passes validation (workspace queries need no device)
     n = ctypes.c_size_t(0)
@@ -188,3 +188,11 @@ def test_static_chunk_refuses_problems_beyond_its_scratch(lib):
     for B, H in [(14, 12), (1, 200), (170, 1)]:
         assert call(B, H) == -4, (B, H)
         assert "scratch" in lib.rehyat_last_error().decode()
+
+
+def test_release_build_has_no_bounds_checks(lib):
+    """The default library is built without the debug-bounds checks; its self test says so
+    instead of launching anything."""
+    assert lib.rehyat_debug_bounds() == 0
+    assert lib.rehyat_selftest_bounds(FAKE, 16, 20, None) == -1
+    assert "debug-bounds" in lib.rehyat_last_error().decode()

@@ -1,12 +1,19 @@
 """The backward pass (and the forward's row statistics it needs) on the GPU against the float64
 oracle of the gradients, on seeded inputs.
 
-Tolerance: the GPU path rounds P, dS, phi and du to bf16 as tensor-core operands (relative 2^-9
-= 2e-3 each) and accumulates in fp32; each gradient is a sum of many such terms, so its relative
-L2 error is of the order of one bf16 rounding.  Measured on the cases below: dq, dk, dv 1.3e-3 to
-2.1e-3 (bound REL_L2 = 1e-2); dW and db, sums over every token in which terms of both signs
-cancel, 2.5e-3 to 8.6e-3 (bound REL_L2_W = 2.5e-2); lse (log2 units) within 2.5e-3 (bound
-1e-2)."""
+Tolerances, from the rounding the GPU path does.  Every tensor-core operand that is not an input
+is rounded to bf16 (relative error at most 2^-9 per element); products accumulate in fp32, whose
+rounding (2^-24 per add) is negligible next to it.  A gradient element is a sum of terms, and the
+rounding errors of different terms are independent, so its relative error is at most the
+per-term bound times the sum's cancellation ratio R = (norm of the terms) / (norm of their sum).
+* dq, dk, dv: a term passes through at most two bf16 roundings (P or dS as a GEMM operand, and
+  the bf16 output o inside D = dO . o), 2 * 2^-9 = 3.9e-3; REL_L2 = 1e-2 allows R up to 2.5.
+* dW, db: sums over every token of du x^T, du passing through three roundings (phi, the
+  dS / P upstream, du itself as the GEMM operand), 3 * 2^-9 = 5.9e-3; terms of both signs cancel
+  across tokens, and REL_L2_W = 2.5e-2 allows R up to 4.3.
+* lse (log2 units): the denominators are fp32 sums of fp32 exponentials plus phi_q . Z with
+  bf16 phi_q, within 2^-9 relative, i.e. 2.8e-3 in log2 units; bound 1e-2.
+Measured: dq, dk, dv 1.3e-3 to 2.1e-3; dW, db 2.5e-3 to 8.6e-3; lse within 2.5e-3."""
 import math
 
 import numpy as np
@@ -44,6 +51,8 @@ def rel_l2(a, b):
 
 CASES = [
     # T, fh, fw, Tc, To, P, G, B, H, bias, phi
+    (7, 30, 52, 3, 1, 2, 8, 1, 2, 0.0, "poly"),   # 1560-token frames of the 480x832 workload
+    (7, 30, 52, 3, 1, 2, 8, 1, 1, -30.0, "poly"),  # ... with the linear branch switched off
     (7, 8, 10, 3, 1, 2, 8, 1, 2, 0.1, "poly"),
     (8, 6, 12, 3, 1, 3, 8, 2, 1, 0.0, "poly"),    # ragged last chunk, B = 2
     (6, 8, 8, 2, 2, 2, 16, 1, 2, 0.2, "poly"),
@@ -86,8 +95,11 @@ def test_backward_matches_oracle(dev, case):
                 den = np.exp(lg).sum(axis=1) + pq[s * L:e * L] @ pk[:wf * L].sum(axis=0)
                 lse_want[s * L:e * L] = np.log2(den)
             errs[f"lse b{b} h{h} (abs)"] = float(np.abs(f64(lse[b, h]) - lse_want).max())
-        for name, wv in zip(("dWq", "dbq", "dWk", "dbk"), sums):
-            errs[f"{name} h{h}"] = rel_l2(f64(g[name][h]), wv)
+        # with bias -30 the feature maps are ~e^(u - 30): their gradients are checked where the
+        # linear branch carries weight, not here
+        if bias > -10:
+            for name, wv in zip(("dWq", "dbq", "dWk", "dbk"), sums):
+                errs[f"{name} h{h}"] = rel_l2(f64(g[name][h]), wv)
     msg = " ".join(f"{k}={v:.2e}" for k, v in errs.items())
     print(msg)
     for k, v in errs.items():
