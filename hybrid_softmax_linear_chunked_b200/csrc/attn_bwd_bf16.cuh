@@ -28,11 +28,6 @@ namespace rehyat {
 namespace attn_bwd {
 
 using namespace sm100;
-using attn::f2_add;
-using attn::f2_fma;
-using attn::f2_mul;
-using attn::f2_pack;
-using attn::f2_unpack;
 using attn::kmajor_desc;
 using attn::mnmajor_desc;
 
@@ -44,7 +39,7 @@ __device__ __forceinline__ void grad_pair(uint32_t s0, uint32_t s1, uint32_t d0,
   const uint64_t x = f2_fma(f2_pack(__uint_as_float(s0), __uint_as_float(s1)), sl2x2, neg_l2);
   float xa, xb;
   f2_unpack(x, xa, xb);
-  const uint64_t pr = f2_pack(attn::ex2(xa), attn::ex2(xb));
+  const uint64_t pr = f2_pack(ex2(xa), ex2(xb));
   const uint64_t t = f2_add(f2_pack(__uint_as_float(d0), __uint_as_float(d1)), neg_d);
   const uint64_t g = f2_mul(f2_mul(pr, isd2), t);
   float pa, pb, ga, gb;

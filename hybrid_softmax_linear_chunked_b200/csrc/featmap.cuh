@@ -62,35 +62,84 @@ __device__ __forceinline__ float softplus_fast(float u) {
   return fmaxf(u, 0.f) + l;
 }
 
+// log2(1 + y) = y r(y) for y in [0, 1], with r(y) = log2(1 + y) / y a quintic fitted for minimax
+// relative error on [0, 1] by iteratively reweighted least squares (softplus_poly_fit.py beside
+// this file): 8.6e-6 relative in fp32 Horner form, against the 2^-9 rounding of the bf16 result.
+constexpr float kL1pC0 = 1.44268286f;
+constexpr float kL1pC1 = -0.720426023f;
+constexpr float kL1pC2 = 0.469173372f;
+constexpr float kL1pC3 = -0.303034991f;
+constexpr float kL1pC4 = 0.146032020f;
+constexpr float kL1pC5 = -0.0344357193f;
+constexpr float kLog2e = 1.44269504f;
+constexpr float kLn2 = 0.693147181f;
+
+// softplus in log2 units for a pair of lanes: with t = u log2(e),
+//     softplus(u) = ln2 * s,   s = max(t, 0) + log2(1 + 2^-|t|),
+// 2^-|t| on the MUFU (one op per element) and log2(1 + y) by the quintic on the FMA pipe.
+__device__ __forceinline__ uint64_t softplus_log2_x2(uint64_t t2) {
+  using namespace sm100;
+  float ta, tb;
+  f2_unpack(t2, ta, tb);
+  const uint64_t y2 = f2_pack(ex2(-fabsf(ta)), ex2(-fabsf(tb)));
+  uint64_t r2 = f2_fma(f2_pack(kL1pC5, kL1pC5), y2, f2_pack(kL1pC4, kL1pC4));
+  r2 = f2_fma(r2, y2, f2_pack(kL1pC3, kL1pC3));
+  r2 = f2_fma(r2, y2, f2_pack(kL1pC2, kL1pC2));
+  r2 = f2_fma(r2, y2, f2_pack(kL1pC1, kL1pC1));
+  r2 = f2_fma(r2, y2, f2_pack(kL1pC0, kL1pC0));
+  return f2_fma(r2, y2, f2_pack(fmaxf(ta, 0.f), fmaxf(tb, 0.f)));
+}
+
 // phi of 16 consecutive features f0 .. f0+15 from their grouped-linear outputs u (fp32 bits):
 // softplus(u + bias)^p, with p the feature's part power (pw[], non-decreasing in f), times
 // `scale`, packed as 8 bf16 pairs.  Parts are contiguous, so a 16-feature chunk nearly always
-// has a single power: that case (a uniform branch) costs at most two multiplies per feature.
+// has a single power p: that case (a uniform branch) folds ln2^p and the scale into one factor,
+// phi = s^p * (ln2^p * scale), in paired instructions.
 __device__ __forceinline__ void phi16(const uint32_t* u, int f0, const float* bias,
                                       const uint8_t* pw, float scale, uint32_t* packed) {
-  float ph[16];
+  using namespace sm100;
   const int p_first = pw[f0], p_last = pw[f0 + 15];
   if (p_last == 0) {  // elu + 1 map (the whole table is 0)
+    float ph[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) ph[i] = elu1_fast(__uint_as_float(u[i]) + bias[f0 + i]);
 #pragma unroll
     for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(ph[2 * i] * scale, ph[2 * i + 1] * scale);
     return;
   }
+  const uint64_t l2e2 = f2_pack(kLog2e, kLog2e);
+  uint64_t s2[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) ph[i] = softplus_fast(__uint_as_float(u[i]) + bias[f0 + i]);
-  if (p_first == p_last) {
-    if (p_first == 2) {
+  for (int i = 0; i < 8; ++i) {
+    const float2 b = *reinterpret_cast<const float2*>(bias + f0 + 2 * i);
+    const uint64_t x2 = f2_add(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])),
+                               f2_pack(b.x, b.y));
+    s2[i] = softplus_log2_x2(f2_mul(x2, l2e2));
+  }
+  if (p_first == p_last && p_first <= 3) {
+    const float c = p_first == 1 ? kLn2 * scale
+                  : p_first == 2 ? (kLn2 * kLn2) * scale
+                                 : (kLn2 * kLn2 * kLn2) * scale;
+    const uint64_t c2 = f2_pack(c, c);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) ph[i] *= ph[i];
-    } else if (p_first == 3) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) ph[i] = ph[i] * ph[i] * ph[i];
-    } else if (p_first != 1) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) ph[i] = int_pow(ph[i], p_first);
+    for (int i = 0; i < 8; ++i) {
+      uint64_t v2 = s2[i];
+      if (p_first == 2) v2 = f2_mul(v2, v2);
+      if (p_first == 3) v2 = f2_mul(f2_mul(v2, v2), v2);
+      float a, b;
+      f2_unpack(f2_mul(v2, c2), a, b);
+      packed[i] = pack_bf16x2(a, b);
     }
-  } else if (p_last <= 4) {
+    return;
+  }
+  float ph[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f2_unpack(s2[i], ph[2 * i], ph[2 * i + 1]);
+    ph[2 * i] *= kLn2;
+    ph[2 * i + 1] *= kLn2;
+  }
+  if (p_last <= 4) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) ph[i] = pow_upto4(ph[i], pw[f0 + i]);
   } else {
