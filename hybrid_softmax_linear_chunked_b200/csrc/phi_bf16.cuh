@@ -3,7 +3,9 @@
 // + lo parts built in shared memory from the fp32 weights, fp32 in TMEM) by tcgen05, then bias,
 // softplus and the part powers on the CUDA cores, written as bf16 rows.  Used for phi_q of the
 // query rows that read a linear state, so that the attention kernel's epilogue only has to load
-// a finished phi_q tile.
+// a finished phi_q tile.  The output leaves by TMA stores from shared memory: the feature-map
+// warps write a tile's phi over the X stage that its MMA has consumed, the producer stores it
+// and refills the stage once the store has read it.
 #pragma once
 
 #include "featmap.cuh"
@@ -34,7 +36,9 @@ struct Layout {
   static constexpr int kCtasPerSm = kDense ? 1 : 2;
 };
 
-enum Bar { kXFull = 0, kXEmpty = 2, kUFull = 4, kUEmpty = 6, kDone = 8, kNumBars = 9 };
+// kOutFull: a tile's phi is in its X stage (256 arrivals); the stage is free again once the
+// producer's store of it has read it.
+enum Bar { kXFull = 0, kOutFull = 2, kUFull = 4, kUEmpty = 6, kDone = 8, kNumBars = 9 };
 
 struct Params {
   int row0;           // first row (of each (b, h) sequence) to map
@@ -44,7 +48,6 @@ struct Params {
   int H, P, G;
   const float* W;     // [H, G, F/G, D/G] fp32
   const float* bias;  // [H, F] or null
-  __nv_bfloat16* phi; // [BH, rows_per_bh, F]
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -52,10 +55,13 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // grid (ceil(n_tiles / tiles_per_cta), BH), block 320.  Feature-map thread tid owns row
-// (tid & 127) = TMEM lane and features [64 (tid >> 7), +64).
+// (tid & 127) = TMEM lane and features [64 (tid >> 7), +64).  tmX reads x [BH, rows_per_bh, D];
+// tmPhi writes phi [BH, rows_per_bh, F] with its row extent cut at row0 + n_rows, so that the
+// rows of a ragged last tile past the range are not written.
 template <bool kDense>
 __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
-    featmap_tc_kernel(const __grid_constant__ CUtensorMap tmX, const Params p) {
+    featmap_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                      const __grid_constant__ CUtensorMap tmPhi, const Params p) {
   using Lay = Layout<kDense>;
   static_assert(Lay::kSmemBytes + 256 <= 232448 / Lay::kCtasPerSm,
                 "shared memory (dynamic + static) over the limit");
@@ -84,7 +90,9 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
   }
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i)
-      mbar_init(&bars[i], (i == kUEmpty || i == kUEmpty + 1) ? kPhiThreads : 1);
+      mbar_init(&bars[i], (i == kUEmpty || i == kUEmpty + 1 || i == kOutFull || i == kOutFull + 1)
+                              ? kPhiThreads
+                              : 1);
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -102,15 +110,34 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
   const bool leader = lane == 0;
 
   if (warp == 8) {
-    // ---- producer ----
-    if (leader) tma_prefetch_desc(&tmX);
+    // ---- producer: loads of x, stores of phi ----
+    if (leader) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmPhi);
+    }
     __syncwarp();
     bool ok = true;
     int issued = 0;
+    const long long out_rows = (long long)p.row0 + p.n_rows;
+    // phi of tile j goes out from X stage j & 1; the stage is reusable once the store read it
+    auto store_tile = [&](int j) {
+      const int s = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOutFull + s], (j >> 1) & 1, abort_flag));
+      if (!ok) return;
+      if (leader) {
+        const uint8_t* src = sm + Lay::kOffX + s * kTileBytes;
+        const int row = p.row0 + (t_begin + j) * kRows;
+        tma_store_3d_chk(23, &tmPhi, src, 0, row, bh, kFD, out_rows, gridDim.y);
+        tma_store_3d_chk(23, &tmPhi, src + kRows * 128, 64, row, bh, kFD, out_rows, gridDim.y);
+        bulk_commit_group();
+        bulk_wait_read_all();
+      }
+      __syncwarp();
+    };
     for (int i = 0; i < n_tiles; ++i) {
       const int s = i & 1;
       const int row = p.row0 + (t_begin + i) * kRows;
-      if (i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kXEmpty + s], ((i >> 1) - 1) & 1, abort_flag));
+      if (i >= 2) store_tile(i - 2);
       if (!ok) break;
       if (leader) {
         uint8_t* dx = sm + Lay::kOffX + s * kTileBytes;
@@ -123,13 +150,16 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
       __syncwarp();
       ++issued;
     }
+    for (int j = max(0, n_tiles - 2); j < n_tiles && ok; ++j) store_tile(j);
+    if (leader) bulk_wait_all();  // the stores are complete before the CTA exits
     if (!ok) {
       for (int i = max(0, issued - 2); i < issued; ++i)
         mbar_wait_drain(&bars[kXFull + (i & 1)], (i >> 1) & 1);
     }
     __syncwarp();
   } else if (warp == 9) {
-    // ---- MMA issuer: U[s] = X_i Wbd_hi^T + X_i Wbd_lo^T, tile by tile of the compact W ----
+    // ---- MMA issuer: U[s] = X_i Wbd_hi^T + X_i Wbd_lo^T, tile by tile of the compact W (its
+    // completion also frees X stage s for the feature-map warps' phi) ----
     const CompactW cw = compact_w(kFD, kHD, p.G);
     const uint32_t id_u = idesc_bf16(kRows, cw.NT, false, false);
     const uint64_t dX0 = sdesc_sw128(smem_u32(sm + Lay::kOffX), 16, 1024);
@@ -159,7 +189,6 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
           }
         }
         mma_commit(&bars[kUFull + s]);
-        mma_commit(&bars[kXEmpty + s]);
       }
       __syncwarp();
     }
@@ -178,10 +207,9 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[kUFull + s], (i >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const int row_in = (t_begin + i) * kRows + r;  // row index inside [row0, row0 + n_rows)
-      const bool valid =
-          row_in < p.n_rows && bounds_ok(22, p.row0 + row_in, 0, p.rows_per_bh);
-      __nv_bfloat16* dst = p.phi + ((size_t)bh * p.rows_per_bh + p.row0 + row_in) * kFD + col0;
+      // the MMA that read X stage s is complete (U_FULL): phi of the tile goes over it, in the
+      // 128B-swizzled layout of the store's two 64-feature boxes
+      uint8_t* xs = sm + Lay::kOffX + s * kTileBytes;
 #pragma unroll 1
       for (int c16 = 0; c16 < 4; ++c16) {
         const int f0 = col0 + c16 * 16;
@@ -189,14 +217,15 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
         tmem_ld16(tmem + lane_base + s * 128 + f0, uu);
         uint32_t packed[8];
         phi16(uu, f0, sB, sPw, 1.f, packed);
-        if (valid) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c16 * 16);
-          d4[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          d4[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-        }
+        *reinterpret_cast<uint4*>(xs + sw128_offset(r, f0, kRows)) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        *reinterpret_cast<uint4*>(xs + sw128_offset(r, f0 + 8, kRows)) =
+            make_uint4(packed[4], packed[5], packed[6], packed[7]);
       }
       tc_fence_before();
       mbar_arrive(&bars[kUEmpty + s]);
+      fence_async_smem();
+      mbar_arrive(&bars[kOutFull + s]);
     }
   }
   tc_fence_before();

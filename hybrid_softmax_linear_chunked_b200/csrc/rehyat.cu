@@ -477,8 +477,8 @@ int launch_lone_combine(const rehyat::attn::Params& ap, int BH, int n_chunks, cu
 // phi ([BH][rows_per_bh][F] bf16) on the tensor cores; W are the fp32 weights [H][G][F/G][D/G]
 // (each CTA builds its head's compact block-diagonal matrix in shared memory).
 template <bool kDense>
-int launch_featmap_tc_inst(const rehyat_dims& d, const CUtensorMap& mx, int n_rows,
-                           rehyat::phi::Params pp, cudaStream_t st) {
+int launch_featmap_tc_inst(const rehyat_dims& d, const CUtensorMap& mx, const CUtensorMap& mphi,
+                           int n_rows, rehyat::phi::Params pp, cudaStream_t st) {
   using Lay = rehyat::phi::Layout<kDense>;
   const int BH = d.B * d.H;
   const int n_tiles = (n_rows + 127) / 128;
@@ -494,22 +494,27 @@ int launch_featmap_tc_inst(const rehyat_dims& d, const CUtensorMap& mx, int n_ro
                                          (int)Lay::kSmemBytes),
                     "featmap_tc attr"));
   k<<<dim3((n_tiles + per_cta - 1) / per_cta, BH), rehyat::phi::kThreads, Lay::kSmemBytes, st>>>(
-      mx, pp);
+      mx, mphi, pp);
   return cuda_check(cudaGetLastError(), "featmap_tc launch");
 }
 
 int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int row0, int n_rows,
                       const float* W, const float* bias, __nv_bfloat16* phi, cudaStream_t st) {
   if (n_rows <= 0) return REHYAT_OK;
-  CUtensorMap mx;
-  RH_TRY(make_map(&mx, x, d.D, rows_per_bh, (long long)d.B * d.H));
+  const long long BH = (long long)d.B * d.H;
+  CUtensorMap mx, mphi;
+  RH_TRY(make_map(&mx, x, d.D, rows_per_bh, BH));
+  // phi rows [row0, row0 + n_rows) of each (b, h): the map's row extent ends there, so a ragged
+  // last tile's store writes nothing past the range
+  RH_TRY(make_map_strided(&mphi, phi, d.F, (long long)row0 + n_rows, BH, d.F,
+                          (long long)rows_per_bh * d.F, 64, 128));
   rehyat::phi::Params pp{};
   pp.row0 = row0; pp.n_rows = n_rows; pp.rows_per_bh = rows_per_bh;
-  pp.H = d.H; pp.P = kernel_P(d); pp.G = d.G; pp.W = W; pp.bias = bias; pp.phi = phi;
+  pp.H = d.H; pp.P = kernel_P(d); pp.G = d.G; pp.W = W; pp.bias = bias;
   // the G = 1 matrix is dense (32 KB per part): its instance runs one CTA per SM
   if (rehyat::compact_w(d.F, d.D, d.G).NT > 64)
-    return launch_featmap_tc_inst<true>(d, mx, n_rows, pp, st);
-  return launch_featmap_tc_inst<false>(d, mx, n_rows, pp, st);
+    return launch_featmap_tc_inst<true>(d, mx, mphi, n_rows, pp, st);
+  return launch_featmap_tc_inst<false>(d, mx, mphi, n_rows, pp, st);
 }
 
 // behind_attention: launch with programmatic stream serialization right after an attention

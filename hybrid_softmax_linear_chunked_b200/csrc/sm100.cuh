@@ -171,6 +171,44 @@ __device__ __forceinline__ void tma_load_3d_chk(int site, void* dst, const CUten
   tma_load_3d(dst, map, bar, c0, c1, c2);
 }
 
+// TMA tile store of one 3-D box from shared memory (128B-swizzled like the loads) into the
+// tensor; the parts of the box past the tensor's extents are not written.  Completion is tracked
+// by this thread's bulk async-groups (bulk_commit_group, then bulk_wait_read_all /
+// bulk_wait_all).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0,
+                                             int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// tma_store_3d with, in debug-bounds builds, the inner coordinate a multiple of 8 elements inside
+// the row and the row and depth coordinates inside the tensor (a store never starts before it);
+// a failed check is recorded and the store skipped.
+__device__ __forceinline__ void tma_store_3d_chk(int site, const CUtensorMap* map, const void* src,
+                                                 int c0, int c1, int c2, long long ext0,
+                                                 long long ext1, long long ext2) {
+#ifdef REHYAT_DEBUG_BOUNDS
+  const bool ok = bounds_ok(site, c0 & 7, 0, 1) & bounds_ok(site, c0, 0, ext0) &
+                  bounds_ok(site, c1, 0, ext1) & bounds_ok(site, c2, 0, ext2);
+  if (!ok) return;
+#else
+  (void)site, (void)ext0, (void)ext1, (void)ext2;
+#endif
+  tma_store_3d(map, src, c0, c1, c2);
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Every committed bulk group of this thread has finished reading its shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Every committed bulk group of this thread is complete.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // Make generic-proxy shared-memory writes visible to the async proxy (tensor core reads).
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
