@@ -16,7 +16,8 @@
 // part powers) and writes it as bf16 over its Q tile in shared memory; one more MMA adds
 // phi_q 2^-m . S_c into O_t, and l_t += 2^-m phi_q . Z_c; the output is O_t / l_t.  m starts at
 // 0 for chunks that have a linear region, so 2^-m <= 1 and a row can never lose both terms to
-// underflow.
+// underflow.  A tile whose 128 rows all lie in the chunk is packed as bf16 into its Q tile's
+// shared memory and leaves by two TMA stores; a ragged tile's rows are stored one by one.
 //
 // Warp roles (320 threads): warps 0-3 softmax/epilogue of tile 0, warps 4-7 of tile 1, warp 8
 // TMA producer (+ TMEM allocation), warp 9 MMA issuer.  TMEM columns: S_0 [0,128), S_1
@@ -149,7 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tmW,
                             const __grid_constant__ CUtensorMap tmPhi,
                             const __grid_constant__ CUtensorMap tmKc,
-                            const __grid_constant__ CUtensorMap tmVc, const Params p) {
+                            const __grid_constant__ CUtensorMap tmVc,
+                            const __grid_constant__ CUtensorMap tmOut, const Params p) {
   static_assert(kSmemBytes + 256 <= 232448, "shared memory (dynamic + static) over the limit");
 
   // ---- chunk geometry (uniform over the CTA) ----
@@ -468,6 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_base + t * 128;
     const uint32_t tO = tmem + lane_base + 256 + t * 128;
     const bool active = (t == 0) || has_t1;
+    // a whole-window CTA's tile whose 128 rows all lie in the chunk is stored by TMA
+    const bool full_tile = part < 0 && tile_row0 + t * kBM + kBM <= nq;
     if (active) {
       const float sl2 = p.scale_log2;
       float m = has_linear ? 0.f : -INFINITY;
@@ -659,12 +663,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv = 1.f / l;
         if (p.lse && row_valid)
           p.lse[(size_t)bh * p.nq_rows + q_row0 + row_in_chunk] = m + log2f(l);
-        __nv_bfloat16* orow = p.out + ((size_t)bh * p.nq_rows + q_row0 + row_in_chunk) * kHD;
+        if (full_tile) {
+          // A full tile leaves by two TMA stores from its Q tile's shared memory, which no MMA
+          // reads any more (its readout, or without one its last S, is complete): rows packed in
+          // the 128B-swizzled layout of the store's two 64-column boxes (stored below).
+          uint8_t* ostage = sm + (t ? kOffQ1 : kOffQ0);
 #pragma unroll
-        for (int cc = 0; cc < kHD / 32; ++cc) {
-          uint32_t rr[32];
-          tmem_ld32(tO + cc * 32, rr);
-          if (row_valid) {
+          for (int cc = 0; cc < kHD / 32; ++cc) {
+            uint32_t rr[32];
+            tmem_ld32(tO + cc * 32, rr);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               uint4 o4;
@@ -672,9 +679,41 @@ __global__ void __launch_bounds__(kThreads, 1)
               o4.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
               o4.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
               o4.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
-              *reinterpret_cast<uint4*>(orow + cc * 32 + q4 * 8) = o4;
+              *reinterpret_cast<uint4*>(ostage + sw128_offset(r, cc * 32 + q4 * 8, kBM)) = o4;
             }
           }
+        } else {
+          __nv_bfloat16* orow = p.out + ((size_t)bh * p.nq_rows + q_row0 + row_in_chunk) * kHD;
+#pragma unroll
+          for (int cc = 0; cc < kHD / 32; ++cc) {
+            uint32_t rr[32];
+            tmem_ld32(tO + cc * 32, rr);
+            if (row_valid) {
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 o4;
+                o4.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
+                o4.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
+                o4.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
+                o4.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
+                *reinterpret_cast<uint4*>(orow + cc * 32 + q4 * 8) = o4;
+              }
+            }
+          }
+        }
+      }
+      if (full_tile) {
+        // every thread of the tile gets here, whatever its waits returned (a named barrier has
+        // no time limit); after an abort the store is skipped
+        fence_async_smem();
+        named_bar_sync(1 + t, kBM);
+        if (r == 0 && !*abort_flag) {
+          uint8_t* ostage = sm + (t ? kOffQ1 : kOffQ0);
+          const int row = q_row0 + tile_row0 + t * kBM;
+          tma_store_3d_chk(32, &tmOut, ostage, 0, row, bh, kHD, p.nq_rows, n_bh);
+          tma_store_3d_chk(32, &tmOut, ostage + kBM * 128, 64, row, bh, kHD, p.nq_rows, n_bh);
+          bulk_commit_group();
+          bulk_wait_all();  // complete before the CTA exits
         }
       }
     }

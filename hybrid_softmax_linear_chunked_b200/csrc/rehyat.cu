@@ -463,7 +463,10 @@ int launch_attn_bf16(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   cfg.attrs = attr;
   cfg.numAttrs = (kPhiGlobal && behind_phiq) ? 1 : 0;
   const CUtensorMap kc = mkc ? *mkc : mk, vc = mvc ? *mvc : mv;
-  return cuda_check(cudaLaunchKernelEx(&cfg, k, mq, mk, mv, ms, mw, mphi, kc, vc, ap),
+  // the output [grid.y (b, h)][nq_rows][D] for the full query tiles' TMA stores
+  CUtensorMap mo;
+  RH_TRY(make_map(&mo, ap.out, rehyat::attn::kHD, ap.nq_rows, grid.y));
+  return cuda_check(cudaLaunchKernelEx(&cfg, k, mq, mk, mv, ms, mw, mphi, kc, vc, mo, ap),
                     "attention launch");
 }
 
