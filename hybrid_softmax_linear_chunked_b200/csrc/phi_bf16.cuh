@@ -66,13 +66,17 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
   static_assert(Lay::kSmemBytes + 256 <= 232448 / Lay::kCtasPerSm,
                 "shared memory (dynamic + static) over the limit");
   // the attention launched behind this kernel may start at once: it reads phi_q only after
-  // waiting for this grid
+  // waiting for this grid.  Launched itself behind the library's state scan, this kernel waits for
+  // that grid before it exits, so that its completion implies the scan's.
   grid_dep_signal();
   const int bh = blockIdx.y, h = bh % p.H;
   const int n_tiles_all = (p.n_rows + kRows - 1) / kRows;
   const int t_begin = blockIdx.x * p.tiles_per_cta;
   const int n_tiles = min(p.tiles_per_cta, n_tiles_all - t_begin);
-  if (n_tiles <= 0) return;
+  if (n_tiles <= 0) {
+    grid_dep_wait();
+    return;
+  }
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -234,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, Layout<kDense>::kCtasPerSm)
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
+  grid_dep_wait();
 }
 
 }  // namespace phi

@@ -481,7 +481,7 @@ int launch_lone_combine(const rehyat::attn::Params& ap, int BH, int n_chunks, cu
 // (each CTA builds its head's compact block-diagonal matrix in shared memory).
 template <bool kDense>
 int launch_featmap_tc_inst(const rehyat_dims& d, const CUtensorMap& mx, const CUtensorMap& mphi,
-                           int n_rows, rehyat::phi::Params pp, cudaStream_t st) {
+                           int n_rows, rehyat::phi::Params pp, cudaStream_t st, bool behind_scan) {
   using Lay = rehyat::phi::Layout<kDense>;
   const int BH = d.B * d.H;
   const int n_tiles = (n_rows + 127) / 128;
@@ -496,13 +496,25 @@ int launch_featmap_tc_inst(const rehyat_dims& d, const CUtensorMap& mx, const CU
   RH_TRY(cuda_check(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lay::kSmemBytes),
                     "featmap_tc attr"));
-  k<<<dim3((n_tiles + per_cta - 1) / per_cta, BH), rehyat::phi::kThreads, Lay::kSmemBytes, st>>>(
-      mx, mphi, pp);
-  return cuda_check(cudaGetLastError(), "featmap_tc launch");
+  // behind_scan: the launch before this one, in the same call, is the library's state scan, whose
+  // outputs this kernel does not read: launched with programmatic stream serialization, it starts
+  // at once and waits for the scan's grid before it exits.
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((n_tiles + per_cta - 1) / per_cta, BH);
+  cfg.blockDim = dim3(rehyat::phi::kThreads);
+  cfg.dynamicSmemBytes = Lay::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = behind_scan ? 1 : 0;
+  return cuda_check(cudaLaunchKernelEx(&cfg, k, mx, mphi, pp), "featmap_tc launch");
 }
 
 int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int row0, int n_rows,
-                      const float* W, const float* bias, __nv_bfloat16* phi, cudaStream_t st) {
+                      const float* W, const float* bias, __nv_bfloat16* phi, cudaStream_t st,
+                      bool behind_scan = false) {
   if (n_rows <= 0) return REHYAT_OK;
   const long long BH = (long long)d.B * d.H;
   CUtensorMap mx, mphi;
@@ -516,8 +528,8 @@ int launch_featmap_tc(const rehyat_dims& d, const void* x, int rows_per_bh, int 
   pp.H = d.H; pp.P = kernel_P(d); pp.G = d.G; pp.W = W; pp.bias = bias;
   // the G = 1 matrix is dense (32 KB per part): its instance runs one CTA per SM
   if (rehyat::compact_w(d.F, d.D, d.G).NT > 64)
-    return launch_featmap_tc_inst<true>(d, mx, mphi, n_rows, pp, st);
-  return launch_featmap_tc_inst<false>(d, mx, mphi, n_rows, pp, st);
+    return launch_featmap_tc_inst<true>(d, mx, mphi, n_rows, pp, st, behind_scan);
+  return launch_featmap_tc_inst<false>(d, mx, mphi, n_rows, pp, st, behind_scan);
 }
 
 // behind_attention: launch with programmatic stream serialization right after an attention
@@ -842,9 +854,21 @@ int rehyat_forward_states(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, 
                             reinterpret_cast<float*>(ws + pl.Zc), st);
 }
 
+// behind_scan: the caller enqueued rehyat_forward_states right before (the phi_q kernel then
+// starts under the state scan, which it does not read).
+static int forward_phiq_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                             const void* q, const float* Wq, const float* bq, void* workspace,
+                             size_t ws_bytes, void* stream, bool behind_scan);
+
 int rehyat_forward_phiq(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
                         const void* q, const float* Wq, const float* bq, void* workspace,
                         size_t ws_bytes, void* stream) {
+  return forward_phiq_impl(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream, false);
+}
+
+static int forward_phiq_impl(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
+                             const void* q, const float* Wq, const float* bq, void* workspace,
+                             size_t ws_bytes, void* stream, bool behind_scan) {
   g_msg[0] = 0;
   ForwardPlan pl;
   RH_TRY(forward_common_checks(d, dt, T, L, Tc, To, workspace, ws_bytes, &pl));
@@ -858,7 +882,8 @@ int rehyat_forward_phiq(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, in
     const long long row_lin = (long long)(To / Tc + 1) * Tc * L;
     if (row_lin < N)
       RH_TRY(launch_featmap_tc(d, q, (int)N, (int)row_lin, (int)(N - row_lin), Wq, bq,
-                               reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16), st));
+                               reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16), st,
+                               behind_scan));
     return REHYAT_OK;
   }
   return launch_featmap(d, REHYAT_F32, (int)N, q, Wq, bq, ws + pl.phiq, st);
@@ -944,7 +969,7 @@ int rehyat_forward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To,
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(REHYAT_ERR_ALIGN, "q/k/v/out not 16-byte aligned");
   RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, workspace, ws_bytes, stream));
-  RH_TRY(rehyat_forward_phiq(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream));
+  RH_TRY(forward_phiq_impl(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream, true));
   return forward_attend_impl(d, dt, T, L, Tc, To, q, k, v, out, nullptr, workspace, ws_bytes,
                              stream, true);
 }
@@ -961,7 +986,7 @@ int rehyat_forward_train(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, i
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(REHYAT_ERR_ALIGN, "q/k/v/out not 16-byte aligned");
   RH_TRY(rehyat_forward_states(d, dt, T, L, Tc, To, k, v, Wk, bk, workspace, ws_bytes, stream));
-  RH_TRY(rehyat_forward_phiq(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream));
+  RH_TRY(forward_phiq_impl(d, dt, T, L, Tc, To, q, Wq, bq, workspace, ws_bytes, stream, true));
   return forward_attend_impl(d, dt, T, L, Tc, To, q, k, v, out, lse, workspace, ws_bytes, stream,
                              true);
 }
@@ -1193,8 +1218,8 @@ static int chunk_step_bf16(const rehyat_dims& d, int L, int frames_before, int c
   RH_TRY(make_map(&ms, St, d.F, d.D, BH));
   __nv_bfloat16* phiq = reinterpret_cast<__nv_bfloat16*>(ws + pl.phiq_bf16);
   // phi_q right before the attention, which overlaps it
-  if (frames_before - pl.o > 0)  // the chunk reads a linear state
-    RH_TRY(launch_featmap_tc(d, q, pl.nq, 0, pl.nq, Wq, bq, phiq, st));
+  if (frames_before - pl.o > 0)  // the chunk reads a linear state; it starts under the S^T copy
+    RH_TRY(launch_featmap_tc(d, q, pl.nq, 0, pl.nq, Wq, bq, phiq, st, true));
   CUtensorMap mphi;
   RH_TRY(make_map(&mphi, phiq, d.F, pl.nq, BH));
   rehyat::attn::Params ap{};

@@ -373,6 +373,9 @@ __global__ void __launch_bounds__(256) state_scan_kernel(
     int F, int D, const float* __restrict__ S0, const float* __restrict__ Z0, int n_prefix,
     __nv_bfloat16* __restrict__ St, float* __restrict__ Zc, float* __restrict__ S_out,
     float* __restrict__ Z_out) {
+  // a phi_q kernel launched behind this one (it reads none of this kernel's outputs) may start
+  // at once; it waits for this grid before it exits
+  grid_dep_signal();
   __shared__ float tile[32][33];
   const int bh = blockIdx.y;
   const int tiles_d = D / 32;
