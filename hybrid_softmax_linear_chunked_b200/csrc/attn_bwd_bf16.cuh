@@ -89,17 +89,56 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
   tma_load_3d(dst + 128 * 128, map, bar, 64, row, bh);
 }
 
-// Adds 32 fp32 values (TMEM words) to a row of a fp32 [..][128] tensor.
-__device__ __forceinline__ void add_row32(float* dst, const uint32_t* r) {
-  float4* d4 = reinterpret_cast<float4*>(dst);
+// Load 32 consecutive columns at each of two TMEM addresses with one wait.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t (&a)[32], uint32_t tb,
+                                            uint32_t (&b)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, "
+      "%41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, "
+      "%58, %59, %60, %61, %62, %63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : REHYAT_R32(a, 0), REHYAT_R32(b, 0)
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+// TMA tile reduce-add of one 3-D box of fp32 from shared memory (128B-swizzled) into the tensor:
+// every element is added to global memory; the parts of the box past the tensor's extents are
+// not touched.  Tracked by this thread's bulk async-groups like tma_store_3d.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int c0,
+                                                  int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// tma_reduce_add_3d of an fp32 tensor with, in debug-bounds builds, the inner coordinate a
+// multiple of 4 elements (16 bytes) inside the row and the row and depth coordinates inside the
+// tensor; a failed check is recorded and the reduction skipped.
+__device__ __forceinline__ void tma_reduce_add_3d_chk(int site, const CUtensorMap* map,
+                                                      const void* src, int c0, int c1, int c2,
+                                                      long long ext0, long long ext1,
+                                                      long long ext2) {
+#ifdef REHYAT_DEBUG_BOUNDS
+  const bool ok = bounds_ok(site, c0 & 3, 0, 1) & bounds_ok(site, c0, 0, ext0) &
+                  bounds_ok(site, c1, 0, ext1) & bounds_ok(site, c2, 0, ext2);
+  if (!ok) return;
+#else
+  (void)site, (void)ext0, (void)ext1, (void)ext2;
+#endif
+  tma_reduce_add_3d(map, src, c0, c1, c2);
+}
+// Writes 32 fp32 values (TMEM words; zeros when !keep) as row r of a [128 rows][32 fp32] box in the
+// 128B-swizzled layout of an fp32 TMA tile (16-byte chunk j of the row at position j ^ (r % 8)).
+__device__ __forceinline__ void stage_row32(uint8_t* box, int r, const uint32_t* v, bool keep) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float4 o = d4[i];
-    o.x += __uint_as_float(r[4 * i]);
-    o.y += __uint_as_float(r[4 * i + 1]);
-    o.z += __uint_as_float(r[4 * i + 2]);
-    o.w += __uint_as_float(r[4 * i + 3]);
-    d4[i] = o;
+  for (int j = 0; j < 8; ++j) {
+    const float4 x = keep ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                        __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(box + r * 128 + ((j ^ (r & 7)) * 16)) = x;
   }
 }
 
@@ -117,6 +156,7 @@ enum KBar { kKvFull = 0, kQFull = 1, kQEmpty = 3, kSdFull = 5, kPdFull = 6, kKDo
 __global__ void __launch_bounds__(kThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                 const Params p) {
   static_assert(kKSmem + 256 <= 232448, "shared memory over the limit");
   const Geometry g = geometry(p);
@@ -248,8 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cc = 0; cc < 2; ++cc) {
         const int c = hc * 2 + cc;  // 32-column chunk of the scores
         uint32_t sv[32], dv[32];
-        tmem_ld32(tS + c * 32, sv);
-        tmem_ld32(tD + c * 32, dv);
+        tmem_ld32x2(tS + c * 32, sv, tD + c * 32, dv);
         uint32_t pp[16], gg[16];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
@@ -269,21 +308,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars[kPdFull]);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kKDone], 0, abort_flag)) && !*abort_flag;
+    // dV and dK are added into global memory by TMA reduce-adds of four 32-column fp32 boxes
+    // each, staged in the Q and dO stages (free: every MMA is complete); rows past the window add
+    // zeros.
     if (ok) {
       tc_fence_after();
       const bool row_ok = key0 + r < g.nw;
-      const long long row = (long long)bh * p.N + g.k_row0 + key0 + r;
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
         const int cc = hc * 2 + c2;
         uint32_t a[32], b[32];
-        tmem_ld32(tmem + lane_base + 256 + cc * 32, a);
-        tmem_ld32(tmem + lane_base + 384 + cc * 32, b);
-        if (row_ok) {
-          add_row32(p.dv + row * 128 + cc * 32, a);
-          add_row32(p.dk + row * 128 + cc * 32, b);
-        }
+        tmem_ld32x2(tmem + lane_base + 256 + cc * 32, a, tmem + lane_base + 384 + cc * 32, b);
+        stage_row32(sm + kKOffQ + cc * 16384, r, a, row_ok);
+        stage_row32(sm + kKOffO + cc * 16384, r, b, row_ok);
       }
+    }
+    // every compute thread gets here, whatever its waits returned; after an abort nothing is added
+    fence_async_smem();
+    named_bar_sync(1, kCompute);
+    if (tid == 0 && !*abort_flag) {
+      const int row = g.k_row0 + key0;
+      for (int cc = 0; cc < 4; ++cc) {
+        tma_reduce_add_3d_chk(41, &tmDV, sm + kKOffQ + cc * 16384, cc * 32, row, bh, 128, p.N,
+                              gridDim.z);
+        tma_reduce_add_3d_chk(41, &tmDK, sm + kKOffO + cc * 16384, cc * 32, row, bh, 128, p.N,
+                              gridDim.z);
+      }
+      bulk_commit_group();
+      bulk_wait_all();
     }
   }
   tc_fence_before();
@@ -307,7 +359,7 @@ enum QBar { kQoFull = 0, kKFull = 1, kKEmpty = 3, kSFull = 5, kDsFull = 6, kQDon
 __global__ void __launch_bounds__(kThreads, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-              const Params p) {
+              const __grid_constant__ CUtensorMap tmDQ, const Params p) {
   static_assert(kQSmem + 256 <= 232448, "shared memory over the limit");
   const Geometry g = geometry(p);
   const int bh = blockIdx.z;
@@ -425,8 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cc = 0; cc < 2; ++cc) {
         const int c = hc * 2 + cc;
         uint32_t sv[32], dv[32];
-        tmem_ld32(tS + c * 32, sv);
-        tmem_ld32(tD + c * 32, dv);
+        tmem_ld32x2(tS + c * 32, sv, tD + c * 32, dv);
         uint32_t gg[16], pp;
         if (valid < 128) {  // the window's last key tile: keys past the window get dS = 0
 #pragma unroll
@@ -444,6 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars[kDsFull]);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQDone], 0, abort_flag)) && !*abort_flag;
+    // dQ is added into global memory by TMA reduce-adds of four 32-column fp32 boxes, staged in
+    // the K stages (free: every MMA is complete); rows past the chunk add zeros.
     if (ok) {
       tc_fence_after();
 #pragma unroll 1
@@ -451,8 +504,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cc = hc * 2 + c2;
         uint32_t a[32];
         tmem_ld32(tmem + lane_base + 256 + cc * 32, a);
-        if (row_ok) add_row32(p.dq + row * 128 + cc * 32, a);
+        stage_row32(sm + kQOffK + cc * 16384, r, a, row_ok);
       }
+    }
+    // every compute thread gets here, whatever its waits returned; after an abort nothing is added
+    fence_async_smem();
+    named_bar_sync(1, kCompute);
+    if (tid == 0 && !*abort_flag) {
+      for (int cc = 0; cc < 4; ++cc)
+        tma_reduce_add_3d_chk(42, &tmDQ, sm + kQOffK + cc * 16384, cc * 32, g.q_row0 + q0, bh, 128,
+                              p.N, gridDim.z);
+      bulk_commit_group();
+      bulk_wait_all();
     }
   }
   tc_fence_before();

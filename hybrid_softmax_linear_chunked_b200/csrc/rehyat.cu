@@ -124,6 +124,22 @@ int make_map(CUtensorMap* m, const void* base, int cols, long long rows, long lo
   return REHYAT_OK;
 }
 
+// fp32 [outer][rows][cols] tensor, boxes of 32 columns (128 bytes) by 128 rows, 128-byte swizzle:
+// the target of the backward's TMA reduce-adds.
+int make_map_f32(CUtensorMap* m, const void* base, int cols, long long rows, long long outer) {
+  EncodeTiledFn enc;
+  RH_TRY(get_encoder(&enc));
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 4, (cuuint64_t)cols * 4 * (cuuint64_t)rows};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(REHYAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return REHYAT_OK;
+}
+
 // bf16 [outer][rows][cols] tensor with explicit strides (elements), box {box_cols, box_rows, 1}.
 int make_map_strided(CUtensorMap* m, const void* base, long long cols, long long rows,
                      long long outer, long long row_stride, long long outer_stride, int box_cols,
@@ -1072,11 +1088,14 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
 
   const float sl2 = (float)(1.4426950408889634 / std::sqrt((double)d.D));
   const float isd = (float)(1.0 / std::sqrt((double)d.D));
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mdq, mdk, mdv;
   RH_TRY(make_map(&mq, q, d.D, N, BH));
   RH_TRY(make_map(&mk, k, d.D, N, BH));
   RH_TRY(make_map(&mv, v, d.D, N, BH));
   RH_TRY(make_map(&mo, dout, d.D, N, BH));
+  RH_TRY(make_map_f32(&mdq, dq, d.D, N, BH));
+  RH_TRY(make_map_f32(&mdk, dk, d.D, N, BH));
+  RH_TRY(make_map_f32(&mdv, dv, d.D, N, BH));
   for (int c = 0; c < C; ++c) {
     const int s = c * Tc, e = (s + Tc < T ? s + Tc : T), w = (s - To > 0 ? s - To : 0);
     const long long nq = (long long)(e - s) * L, nw = (long long)(e - w) * L;
@@ -1095,10 +1114,10 @@ int rehyat_backward(rehyat_dims d, rehyat_dtype dt, int T, int L, int Tc, int To
       RH_TRY(cuda_check(cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)rehyat::attn_bwd::kQSmem), "dq attr"));
       kkv<<<dim3((unsigned)((nw + 127) / 128), 1, BH), rehyat::attn_bwd::kThreads,
-            rehyat::attn_bwd::kKSmem, st>>>(mq, mk, mv, mo, bp);
+            rehyat::attn_bwd::kKSmem, st>>>(mq, mk, mv, mo, mdk, mdv, bp);
       RH_TRY(cuda_check(cudaGetLastError(), "dkdv launch"));
       kq<<<dim3((unsigned)((nq + 127) / 128), 1, BH), rehyat::attn_bwd::kThreads,
-           rehyat::attn_bwd::kQSmem, st>>>(mq, mk, mv, mo, bp);
+           rehyat::attn_bwd::kQSmem, st>>>(mq, mk, mv, mo, mdq, bp);
       RH_TRY(cuda_check(cudaGetLastError(), "dq launch"));
     }
     if (w > 0) {
