@@ -4,7 +4,8 @@ REHYAT_ERR_BOUNDS instead of faulting.
 
 * No false positives: the whole-sequence forward, the streaming step on carried frames (two-segment
   windows, a lone last tile split into parts) and the segment calls run through the checking
-  build, match the oracle and leave the error word clear.
+  build, match the oracle and leave the error word clear; so does the backward (its TMA
+  reduce-adds are checked), whose gradients match the normal build's.
 * The check fires: the self test's out-of-range store (into slack the test allocated, so the
   write would stay inside the buffer even without the check) is recorded and skipped.
 The normal library is restored for the tests that follow."""
@@ -64,6 +65,34 @@ def test_forward_and_streaming_pass_the_checks(dev):
                                             f64(inp.v[0, h]), pq, pk, L, w.Tc, w.To)
         check(f64(out[0, h]), want)
         check(f64(stream_out[0, h]), want)
+
+
+def test_backward_passes_the_checks(dev):
+    w = C.Workload("dbg bwd", B=1, H=2, D=128, T=7, frame_h=8, frame_w=10, Tc=3, To=1, P=2,
+                   F=128, G=8, dtype="bf16", seed=29)
+    inp = make_inputs(w)
+    t = [x.to(dev) for x in (inp.q, inp.k, inp.v, inp.Wq, inp.bq, inp.Wk, inp.bk)]
+    kw = dict(P=w.P, frame_tokens=w.frame_tokens, Tc=w.Tc, To=w.To)
+    dout = torch.randn(inp.q.shape, generator=torch.Generator().manual_seed(3)).to(
+        torch.bfloat16).to(dev)
+
+    def grads():
+        out, lse = rb.forward_train(*t, **kw)
+        g = rb.backward(*t, out, lse, dout, **kw)
+        rb.sync_status(dev)  # raises on a failed check
+        return {n: g[n].detach().clone() for n in ("dq", "dk", "dv", "dWq", "dWk")}
+
+    checked = grads()
+    rb.use_library(build.build())
+    try:
+        plain = grads()
+    finally:
+        rb.use_library(build.build(debug_bounds=True))
+    for n, x in checked.items():
+        y = plain[n]
+        # same kernels and arithmetic; the split-K GEMMs add in a varying order
+        assert torch.isfinite(x).all(), n
+        assert float((x - y).norm() / y.norm()) <= 1e-5, n
 
 
 def test_out_of_range_store_is_caught(dev):
