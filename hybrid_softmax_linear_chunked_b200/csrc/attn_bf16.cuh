@@ -500,10 +500,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(rr[i]);
 #pragma unroll
-          for (int i = 8; i < kBN; i += 16)
+          for (int i = 8; i + 16 <= kBN; i += 16)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               m8[e] = max3(m8[e], __uint_as_float(rr[i + e]), __uint_as_float(rr[i + 8 + e]));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], __uint_as_float(rr[kBN - 8 + e]));
           mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         }
         const float m_tile = mx * sl2;
