@@ -144,6 +144,86 @@ def read_traffic():
     return None
 
 
+# ---------------------------------------------------------------------------------------------
+# Launch counts: the library kernels each call enqueues, following the library's own decisions
+# (which kernels a call needs, and when a chunk's lone last query tile is cut into parts)
+# ---------------------------------------------------------------------------------------------
+
+def _tiles(rows: int) -> int:
+    return -(-rows // 128)
+
+
+def lone_parts(L: int, Tc: int, To: int, frames_before: int, T: int, n_chunks: int) -> int:
+    """Parts a whole-sequence or segment attention launch cuts its chunks' lone last query tiles
+    into (1: no chunk has an odd tile count): up to 4, at most the fewest key tiles of a window
+    that has one."""
+    min_key = None
+    for c in range(n_chunks):
+        gs = frames_before + c * Tc
+        ge = min(gs + Tc, frames_before + T)
+        if _tiles((ge - gs) * L) % 2:
+            k = _tiles((ge - max(0, gs - To)) * L)
+            min_key = k if min_key is None else min(min_key, k)
+    return 1 if min_key is None else max(1, min(4, min_key))
+
+
+def forward_launches(w: C.Workload) -> int:
+    """One whole-sequence bf16 forward (in one call or its three phases): the fold (when a chunk
+    folds), the state scan, phi_q (when a chunk reads a state), the attention, and the lone-tile
+    combine (when a lone tile is cut into parts)."""
+    row_lin = (w.To // w.Tc + 1) * w.Tc * w.frame_tokens
+    parts = lone_parts(w.frame_tokens, w.Tc, w.To, 0, w.T, w.n_chunks)
+    return ((1 if w.n_chunks > 1 else 0) + 1 + (1 if row_lin < w.N else 0) + 1
+            + (1 if parts > 1 else 0))
+
+
+def segment_launches(w: C.Workload, c0: int, c1: int) -> int:
+    """The two context-parallel calls of the chunk range [c0, c1): the fold (when the range folds)
+    and the segment sum; then the scan, phi_q (when a chunk reads a state), the attention and
+    the lone-tile combine."""
+    L = w.frame_tokens
+    n_fold = max(0, min(c1, w.n_chunks - 1) - c0)
+    s0, s1 = c0 * w.Tc, min(c1 * w.Tc, w.T)
+    row_lin = (max(w.To // w.Tc + 1, c0) - c0) * w.Tc * L
+    parts = lone_parts(L, w.Tc, w.To, s0, s1 - s0, c1 - c0)
+    return ((1 if n_fold else 0) + 1 + 1 + (1 if row_lin < (s1 - s0) * L else 0) + 1
+            + (1 if parts > 1 else 0))
+
+
+def backward_launches(w: C.Workload) -> int:
+    """One bf16 backward pass: per chunk the dK/dV and dQ kernels (and, for a chunk with a
+    linear region, a GEMM, the phi_q gradient, a GEMM and the r partial sums); the row
+    statistics, the r reduction and the suffix sums; two GEMMs per group of folded frames; two
+    feature-map backwards (per batch three GEMMs: U, dx, dW; then the feature gradient, the
+    block-diagonal gradient, the column sums and the bias gradient); and the recomputed states
+    and feature maps (two block-diagonal weight preparations, phi_q and phi_k, fold, scan)."""
+    b = w.chunk_bounds()
+    C_ = len(b)
+    lin = sum(1 for (wf, _, _) in b if wf > 0)
+    groups = sum(1 for c in range(C_ - 1) if b[c + 1][0] > b[c][0])
+    return 2 * C_ + 4 * lin + 3 + 2 * groups + 2 * (3 * w.B + 4) + 6
+
+
+def stream_call_launches(L: int, s: int, e: int, ov: int, nxt: int, cap: int) -> int:
+    """One bf16 streaming call on frames [s, e) with overlap ov, next overlap nxt and a carry of
+    cap frames: the S^T copy, phi_q (when the chunk reads a state), the attention, the fold (when
+    frames leave the window), the lone-tile combine (odd query tile count), then the closing
+    state add with the next carry copied in the same launch, or, for a chunk shorter than the
+    carry, the state add (when it folded) and two carry gathers."""
+    o = min(ov, s)
+    wf = s - o
+    fold = max(0, max(0, e - nxt) - wf) > 0
+    q_tiles = _tiles((e - s) * L)
+    key_tiles = _tiles(o * L) + _tiles((e - s) * L)
+    n = 1 + (1 if wf > 0 else 0) + 1 + (1 if fold else 0)
+    n += 1 if (q_tiles % 2 and min(4, key_tiles) > 1) else 0
+    if e - s >= cap:
+        n += 1 if (cap > 0 or fold) else 0
+    else:
+        n += (1 if fold else 0) + 2
+    return n
+
+
 class ClockSampler:
     """nvidia-smi samples (every 200 ms) while the timed region runs."""
 
@@ -521,7 +601,7 @@ def full_runner(w: C.Workload, inp, dev, args) -> _Run:
     r.d2h = out_h.numel() * out_h.element_size()
     r.attn_flops = w.attn_tensor_flops()
     r.step_flops = w.flops(streaming=False)
-    r.launches_per_step = 6  # 2 weight preps, fold, scan, phi_q, attention
+    r.launches_per_step = forward_launches(w)
     bnd = w.chunk_bounds()
     folded = bnd[-1][0] * w.frame_tokens                       # tokens folded (frames < w_{C-1})
     phiq_rows = sum((e - s) * w.frame_tokens for (wf, s, e) in bnd if wf > 0)
@@ -572,14 +652,7 @@ def backward_runner(w: C.Workload, inp, dev, args) -> _Run:
     r.d2h = 3 * q.numel() * 4 + 2 * Wq.numel() * 4 + 2 * w.H * w.F * 4
     r.attn_flops = w.backward_flops()
     r.step_flops = w.backward_flops()
-    C_ = w.n_chunks
-    lin = sum(1 for (wf, _, _) in w.chunk_bounds() if wf > 0)
-    groups = sum(1 for c in range(C_ - 1) if w.chunk_bounds()[c + 1][0] > w.chunk_bounds()[c][0])
-    # per chunk dK/dV + dQ (+ linear: GEMM, phi_q grad, GEMM, r partials), row statistics,
-    # r reduction, suffix, per fold group 2 GEMM, two feature backwards (per batch 3 GEMM: U,
-    # dx, dW; feature grad, block-diagonal grad, column sums, bias grad), plus the recomputed
-    # states/phi_q/phi_k (2 weight preps, 2 feature maps, fold, scan)
-    r.launches_per_step = (2 * C_ + 4 * lin + 3 + 2 * groups + 2 * (3 * w.B + 4) + 6)
+    r.launches_per_step = backward_launches(w)
     r.roofline_kernel = "backward pass (all launches; algorithmic FLOPs / time)"
     r.config = {"pass": "backward"}
     return r
@@ -626,10 +699,7 @@ def context_runner(w: C.Workload, inp, dev, args, rep) -> _Run:
     r.d2h = host_out.numel() * host_out.element_size()
     r.step_flops = w.flops(streaming=False)
     r.attn_flops = w.flops(streaming=False)
-    # per rank: [W_k block-diagonal, fold], segment sum; scan, W_q block-diagonal, [phi_q],
-    # attention
-    n_fold = max(0, min(cp.c1, w.n_chunks - 1) - cp.c0)
-    r.launches_per_step = (2 if n_fold else 0) + 1 + 4
+    r.launches_per_step = segment_launches(w, cp.c0, cp.c1)  # this rank's
     r.roofline_kernel = "context-parallel forward step (whole-sequence FLOPs / step time)"
     r.config = {"parallelism": f"cp{rep.world} (chunk ranges [c0, c1) per rank: "
                                f"{split_chunks(w.n_chunks, rep.world)}; halo point to point, "
@@ -674,7 +744,7 @@ def heads_runner(w: C.Workload, inp, dev, args, rep) -> _Run:
     r.d2h = host_out.numel() * host_out.element_size()
     r.step_flops = w.flops(streaming=False)
     r.attn_flops = w.flops(streaming=False)
-    r.launches_per_step = 6  # 2 weight preps, fold, scan, phi_q, attention (+ the all-gather)
+    r.launches_per_step = forward_launches(w)  # this rank's forward (the all-gather is NCCL's)
     r.roofline_kernel = "head-sharded forward step (whole-problem FLOPs / step time)"
     r.config = {"parallelism": f"heads{rep.world} ((batch, head) units per rank: "
                                f"{hs.ranges}; output slices all-gathered)"}
@@ -748,17 +818,14 @@ def stream_runner(w: C.Workload, inp, dev, args) -> _Run:
     D, F = w.D, w.F
     attn = step_f = 0.0
     launches = 0
+    cap = max(ov_ for _, ov_ in sched)  # the session's carry
     for (wf, s, e, ov, nxt) in bounds:
         nq, nw = (e - s) * L, (e - wf) * L
         attn += 4.0 * nq * nw * D + (2.0 * nq * F * D if wf > 0 else 0.0)
         fold = max(0, max(0, e - nxt) - wf) * L
         step_f += (2.0 * nq * F + (2.0 * nq * D * F / w.G) if wf > 0 else 0.0)
         step_f += fold * (2.0 * F * D + F + 2.0 * D * F / w.G)
-        # S transpose, W_q block-diagonal, attention; [phi_q]; [W_k block-diagonal, fold, state
-        # add]; the carry update is a device copy, or 2 gathers when the chunk is shorter
-        cap = max(ov_ for _, ov_ in sched)
-        launches += (3 + (1 if wf > 0 else 0) + (3 if fold > 0 else 0)
-                     + (2 if 0 < e - s < cap else 0))
+        launches += stream_call_launches(L, s, e, ov, nxt, cap)
     r.attn_flops = attn * w.B * w.H
     r.step_flops = (attn + step_f) * w.B * w.H
     r.step, r.e2e_step = step, e2e_step
