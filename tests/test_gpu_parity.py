@@ -359,7 +359,7 @@ def test_full_size_streaming_session_20s(dev):
 
 
 # ------------------------------------------------------------------------------------------
-# argument errors reported through the C ABI on a GPU machine
+# argument errors reported through the C ABI with a GPU present
 # ------------------------------------------------------------------------------------------
 
 def test_errors_reported(dev):
